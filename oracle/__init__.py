@@ -1,0 +1,195 @@
+"""CPU fp64 oracle for streaming sparse decode attention -- TEST INFRASTRUCTURE.
+
+Only tests/, the smoke check in __graft_entry__ and the CPU-baseline leg of
+bench.py may import this package.  The library never does: it has no CPU
+fallback.  The numeric work lives in oracle.c (plain C, fp64, OpenMP over
+independent units); this module marshals numpy arrays and builds the key sets
+each option attends, following the pages:
+
+* full traversal           -- every token of the sequence
+* ART traversal            -- block 0 first, then the caller's order
+                              ("ART" 2.4: attention sinks, orthogonal order)
+* sink + recent window     -- tokens [0, sink) U [L - recent, L)
+                              ("Flux Attention" 2: sparse layers keep minimal KV;
+                              "Pulsar Attention" Phase 1: 64-token sink prefix)
+* selected clusters        -- the union of the chosen clusters' key ranges
+                              ("Squeezed Attention" Q2, steps 2-3)
+* causal query chunk       -- chunk token t sees the context and chunk keys 0..t
+* shard merge              -- "Pulsar Attention" Phase 2
+
+Parity pins for every function are in tests/test_oracle_pins.py.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import _build
+
+_LIB = None
+_p = ctypes.c_void_p
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(_build.SO) or os.path.getmtime(_build.SO) < os.path.getmtime(
+                os.path.join(_build.HERE, "oracle.c")):
+            _build.build()
+        L = ctypes.CDLL(_build.SO)
+        i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+        L.orc_attend.argtypes = [i64, i32, i32, _p, _p, _p, i64, _p, _p, i64, dbl, _p, _p]
+        L.orc_art_metrics.argtypes = [_p, _p, i32, _p, _p]
+        L.orc_art_stop.argtypes = [_p, i32, i32, dbl, dbl, i32, _p]
+        L.orc_art_stop.restype = i32
+        L.orc_art.argtypes = [i64, i32, i32, _p, _p, _p, i64, _p, i32, _p, _p, i64, dbl, dbl, dbl,
+                              i32, i32, _p, _p, _p, _p, _p]
+        L.orc_select.argtypes = [i64, i32, i32, _p, _p, i32, i32, _p, _p]
+        L.orc_merge.argtypes = [i32, i64, i32, _p, _p, _p, _p]
+        _LIB = L
+    return _LIB
+
+
+def _u16(a):
+    return np.ascontiguousarray(a, dtype=np.uint16)
+
+
+# --------------------------------------------------------------------------- key sets
+
+def keys_full(L):
+    return np.arange(L, dtype=np.int64)
+
+
+def keys_window(L, sink, recent):
+    """Tokens [0, sink) U [L - recent, L), as one sorted set (overlap counted once)."""
+    s = set(range(min(sink, L)))
+    s.update(range(max(0, L - recent), L))
+    return np.array(sorted(s), dtype=np.int64)
+
+
+def keys_segments(starts, ends):
+    """Union of token ranges [starts[i], ends[i])."""
+    s = set()
+    for a, b in zip(starts, ends):
+        s.update(range(int(a), int(b)))
+    return np.array(sorted(s), dtype=np.int64)
+
+
+def keys_chunk(L_ctx, t):
+    """Chunk token t (0-based) sees context keys [0, L_ctx) and chunk keys 0..t."""
+    return np.arange(L_ctx + t + 1, dtype=np.int64)
+
+
+def art_traversal(nb, order=None):
+    """ART traversal: block 0 first ("ART" 2.4), then `order` without block 0.
+
+    order=None means recency-first: nb-1, nb-2, ..., 1."""
+    if order is None:
+        order = list(range(nb - 1, -1, -1))
+    return np.array([0] + [int(j) for j in order if int(j) != 0], dtype=np.int32)
+
+
+# --------------------------------------------------------------------------- numeric entry points
+
+def attend(q, K, V, idx, scale):
+    """Plain softmax attention.  q [U][nq][d] bf16 bits; K, V [U][Lk][d];
+    idx: list (per unit) of lists (per query row) of key index arrays.
+    Returns O [U][nq][d], lse [U][nq] (fp64)."""
+    q, K, V = _u16(q), _u16(K), _u16(V)
+    U, nq, d = q.shape
+    Lk = K.shape[1]
+    stride = max(1, max(len(r) for u in idx for r in u))
+    I = np.zeros((U, nq, stride), dtype=np.int64)
+    M = np.zeros((U, nq), dtype=np.int64)
+    for u in range(U):
+        for r in range(nq):
+            n = len(idx[u][r])
+            I[u, r, :n] = idx[u][r]
+            M[u, r] = n
+    O = np.empty((U, nq, d), dtype=np.float64)
+    lse = np.empty((U, nq), dtype=np.float64)
+    lib().orc_attend(U, nq, d, _ptr(q), _ptr(K), _ptr(V), Lk, _ptr(I), _ptr(M), stride, scale,
+                     _ptr(O), _ptr(lse))
+    return O, lse
+
+
+def art_metrics(x_prev, x):
+    a = np.ascontiguousarray(x_prev, dtype=np.float64)
+    b = np.ascontiguousarray(x, dtype=np.float64)
+    ds, dc = ctypes.c_double(), ctypes.c_double()
+    lib().orc_art_metrics(_ptr(a), _ptr(b), a.size, ctypes.byref(ds), ctypes.byref(dc))
+    return ds.value, dc.value
+
+
+def art_stop(x, tau, phi, patience):
+    """Stopping rule on a probe trajectory x [T][n] -> (blocks consumed, min margin)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    mg = ctypes.c_double()
+    c = lib().orc_art_stop(_ptr(x), x.shape[0], x.shape[1], tau, phi, patience, ctypes.byref(mg))
+    return c, mg.value
+
+
+def art(q, K, V, Ls, bs, blocks, scale, tau, phi, patience, n_probe=8, forced=None):
+    """Sequential ART per query head.  q [U][G][d]; K, V [U][Lk][d]; Ls [U];
+    blocks: list (per unit) of traversal arrays.  forced: None or int [U][G].
+    Returns O [U][G][d], lse [U][G], consumed [U][G], margin [U][G]."""
+    q, K, V = _u16(q), _u16(K), _u16(V)
+    U, G, d = q.shape
+    Lk = K.shape[1]
+    stride = max(1, max(len(b) for b in blocks))
+    Bl = np.zeros((U, stride), dtype=np.int32)
+    nb = np.zeros(U, dtype=np.int32)
+    for u in range(U):
+        Bl[u, :len(blocks[u])] = blocks[u]
+        nb[u] = len(blocks[u])
+    Ls = np.ascontiguousarray(Ls, dtype=np.int64)
+    fo = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
+    O = np.empty((U, G, d))
+    lse = np.empty((U, G))
+    cons = np.empty((U, G), dtype=np.int32)
+    mg = np.empty((U, G))
+    lib().orc_art(U, G, d, _ptr(q), _ptr(K), _ptr(V), Lk, _ptr(Ls), bs, _ptr(Bl), _ptr(nb), stride,
+                  scale, tau, phi, patience, n_probe, _ptr(fo), _ptr(O), _ptr(lse), _ptr(cons), _ptr(mg))
+    return O, lse, cons, mg
+
+
+def select(q, cent, k):
+    """Centroid top-k per unit.  q [U][G][d]; cent [U][C][d].  Returns ids [U][k]
+    (ascending) and all scores [U][C] (fp64)."""
+    q, cent = _u16(q), _u16(cent)
+    U, G, d = q.shape
+    C = cent.shape[1]
+    ids = np.empty((U, k), dtype=np.int32)
+    sc = np.empty((U, C))
+    lib().orc_select(U, G, d, _ptr(q), _ptr(cent), C, k, _ptr(ids), _ptr(sc))
+    return ids, sc
+
+
+def merge(o_parts, lse_parts):
+    """Exact LSE merge.  o_parts [S][N][d], lse_parts [S][N] -> O [N][d], lse [N]."""
+    o = np.ascontiguousarray(o_parts, dtype=np.float64)
+    l = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    S, N, d = o.shape
+    out = np.empty((N, d))
+    lse = np.empty(N)
+    lib().orc_merge(S, N, d, _ptr(o), _ptr(l), _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def topk_boundary_gap(scores, k):
+    """Relative gap between the k-th and (k+1)-th best score of each unit
+    (ranking by score desc, index asc); +inf when k >= C."""
+    out = []
+    for s in np.atleast_2d(scores):
+        C = s.shape[0]
+        if k >= C:
+            out.append(np.inf)
+            continue
+        order = sorted(range(C), key=lambda i: (-s[i], i))
+        a, b = s[order[k - 1]], s[order[k]]
+        out.append(abs(a - b) / max(abs(a), 1e-300))
+    return np.array(out)
