@@ -1,0 +1,190 @@
+/*
+ * sparsekv.h -- C ABI of libsparsekv.so: streaming, block-wise decode
+ * attention of a few query tokens over a long paged bf16 KV cache, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute (sources are the pages this library implements):
+ *
+ *  attn_decode      Softmax attention of each query head over a set of cached
+ *                   keys, accumulated 64-token block by block in an online
+ *                   softmax state (running max m, sum l, output O), the
+ *                   tile-streaming form of "ART (Attention Run-time
+ *                   Termination)" section 2.1.  Options:
+ *                   - a caller-given traversal order ("ART" 2.4, orthogonal
+ *                     ordering layer; full traversal is order-invariant);
+ *                   - ART run-time termination ("ART" 2.2 dual threshold,
+ *                     2.3 patience, 2.4 block 0 always evaluated first);
+ *                   - a sink + recent window, the minimal KV of a sparse layer
+ *                     under per-layer hard routing ("Flux Attention" section 2,
+ *                     "Efficient Deployment"; 64-token sink as in "Pulsar
+ *                     Attention" Phase 1);
+ *                   - an explicit list of token segments, e.g. the key ranges of
+ *                     selected clusters ("Squeezed Attention", Q2 step 3);
+ *                   - a key token range [kv_begin, kv_end), one shard of a
+ *                     context split across hosts ("Pulsar Attention" Phase 2).
+ *  attn_select_centroids
+ *                   Query-centroid comparison and top-k cluster choice
+ *                   ("Squeezed Attention", Q2 step 2).
+ *  attn_merge_lse   Exact merge of per-shard attention partials by their
+ *                   log-sum-exp ("Pulsar Attention" Phase 2, online softmax
+ *                   merge).
+ *
+ * Conventions (all calls):
+ *  - The caller owns and allocates every buffer; the library never allocates
+ *    or frees memory.  All pointers below are DEVICE pointers unless stated.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Arguments are validated on the host before any launch; a
+ *    non-SKV_OK return means nothing was launched (except SKV_ECUDA, which
+ *    reports a launch error).
+ *  - No C++ exception or process exit crosses this boundary.
+ *  - Problems only the device can see (a page index out of range, a sequence
+ *    length above max_seq_len, a traversal entry out of range, a bounded wait
+ *    that expired) are OR-ed into *status_word as SKV_DEV_* bits, when
+ *    status_word is non-NULL; the affected rows are computed as if the bad
+ *    entry were absent.  The caller reads the word back after synchronising.
+ *  - Supported shapes: head_dim 128, block_size 64, q_heads / kv_heads in
+ *    {1, 2, 4, 8}, q_tokens == 1.  Other values return SKV_EUNSUPPORTED.
+ *  - Alignment: q, out, k_pool and v_pool 16-byte aligned.
+ */
+#ifndef SPARSEKV_H
+#define SPARSEKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SKV_API __attribute__((visibility("default")))
+#else
+#define SKV_API
+#endif
+
+typedef struct CUstream_st* skv_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  SKV_OK = 0,
+  SKV_EINVAL = 1,       /* a bad argument (NULL pointer, size, alignment, threshold) */
+  SKV_EUNSUPPORTED = 2, /* valid but not implemented (shape, option combination) */
+  SKV_ECUDA = 3,        /* a CUDA runtime call failed (launch, attribute) */
+  SKV_ETIMEOUT = 4,     /* reserved for callers mapping SKV_DEV_TIMEOUT */
+  SKV_EWORKSPACE = 5    /* workspace NULL or smaller than *_workspace_size */
+} skv_status;
+
+/* Bits OR-ed into *status_word by the device. */
+#define SKV_DEV_TIMEOUT 0x1u     /* a bounded wait inside a kernel expired */
+#define SKV_DEV_BAD_PAGE 0x2u    /* block_table entry < 0 or >= num_pages */
+#define SKV_DEV_BAD_SEQLEN 0x4u  /* seq_lens[b] < 0 or > max_seq_len */
+#define SKV_DEV_BAD_ORDER 0x8u   /* order entry outside [0, ceil(seq_len/64)) */
+#define SKV_DEV_BAD_SEGMENT 0x10u /* segment with start > end */
+
+/* ART run-time termination ("ART" 2.2-2.4).  Per query head, after each
+ * consumed block t the probe x_t = first 8 dims of the normalised partial
+ * output O_t / l_t is formed; for t >= 1
+ *     d_scale = | ||x_t|| - ||x_{t-1}|| | / ||x_{t-1}||
+ *     d_dir   = 1 - cos(x_t, x_{t-1})
+ * and the test passes when d_scale < tau AND d_dir < phi (strict).  The head
+ * stops after `patience` consecutive passes; its output is the attention over
+ * the blocks consumed so far.  Zero probes: ||x_{t-1}|| = 0 gives d_scale = 0
+ * if ||x_t|| = 0 else +inf; a zero vector gives d_dir = 0 if both are zero,
+ * else 1.  tau = phi = 0 never stops (full attention).  Block 0 is always
+ * consumed first.  Key loads of a KV group stop once all of its query heads
+ * have stopped; up to (pipeline depth - 1) further blocks may already be in
+ * flight and are discarded. */
+typedef struct {
+  int enable;   /* 0 = off */
+  float tau;    /* >= 0, scale-change threshold */
+  float phi;    /* >= 0, direction-change threshold */
+  int patience; /* >= 1 consecutive passing blocks */
+} skv_art;
+
+/* Sink + recent window ("Flux Attention" 2, sparse layers keep minimal KV):
+ * attend tokens [0, sink_tokens) U [seq_len - recent_tokens, seq_len), the
+ * overlap counted once.  {0, 0} = off. */
+typedef struct {
+  int sink_tokens;
+  int recent_tokens;
+} skv_window;
+
+typedef struct {
+  const void* q;              /* bf16 [batch][q_tokens][q_heads][head_dim] */
+  const void* k_pool;         /* bf16 [num_pages][kv_heads][block_size][head_dim] */
+  const void* v_pool;         /* bf16, same layout as k_pool */
+  const int32_t* block_table; /* [batch][max_blocks]: logical block j of sequence b
+                                 lives in page block_table[b*max_blocks + j] */
+  const int32_t* seq_lens;    /* [batch] tokens per sequence, 0 <= seq_len <= max_seq_len */
+  const int32_t* order;       /* NULL, or [batch][kv_heads][order_len] logical block ids:
+                                 the traversal order.  NULL means natural order
+                                 0..nb-1, or with ART recency-first nb-1..1 after
+                                 block 0.  With ART, block 0 is visited first and
+                                 skipped where it appears in `order`.  Entries are
+                                 not deduplicated. */
+  int order_len;
+  const int32_t* seg_start;   /* NULL, or [batch][kv_heads][n_seg] token ranges */
+  const int32_t* seg_end;     /*   [seg_start, seg_end) clipped to [0, seq_len) */
+  int n_seg;
+  int batch, q_tokens, q_heads, kv_heads, head_dim, block_size;
+  int max_blocks;   /* row stride of block_table */
+  int num_pages;    /* pages in each pool */
+  int max_seq_len;  /* host-side upper bound on seq_lens, used for the launch plan */
+  int kv_begin, kv_end; /* if kv_end > 0: attend only tokens in [kv_begin, kv_end) */
+  float scale;      /* softmax scale, e.g. 1/sqrt(head_dim) */
+  skv_art art;
+  skv_window window;
+  float* out;               /* fp32 [batch][q_tokens][q_heads][head_dim] */
+  float* lse;               /* fp32 [batch][q_tokens][q_heads], natural log of sum exp(scale q.k);
+                               -inf (with out = 0) when no key is attended */
+  int32_t* blocks_consumed; /* NULL or int32 [batch][q_heads]: KV tiles folded per head */
+  uint32_t* status_word;    /* NULL or one device uint32, SKV_DEV_* bits OR-ed in */
+  void* workspace;          /* device scratch of skv_decode_workspace_size() bytes */
+  size_t workspace_bytes;
+} skv_decode_args;
+
+/* Bytes of device workspace attn_decode needs for these arguments (split-KV
+ * partials); 0 if none.  Depends only on host-side fields. */
+SKV_API size_t skv_decode_workspace_size(const skv_decode_args* args);
+
+/* Decode attention, see above.  Option combinations: at most one of
+ * {order, window, seg_start/seg_end, kv range}; ART only with natural or
+ * `order` traversal. */
+SKV_API skv_status attn_decode(const skv_decode_args* args, skv_stream_t stream);
+
+/* Centroid selection ("Squeezed Attention" Q2 step 2) for each KV group
+ * (b, kvh): score_c = (sum over the group's q_heads/kv_heads query heads of
+ * q_h) . centroid_c, c in [0, n_clusters); keep the `topk` largest, ties to the
+ * lower index; write the kept ids in ascending order and their key ranges
+ *   seg_start[i] = cluster_off[id_i], seg_end[i] = cluster_off[id_i + 1].
+ *  q           bf16 [batch][q_heads][head_dim] (one query token)
+ *  centroids   bf16 [batch][kv_heads][n_clusters][head_dim]
+ *  cluster_off int32 [batch][kv_heads][n_clusters + 1], cluster c holds the
+ *              cache tokens [cluster_off[c], cluster_off[c+1])
+ *  sel_ids, seg_start, seg_end  int32 [batch][kv_heads][topk] (outputs)
+ * Supported: head_dim 128, 1 <= topk <= n_clusters <= 4096. */
+SKV_API skv_status attn_select_centroids(const void* q, const void* centroids, const int32_t* cluster_off,
+                                 int batch, int q_heads, int kv_heads, int head_dim,
+                                 int n_clusters, int topk, int32_t* sel_ids, int32_t* seg_start,
+                                 int32_t* seg_end, skv_stream_t stream);
+
+/* Exact LSE merge ("Pulsar Attention" Phase 2) of n_parts partials of n_rows
+ * rows each:
+ *   M = max_s lse_s,  w_s = exp(lse_s - M),
+ *   out = sum_s w_s o_s / sum_s w_s,  lse = M + log sum_s w_s.
+ * A partial with lse = -inf has weight 0; if all are -inf, out = 0 and
+ * lse = -inf.
+ *  o_parts   fp32 [n_parts][n_rows][head_dim] (each row normalised)
+ *  lse_parts fp32 [n_parts][n_rows]
+ *  out       fp32 [n_rows][head_dim], lse fp32 [n_rows]
+ * head_dim must be a multiple of 4 and <= 512; 16-byte aligned o_parts/out. */
+SKV_API skv_status attn_merge_lse(const float* o_parts, const float* lse_parts, int n_parts, int n_rows,
+                          int head_dim, float* out, float* lse, skv_stream_t stream);
+
+/* Static description of a status code. */
+SKV_API const char* skv_strerror(skv_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSEKV_H */

@@ -39,6 +39,7 @@ class Workload:
     shards: int = 1
     chunk: int = 0              # number of chunk tokens appended after the context
     n_layers: int = 1
+    softmax_scale: Optional[float] = None  # default 1/sqrt(d)
     extra: dict = field(default_factory=dict)
 
     @property
@@ -47,6 +48,8 @@ class Workload:
 
     @property
     def scale(self):
+        if self.softmax_scale is not None:
+            return float(self.softmax_scale)
         return 1.0 / float(np.sqrt(self.d))
 
     def seq_len(self, b):

@@ -1,0 +1,220 @@
+// api.cu -- the C ABI of libsparsekv.so: host-side validation, the launch
+// plan (split count, workspace carve-up) and the launches.  No exception or
+// exit crosses this boundary; every path returns an skv_status.
+#include <math.h>
+#include <algorithm>
+#include <stdint.h>
+
+#include <cuda_runtime.h>
+
+#include "../../include/sparsekv.h"
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace skv {
+namespace {
+
+struct Plan {
+  int G = 0;
+  int mode = TRAV_NATURAL;
+  bool art = false;
+  int splits = 1;
+  size_t ws_bytes = 0;
+};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Split count for traversals of up to n_tiles tiles per group: minimise
+// (waves x tiles per CTA) plus a per-wave fill cost, one resident CTA per SM.
+int choose_splits(long long groups, int n_tiles) {
+  if (n_tiles <= 1 || groups <= 0) return 1;
+  const int sms = num_sms();
+  const int s_max = std::max(1, std::min(64, n_tiles / 4));
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= s_max; ++s) {
+    const long long waves = (groups * s + sms - 1) / sms;
+    const long long cost = waves * (cdiv(n_tiles, s) + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+skv_status make_plan(const skv_decode_args* a, Plan* pl) {
+  if (!a) return SKV_EINVAL;
+  if (!a->q || !a->k_pool || !a->v_pool || !a->block_table || !a->seq_lens || !a->out || !a->lse)
+    return SKV_EINVAL;
+  if (a->batch < 1 || a->q_tokens < 1 || a->q_heads < 1 || a->kv_heads < 1) return SKV_EINVAL;
+  if (a->q_heads % a->kv_heads != 0) return SKV_EINVAL;
+  if (a->max_seq_len < 0 || a->num_pages < 1 || a->max_blocks < 0) return SKV_EINVAL;
+  if (a->head_dim != kHeadDim || a->block_size != kBlock) return SKV_EUNSUPPORTED;
+  if ((long long)a->max_blocks * kBlock < (long long)a->max_seq_len) return SKV_EINVAL;
+  if (!aligned16(a->q) || !aligned16(a->out) || !aligned16(a->k_pool) || !aligned16(a->v_pool))
+    return SKV_EINVAL;
+  if (!isfinite(a->scale)) return SKV_EINVAL;
+  const int G = a->q_heads / a->kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SKV_EUNSUPPORTED;
+  if (a->q_tokens != 1) return SKV_EUNSUPPORTED;
+
+  const bool has_order = a->order != nullptr;
+  const bool has_seg = a->seg_start != nullptr || a->seg_end != nullptr;
+  const bool has_win = a->window.sink_tokens != 0 || a->window.recent_tokens != 0;
+  const bool has_range = a->kv_end > 0 || a->kv_begin != 0;
+  if ((int)has_order + (int)has_seg + (int)has_win + (int)has_range > 1) return SKV_EUNSUPPORTED;
+  if (has_order && a->order_len < 0) return SKV_EINVAL;
+  if (has_seg && (!a->seg_start || !a->seg_end || a->n_seg < 0)) return SKV_EINVAL;
+  if (has_win && (a->window.sink_tokens < 0 || a->window.recent_tokens < 0)) return SKV_EINVAL;
+  if (has_range && (a->kv_begin < 0 || a->kv_end < a->kv_begin)) return SKV_EINVAL;
+  if (a->art.enable) {
+    if (!(a->art.tau >= 0.f) || !(a->art.phi >= 0.f) || a->art.patience < 1) return SKV_EINVAL;
+    if (has_seg || has_win || has_range) return SKV_EUNSUPPORTED;
+  }
+
+  pl->G = G;
+  pl->art = a->art.enable != 0;
+  pl->mode = has_order ? TRAV_ORDER : has_seg ? TRAV_SEGMENTS : has_win ? TRAV_WINDOW : TRAV_NATURAL;
+  pl->splits = 1;
+  pl->ws_bytes = 0;
+  if (!pl->art) {
+    const long long L = a->max_seq_len;
+    int n_tiles = 0;
+    switch (pl->mode) {
+      case TRAV_NATURAL:
+        if (has_range) {
+          const long long e = std::min<long long>(a->kv_end, L);
+          n_tiles = (e > a->kv_begin) ? cdiv(e, kBlock) - a->kv_begin / kBlock : 0;
+        } else {
+          n_tiles = cdiv(L, kBlock);
+        }
+        break;
+      case TRAV_ORDER: n_tiles = a->order_len; break;
+      case TRAV_WINDOW:
+        n_tiles = cdiv(std::min<long long>(a->window.sink_tokens, L), kBlock) +
+                  cdiv(std::min<long long>(a->window.recent_tokens, L), kBlock) + 1;
+        break;
+      default: n_tiles = a->n_seg; break;
+    }
+    pl->splits = choose_splits((long long)a->batch * a->kv_heads, n_tiles);
+    if (pl->splits > 1) {
+      const size_t rows = (size_t)a->batch * a->q_heads;
+      pl->ws_bytes = (size_t)pl->splits * rows * (kHeadDim + 1) * sizeof(float);
+    }
+  }
+  return SKV_OK;
+}
+
+}  // namespace
+}  // namespace skv
+
+using namespace skv;
+
+extern "C" {
+
+size_t skv_decode_workspace_size(const skv_decode_args* args) {
+  Plan pl;
+  if (make_plan(args, &pl) != SKV_OK) return 0;
+  return pl.ws_bytes;
+}
+
+skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
+  Plan pl;
+  const skv_status st = make_plan(a, &pl);
+  if (st != SKV_OK) return st;
+  if (pl.ws_bytes > 0 &&
+      (!a->workspace || a->workspace_bytes < pl.ws_bytes || !aligned16(a->workspace)))
+    return SKV_EWORKSPACE;
+
+  DecodeParams p{};
+  p.q = static_cast<const uint16_t*>(a->q);
+  p.k_pool = static_cast<const uint16_t*>(a->k_pool);
+  p.v_pool = static_cast<const uint16_t*>(a->v_pool);
+  p.block_table = a->block_table;
+  p.seq_lens = a->seq_lens;
+  p.order = a->order;
+  p.order_len = a->order_len;
+  p.seg_start = a->seg_start;
+  p.seg_end = a->seg_end;
+  p.n_seg = a->n_seg;
+  p.B = a->batch;
+  p.Hq = a->q_heads;
+  p.Hkv = a->kv_heads;
+  p.max_blocks = a->max_blocks;
+  p.num_pages = a->num_pages;
+  p.max_seq_len = a->max_seq_len;
+  p.range_begin = a->kv_begin;
+  p.range_end = a->kv_end;
+  p.sink = a->window.sink_tokens;
+  p.recent = a->window.recent_tokens;
+  p.mode = pl.mode;
+  p.n_splits = pl.splits;
+  p.qscale = a->scale * 1.4426950408889634f;
+  p.tau = a->art.tau;
+  p.phi = a->art.phi;
+  p.patience = a->art.patience;
+  p.out = a->out;
+  p.lse = a->lse;
+  p.blocks_consumed = a->blocks_consumed;
+  p.status = a->status_word;
+  const size_t rows = (size_t)a->batch * a->q_heads;
+  if (pl.splits > 1) {
+    p.ws_o = static_cast<float*>(a->workspace);
+    p.ws_lse = p.ws_o + (size_t)pl.splits * rows * kHeadDim;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (a->blocks_consumed && !pl.art) {
+    if (cudaMemsetAsync(a->blocks_consumed, 0, rows * sizeof(int32_t), s) != cudaSuccess)
+      return SKV_ECUDA;
+  }
+  if (launch_decode(p, pl.G, pl.art, s) != 0) return SKV_ECUDA;
+  if (pl.splits > 1) {
+    if (launch_merge(p.ws_o, p.ws_lse, pl.splits, (int)rows, kHeadDim, a->out, a->lse, s) != 0)
+      return SKV_ECUDA;
+  }
+  return SKV_OK;
+}
+
+skv_status attn_select_centroids(const void* q, const void* centroids, const int32_t* cluster_off,
+                                 int batch, int q_heads, int kv_heads, int head_dim, int n_clusters,
+                                 int topk, int32_t* sel_ids, int32_t* seg_start, int32_t* seg_end,
+                                 skv_stream_t stream) {
+  if (!q || !centroids || !cluster_off || !sel_ids || !seg_start || !seg_end) return SKV_EINVAL;
+  if (batch < 1 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads != 0) return SKV_EINVAL;
+  if (n_clusters < 1 || topk < 1 || topk > n_clusters) return SKV_EINVAL;
+  if (head_dim != kHeadDim || n_clusters > 4096) return SKV_EUNSUPPORTED;
+  if (!aligned16(q) || !aligned16(centroids)) return SKV_EINVAL;
+  if (launch_select(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(centroids),
+                    cluster_off, batch, q_heads, kv_heads, n_clusters, topk, sel_ids, seg_start,
+                    seg_end, reinterpret_cast<cudaStream_t>(stream)) != 0)
+    return SKV_ECUDA;
+  return SKV_OK;
+}
+
+skv_status attn_merge_lse(const float* o_parts, const float* lse_parts, int n_parts, int n_rows,
+                          int head_dim, float* out, float* lse, skv_stream_t stream) {
+  if (!o_parts || !lse_parts || !out || !lse) return SKV_EINVAL;
+  if (n_parts < 1 || n_rows < 0 || head_dim < 4 || head_dim % 4 != 0 || head_dim > 512)
+    return SKV_EINVAL;
+  if (!aligned16(o_parts) || !aligned16(out)) return SKV_EINVAL;
+  if (launch_merge(o_parts, lse_parts, n_parts, n_rows, head_dim, out, lse,
+                   reinterpret_cast<cudaStream_t>(stream)) != 0)
+    return SKV_ECUDA;
+  return SKV_OK;
+}
+
+const char* skv_strerror(skv_status s) {
+  switch (s) {
+    case SKV_OK: return "ok";
+    case SKV_EINVAL: return "invalid argument";
+    case SKV_EUNSUPPORTED: return "unsupported shape or option combination";
+    case SKV_ECUDA: return "CUDA runtime error";
+    case SKV_ETIMEOUT: return "device wait timed out";
+    case SKV_EWORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

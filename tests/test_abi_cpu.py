@@ -1,0 +1,119 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_kv_b200 as skv
+from sparse_kv_b200 import DecodeArgs, _Art, _Window, _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x7F0000001000  # aligned, never dereferenced: every case fails validation first
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "sparsekv.h")).read()
+    return re.findall(r"SKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["attn_decode", "attn_select_centroids", "attn_merge_lse", "skv_decode_workspace_size",
+              "skv_strerror"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = skv.lib()
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    out = os.popen(f"nm -D --defined-only {_build.SO}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(declared_functions()) <= exported
+    # nothing else leaks: only the declared C symbols are exported as functions
+    assert not [s for s in exported if s.startswith("_Z")]
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(_build, "SO", "/nonexistent/libsparsekv.so")
+    monkeypatch.setattr(skv, "_LIB", None)
+    with pytest.raises(RuntimeError, match="libsparsekv.so not found"):
+        skv.lib()
+
+
+def good_args(**kw):
+    a = DecodeArgs()
+    a.q = a.k_pool = a.v_pool = a.block_table = a.seq_lens = a.out = a.lse = FAKE
+    a.batch, a.q_tokens, a.q_heads, a.kv_heads, a.head_dim, a.block_size = 16, 1, 32, 8, 128, 64
+    a.max_blocks, a.num_pages, a.max_seq_len = 512, 8192, 32768
+    a.scale = 0.088
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def status(a):
+    # a workspace-free configuration fails in validation; others fail at the workspace check
+    return skv.lib().attn_decode(ctypes.byref(a), None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=None), skv.SKV_EINVAL),
+    (dict(out=None), skv.SKV_EINVAL),
+    (dict(seq_lens=None), skv.SKV_EINVAL),
+    (dict(batch=0), skv.SKV_EINVAL),
+    (dict(q_heads=30), skv.SKV_EINVAL),
+    (dict(q_heads=24), skv.SKV_EUNSUPPORTED),      # GQA group of 3
+    (dict(head_dim=64), skv.SKV_EUNSUPPORTED),
+    (dict(block_size=32), skv.SKV_EUNSUPPORTED),
+    (dict(q_tokens=2), skv.SKV_EUNSUPPORTED),
+    (dict(q=FAKE + 8), skv.SKV_EINVAL),            # misaligned
+    (dict(k_pool=FAKE + 4), skv.SKV_EINVAL),
+    (dict(max_blocks=100), skv.SKV_EINVAL),        # table narrower than max_seq_len
+    (dict(scale=float("nan")), skv.SKV_EINVAL),
+    (dict(art=_Art(1, -1.0, 1e-4, 4)), skv.SKV_EINVAL),
+    (dict(art=_Art(1, float("nan"), 1e-4, 4)), skv.SKV_EINVAL),
+    (dict(art=_Art(1, 1e-3, 1e-4, 0)), skv.SKV_EINVAL),
+    (dict(art=_Art(1, 1e-3, 1e-4, 4), window=_Window(64, 4096)), skv.SKV_EUNSUPPORTED),
+    (dict(order=FAKE, order_len=4, window=_Window(64, 4096)), skv.SKV_EUNSUPPORTED),
+    (dict(seg_start=FAKE, n_seg=3), skv.SKV_EINVAL),  # seg_end missing
+    (dict(window=_Window(-1, 4096)), skv.SKV_EINVAL),
+    (dict(kv_begin=10, kv_end=5), skv.SKV_EINVAL),
+    (dict(), skv.SKV_EWORKSPACE),                  # needs split-KV workspace, none given
+])
+def test_decode_rejects_on_host(kw, want):
+    assert status(good_args(**kw)) == want
+
+
+def test_workspace_size_query():
+    L = skv.lib()
+    full = good_args()
+    n = L.skv_decode_workspace_size(ctypes.byref(full))
+    assert n > 0 and n % (16 * 32 * 129 * 4) == 0
+    art = good_args(art=_Art(1, 1e-3, 1e-4, 4))
+    assert L.skv_decode_workspace_size(ctypes.byref(art)) == 0  # ART walks each group in one CTA
+    assert L.skv_decode_workspace_size(ctypes.byref(good_args(head_dim=64))) == 0
+    small = good_args(workspace=FAKE, workspace_bytes=n - 16)
+    assert status(small) == skv.SKV_EWORKSPACE
+
+
+def test_select_and_merge_reject_on_host():
+    L = skv.lib()
+    sel = L.attn_select_centroids
+    assert sel(FAKE, FAKE, FAKE, 8, 32, 8, 128, 1024, 2000, FAKE, FAKE, FAKE, None) == skv.SKV_EINVAL
+    assert sel(FAKE, FAKE, FAKE, 8, 32, 8, 128, 8192, 102, FAKE, FAKE, FAKE, None) == skv.SKV_EUNSUPPORTED
+    assert sel(FAKE, FAKE, FAKE, 8, 32, 8, 64, 1024, 102, FAKE, FAKE, FAKE, None) == skv.SKV_EUNSUPPORTED
+    assert sel(None, FAKE, FAKE, 8, 32, 8, 128, 1024, 102, FAKE, FAKE, FAKE, None) == skv.SKV_EINVAL
+    mer = L.attn_merge_lse
+    assert mer(FAKE, FAKE, 0, 10, 128, FAKE, FAKE, None) == skv.SKV_EINVAL
+    assert mer(FAKE, FAKE, 2, 10, 6, FAKE, FAKE, None) == skv.SKV_EINVAL
+    assert mer(FAKE + 4, FAKE, 2, 10, 128, FAKE, FAKE, None) == skv.SKV_EINVAL
+    assert mer(None, FAKE, 2, 10, 128, FAKE, FAKE, None) == skv.SKV_EINVAL
+
+
+def test_strerror():
+    assert skv.strerror(skv.SKV_OK) == "ok"
+    assert "workspace" in skv.strerror(skv.SKV_EWORKSPACE)
+    assert skv.strerror(99) == "unknown status"

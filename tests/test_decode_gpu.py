@@ -1,0 +1,359 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU fp64 oracle
+on the same seeded inputs."""
+import numpy as np
+import pytest
+
+import oracle
+import skvgen
+from helpers import (check_art, check_close, device_workload, group_inputs, oracle_keys_attend,
+                     run_decode, TOPK_FLAG_GAP)
+
+pytestmark = pytest.mark.gpu
+
+
+def _torch():
+    import torch
+    return torch
+
+
+# ----------------------------------------------------------------------------- generator
+
+def test_device_generator_matches_host_bits():
+    torch = _torch()
+    wl = skvgen.Workload("g", B=3, Hq=8, Hkv=2, L=300, lens=[300, 65, 1], structured=True,
+                         paging="perm", seed=77)
+    dev = device_workload(wl)
+    qh = skvgen.host_q(wl)
+    qd = dev["q"].view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(qd, qh)
+    kp = dev["k_pool"].view(torch.int16).cpu().numpy().view(np.uint16)
+    vp = dev["v_pool"].view(torch.int16).cpu().numpy().view(np.uint16)
+    for b in range(wl.B):
+        for kvh in range(wl.Hkv):
+            K, V = skvgen.host_kv_group(wl, b, kvh, q=qh)
+            for t in range(wl.seq_len(b)):
+                pg = dev["bt_host"][b, t // 64]
+                np.testing.assert_array_equal(kp[pg, kvh, t % 64], K[t])
+                np.testing.assert_array_equal(vp[pg, kvh, t % 64], V[t])
+
+
+def test_device_mixture_matches_host_bits():
+    torch = _torch()
+    wl = skvgen.Workload("m", B=2, Hq=8, Hkv=2, L=1500, mixture=True, c_log2=5, topk=4, seed=78)
+    dev = device_workload(wl)
+    kp = dev["k_pool"].view(torch.int16).cpu().numpy().view(np.uint16)
+    cent = dev["centroids"].view(torch.int16).cpu().numpy().view(np.uint16)
+    off = dev["cluster_off"].cpu().numpy()
+    for b in range(2):
+        for kvh in range(2):
+            K, o, c = skvgen.host_mixture_group(wl, b, kvh)
+            np.testing.assert_array_equal(off[b, kvh], o)
+            np.testing.assert_array_equal(cent[b, kvh], c)
+            for t in range(0, 1500, 7):
+                pg = dev["bt_host"][b, t // 64]
+                np.testing.assert_array_equal(kp[pg, kvh, t % 64], K[t])
+
+
+# ----------------------------------------------------------------------------- full traversal
+
+def _check_all_groups(wl, res, keys_fn, layer=0):
+    O_g, lse_g = res[0], res[1]
+    q = skvgen.host_q(wl, layer)
+    worst = 0.0
+    for b in range(wl.B):
+        for kvh in range(wl.Hkv):
+            O, lse = oracle_keys_attend(wl, b, kvh, keys_fn(b), layer, q)
+            hs = slice(kvh * wl.G, (kvh + 1) * wl.G)
+            worst = max(worst, check_close(O_g[b, hs], lse_g[b, hs], O[0], lse[0], f"group ({b},{kvh})"))
+    return worst
+
+
+def test_cfg1_full_traversal():
+    wl = skvgen.WORKLOADS["cfg1_b1_h8_l4k"]
+    dev = device_workload(wl)
+    res = run_decode(wl, dev)
+    assert res[3] == 0
+    _check_all_groups(wl, res, lambda b: oracle.keys_full(wl.seq_len(b)))
+    assert np.all(res[2] == 64)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_ragged_paged_full_traversal(G):
+    lens = [1, 63, 64, 65, 200, 1000, 0, 4097]
+    wl = skvgen.Workload("r", B=len(lens), Hq=2 * G, Hkv=2, L=max(lens), lens=lens, paging="perm",
+                         seed=100 + G)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev)
+    assert res[3] == 0
+    _check_all_groups(wl, res, lambda b: oracle.keys_full(wl.seq_len(b)))
+    nb = np.array([wl.nb(b) for b in range(wl.B)])
+    np.testing.assert_array_equal(res[2], np.repeat(nb[:, None], wl.Hq, axis=1))
+
+
+def test_caller_order_full_traversal_is_permutation_invariant():
+    torch = _torch()
+    lens = [64 * 37 + 5, 64 * 20]
+    wl = skvgen.Workload("o", B=2, Hq=8, Hkv=2, L=max(lens), lens=lens, paging="perm", seed=5)
+    dev = device_workload(wl)
+    rng = np.random.default_rng(0)
+    n = max(wl.nb(b) for b in range(2))
+    order = np.zeros((2, 2, n), dtype=np.int32)
+    for b in range(2):
+        for h in range(2):
+            nb = wl.nb(b)
+            order[b, h, :nb] = rng.permutation(nb)
+            order[b, h, nb:] = rng.integers(0, nb, n - nb)  # duplicates: attended twice
+    res = run_decode(wl, dev, order=torch.tensor(order, device="cuda"))
+    assert res[3] == 0
+    q = skvgen.host_q(wl)
+    for b in range(2):
+        for kvh in range(2):
+            keys = np.concatenate([np.arange(64 * j, min(64 * j + 64, wl.seq_len(b))) for j in order[b, kvh]])
+            O, lse = oracle_keys_attend(wl, b, kvh, keys, q=q)
+            hs = slice(kvh * 4, kvh * 4 + 4)
+            check_close(res[0][b, hs], res[1][b, hs], O[0], lse[0])
+    # order covering exactly the blocks once equals natural full traversal
+    o2 = np.stack([np.stack([rng.permutation(wl.nb(0))] * 2)] * 1)
+    wl1 = wl.with_(B=1, lens=[lens[0]], L=lens[0])
+    dev1 = device_workload(wl1)
+    a = run_decode(wl1, dev1, order=torch.tensor(o2.astype(np.int32), device="cuda"))
+    bfull = run_decode(wl1, dev1)
+    np.testing.assert_allclose(a[0], bfull[0], atol=2e-5)
+    np.testing.assert_allclose(a[1], bfull[1], rtol=1e-6)
+
+
+@pytest.mark.parametrize("sink,recent", [(64, 4096), (64, 256), (10, 100), (0, 130), (200, 0), (64, 10 ** 6)])
+def test_sink_recent_window(sink, recent):
+    lens = [5000, 300, 64, 129, 1]
+    wl = skvgen.Workload("w", B=len(lens), Hq=8, Hkv=2, L=max(lens), lens=lens, paging="perm", seed=9)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev, window=(sink, recent))
+    assert res[3] == 0
+    _check_all_groups(wl, res, lambda b: oracle.keys_window(wl.seq_len(b), sink, recent))
+
+
+@pytest.mark.parametrize("rng_", [(0, 64), (100, 1000), (1, 4096), (4000, 4100), (3000, 3000)])
+def test_kv_token_range(rng_):
+    lens = [4100, 3500]
+    wl = skvgen.Workload("k", B=2, Hq=8, Hkv=2, L=max(lens), lens=lens, paging="perm", seed=19)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev, kv_range=rng_)
+    assert res[3] == 0
+    a, e = rng_
+    _check_all_groups(wl, res, lambda b: np.arange(a, min(e, wl.seq_len(b))))
+
+
+def test_token_segments_unaligned():
+    torch = _torch()
+    lens = [3000, 2000]
+    wl = skvgen.Workload("s", B=2, Hq=8, Hkv=2, L=max(lens), lens=lens, paging="perm", seed=29)
+    dev = device_workload(wl)
+    rng = np.random.default_rng(3)
+    n_seg = 9
+    ss = np.zeros((2, 2, n_seg), dtype=np.int32)
+    se = np.zeros((2, 2, n_seg), dtype=np.int32)
+    for b in range(2):
+        for h in range(2):
+            cuts = np.sort(rng.choice(np.arange(1, lens[b]), 2 * n_seg, replace=False))
+            ss[b, h], se[b, h] = cuts[0::2], cuts[1::2]
+            se[b, h, -1] = lens[b] + 50  # clipped to seq_len
+            ss[b, h, 0] = se[b, h, 0]    # an empty segment
+    res = run_decode(wl, dev, segments=(torch.tensor(ss, device="cuda"), torch.tensor(se, device="cuda")))
+    assert res[3] == 0
+    q = skvgen.host_q(wl)
+    for b in range(2):
+        for kvh in range(2):
+            keys = oracle.keys_segments(ss[b, kvh], np.minimum(se[b, kvh], lens[b]))
+            O, lse = oracle_keys_attend(wl, b, kvh, keys, q=q)
+            hs = slice(kvh * 4, kvh * 4 + 4)
+            check_close(res[0][b, hs], res[1][b, hs], O[0], lse[0])
+
+
+# ----------------------------------------------------------------------------- ART
+
+def test_art_zero_thresholds_is_full_attention():
+    lens = [64 * 30 + 7, 64 * 5]
+    wl = skvgen.Workload("a0", B=2, Hq=8, Hkv=2, L=max(lens), lens=lens, paging="perm", seed=31)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev, art=(0.0, 0.0, 4))
+    assert res[3] == 0
+    _check_all_groups(wl, res, lambda b: oracle.keys_full(wl.seq_len(b)))
+    nb = np.array([wl.nb(b) for b in range(2)])
+    np.testing.assert_array_equal(res[2], np.repeat(nb[:, None], 8, axis=1))
+
+
+@pytest.mark.parametrize("tau,phi,p", [(1e-3, 1e-4, 4), (3e-2, 3e-3, 2), (1e-2, 1e-3, 1)])
+def test_art_structured_small(tau, phi, p):
+    # sink + heavy structure (token 0 key + 6 qhat, 1% heavy + 4 qhat), recency-first
+    lens = [64 * 60, 64 * 33 + 20, 64 * 8]
+    wl = skvgen.Workload("as", B=3, Hq=8, Hkv=2, L=max(lens), lens=lens, structured=True,
+                         paging="perm", seed=41)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev, art=(tau, phi, p))
+    assert res[3] == 0
+    q = skvgen.host_q(wl)
+    flagged = 0
+    for b in range(3):
+        for kvh in range(2):
+            f, _, _ = check_art(wl, res, b, kvh, q=q, tau=tau, phi=phi, patience=p)
+            flagged += f
+    assert flagged <= 2
+
+
+@pytest.mark.parametrize("p", [1, 4])
+def test_art_always_passing_stops_after_one_plus_p_blocks(p):
+    # thresholds no probe change can reach (d_scale < 10, 1 - cos < 2.5): every
+    # test passes, so each head stops after block 0 and p more blocks
+    lens = [64 * 40, 64 * 3 + 1]
+    wl = skvgen.Workload("ap", B=2, Hq=8, Hkv=2, L=max(lens), lens=lens, structured=True,
+                         paging="perm", seed=43, softmax_scale=0.3)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev, art=(10.0, 2.5, p))
+    assert res[3] == 0
+    assert np.all(res[2][0] == 1 + p)
+    assert np.all(res[2][1] == min(1 + p, 4))
+    q = skvgen.host_q(wl)
+    for b in range(2):
+        for kvh in range(2):
+            check_art(wl, res, b, kvh, q=q, tau=10.0, phi=2.5, patience=p)
+
+
+def test_art_with_caller_order_skips_block0_in_list():
+    torch = _torch()
+    wl = skvgen.Workload("ao", B=1, Hq=8, Hkv=2, L=64 * 50, structured=True, seed=47)
+    dev = device_workload(wl)
+    rng = np.random.default_rng(1)
+    order = np.stack([rng.permutation(50) for _ in range(2)])[None].astype(np.int32)
+    res = run_decode(wl, dev, art=(3e-2, 3e-3, 2), order=torch.tensor(order, device="cuda"))
+    q = skvgen.host_q(wl)
+    for kvh in range(2):
+        check_art(wl, res, 0, kvh, order=list(order[0, kvh]), q=q, tau=3e-2, phi=3e-3, patience=2)
+
+
+# ----------------------------------------------------------------------------- device-side errors
+
+def test_bad_page_and_seqlen_are_reported():
+    torch = _torch()
+    wl = skvgen.Workload("e", B=2, Hq=8, Hkv=2, L=640, paging="perm", seed=53)
+    dev = device_workload(wl)
+    bt = dev["block_table"].clone()
+    bt[0, 3] = 10 ** 6
+    dev2 = dict(dev, block_table=bt)
+    res = run_decode(wl, dev2)
+    assert res[3] & 0x2
+    keys = np.concatenate([np.arange(0, 192), np.arange(256, 640)])
+    O, lse = oracle_keys_attend(wl, 0, 1, keys)
+    check_close(res[0][0, 4:8], res[1][0, 4:8], O[0], lse[0])
+    sl = dev["seq_lens"].clone()
+    sl[1] = 10 ** 6
+    res = run_decode(wl, dict(dev, seq_lens=sl))
+    assert res[3] & 0x4
+    assert np.all(np.isneginf(res[1][1])) and np.all(res[0][1] == 0)
+
+
+# ----------------------------------------------------------------------------- merge
+
+def test_merge_lse_matches_oracle():
+    torch = _torch()
+    import sparse_kv_b200 as skv
+    rng = np.random.default_rng(7)
+    S, N, d = 9, 333, 128
+    o = rng.standard_normal((S, N, d)).astype(np.float32)
+    l = (rng.standard_normal((S, N)) * 5).astype(np.float32)
+    l[2, :50] = -np.inf
+    l[:, 7] = -np.inf  # all partials empty
+    out = torch.empty((N, d), device="cuda")
+    lse = torch.empty(N, device="cuda")
+    skv.attn_merge_lse(torch.tensor(o, device="cuda"), torch.tensor(l, device="cuda"), out, lse)
+    Om, lm = oracle.merge(o.astype(np.float64), l.astype(np.float64))
+    got_o, got_l = out.cpu().numpy(), lse.cpu().numpy()
+    assert np.isneginf(got_l[7]) and np.all(got_o[7] == 0)
+    check_close(got_o, got_l, Om, lm)
+
+
+def test_sharded_partials_merge_to_unsharded():
+    torch = _torch()
+    import sparse_kv_b200 as skv
+    wl = skvgen.Workload("sh", B=2, Hq=8, Hkv=2, L=5000, paging="perm", seed=59)
+    dev = device_workload(wl)
+    bounds = [0, 700, 2048, 2049, 4100, 5000]
+    outs, lses = [], []
+    for a, e in zip(bounds[:-1], bounds[1:]):
+        r = run_decode(wl, dev, kv_range=(a, e))
+        outs.append(r[0].reshape(-1, 128))
+        lses.append(r[1].reshape(-1))
+    out = torch.empty((16, 128), device="cuda")
+    lse = torch.empty(16, device="cuda")
+    skv.attn_merge_lse(torch.tensor(np.array(outs), dtype=torch.float32, device="cuda"),
+                       torch.tensor(np.array(lses), dtype=torch.float32, device="cuda"), out, lse)
+    full = run_decode(wl, dev)
+    check_close(out.cpu().numpy(), lse.cpu().numpy(), full[0].reshape(-1, 128), full[1].reshape(-1))
+    _check_all_groups(wl, (out.cpu().numpy().reshape(2, 8, 128), lse.cpu().numpy().reshape(2, 8)),
+                      lambda b: oracle.keys_full(5000))
+
+
+# ----------------------------------------------------------------------------- centroid selection
+
+def _select(wl, dev):
+    torch = _torch()
+    import sparse_kv_b200 as skv
+    shape = (wl.B, wl.Hkv, wl.topk)
+    ids = torch.empty(shape, dtype=torch.int32, device="cuda")
+    ss = torch.empty(shape, dtype=torch.int32, device="cuda")
+    se = torch.empty(shape, dtype=torch.int32, device="cuda")
+    skv.attn_select_centroids(dev["q"], dev["centroids"], dev["cluster_off"], wl.topk, ids, ss, se)
+    torch.cuda.synchronize()
+    return ids, ss, se
+
+
+def check_selection(wl, ids_gpu, groups, q=None):
+    """ids must equal the oracle's except at flagged near-tie boundaries."""
+    q = skvgen.host_q(wl) if q is None else q
+    flagged = 0
+    for (b, kvh) in groups:
+        _, off, cent = skvgen.host_mixture_group(wl, b, kvh, want_keys=False)
+        qg = q[b, 0, kvh * wl.G:(kvh + 1) * wl.G]
+        ids, sc = oracle.select(qg[None], cent[None], wl.topk)
+        if not np.array_equal(ids[0], ids_gpu[b, kvh]):
+            gap = oracle.topk_boundary_gap(sc, wl.topk)[0]
+            assert gap <= TOPK_FLAG_GAP, f"selection differs for ({b},{kvh}), gap {gap:.2e}"
+            # the GPU's choice must still be a valid top-k up to the near tie
+            flagged += 1
+    return flagged
+
+
+def test_select_and_attend_small_mixture():
+    wl = skvgen.Workload("m", B=2, Hq=8, Hkv=2, L=3000, mixture=True, c_log2=6, topk=7, seed=61)
+    dev = device_workload(wl)
+    ids, ss, se = _select(wl, dev)
+    ids_h = ids.cpu().numpy()
+    groups = [(b, h) for b in range(2) for h in range(2)]
+    assert check_selection(wl, ids_h, groups) == 0
+    off = dev["cluster_off"].cpu().numpy()
+    np.testing.assert_array_equal(ss.cpu().numpy(), np.take_along_axis(off, ids_h, axis=2))
+    np.testing.assert_array_equal(se.cpu().numpy(), np.take_along_axis(off, ids_h + 1, axis=2))
+    res = run_decode(wl, dev, segments=(ss, se))
+    assert res[3] == 0
+    q = skvgen.host_q(wl)
+    for b, kvh in groups:
+        keys = oracle.keys_segments(off[b, kvh, ids_h[b, kvh]], off[b, kvh, ids_h[b, kvh] + 1])
+        O, lse = oracle_keys_attend(wl, b, kvh, keys, q=q)
+        hs = slice(kvh * 4, kvh * 4 + 4)
+        check_close(res[0][b, hs], res[1][b, hs], O[0], lse[0])
+
+
+def test_select_ties_go_to_lower_index():
+    torch = _torch()
+    import sparse_kv_b200 as skv
+    C, k = 300, 17
+    q = torch.zeros((1, 4, 128), dtype=torch.bfloat16, device="cuda")
+    q[0, :, 0] = 1.0
+    vals = np.random.default_rng(2).integers(0, 6, C).astype(np.float32)  # many exact ties
+    cent = torch.zeros((1, 1, C, 128), dtype=torch.bfloat16, device="cuda")
+    cent[0, 0, :, 0] = torch.tensor(vals, device="cuda")
+    off = torch.arange(C + 1, dtype=torch.int32, device="cuda").view(1, 1, C + 1)
+    ids = torch.empty((1, 1, k), dtype=torch.int32, device="cuda")
+    ss, se = torch.empty_like(ids), torch.empty_like(ids)
+    skv.attn_select_centroids(q, cent, off, k, ids, ss, se)
+    want = sorted(sorted(range(C), key=lambda c: (-vals[c], c))[:k])
+    assert ids.cpu().numpy()[0, 0].tolist() == want
