@@ -23,7 +23,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -36,8 +35,8 @@ METRIC = "decode-attn effective KV GB/s (fraction of B200 HBM peak); attended to
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="cfg2_b16_h32_l32k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -56,110 +55,142 @@ def peaks():
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and clock-event reasons through NVML every few ms in a
+    background thread while the timed region runs (read-only queries)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, uuid):
-        self.uuid = uuid
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+    def __init__(self, uuid, period_s=0.005):
+        self.uuid, self.period = uuid, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.ok = False
 
     def __enter__(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", self.uuid], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report it, do not guess
+            self.err = str(e)
+            return self
+        self.stop = threading.Event()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
         return self
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
             try:
-                self.proc.wait(timeout=5)
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, name in self.REASONS.items():
+                    if bits & k:
+                        self.reasons.add(name)
             except Exception:
-                self.proc.kill()
-            self.f.close()
+                pass
+            self.stop.wait(self.period)
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self.stop.set()
+            self.t.join(timeout=2)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # --------------------------------------------------------------------------- CPU baseline (oracle)
 
-def cpu_baseline(wl, max_groups=16, budget_s=20.0):
-    """The fp64 oracle, as it stands, on a bounded sample of the workload:
-    full-traversal attention of `n` KV groups (all G query heads each)."""
+def _oracle_sample(wl, n_groups):
     import numpy as np
-    import oracle
     import skvgen
     q = skvgen.host_q(wl)
-    n = max_groups
-    groups = [(g // wl.Hkv, g % wl.Hkv) for g in range(0, wl.B * wl.Hkv, max(1, wl.B * wl.Hkv // n))][:n]
+    step = max(1, wl.B * wl.Hkv // n_groups)
+    groups = [(g // wl.Hkv, g % wl.Hkv) for g in range(0, wl.B * wl.Hkv, step)][:n_groups]
     Ks, Vs, qs = [], [], []
     for b, kvh in groups:
         K, V = skvgen.host_kv_group(wl, b, kvh, q=q)
         Ks.append(K)
         Vs.append(V)
         qs.append(q[b, 0, kvh * wl.G:(kvh + 1) * wl.G])
-    Ks, Vs, qs = np.stack(Ks), np.stack(Vs), np.stack(qs)
     keys = [[np.arange(wl.L)] * wl.G for _ in groups]
-    t0 = time.perf_counter()
-    oracle.attend(qs, Ks, Vs, keys, wl.scale)
-    dt = time.perf_counter() - t0
-    nbytes = len(groups) * wl.L * wl.d * 2 * 2
+    return np.stack(qs), np.stack(Ks), np.stack(Vs), keys, groups
+
+
+def cpu_baseline(wl, budget_s=20.0, chunk=16):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload:
+    full-traversal attention of whole KV groups (all G query heads each), in
+    chunks of `chunk` groups until every group is done or `budget_s` of oracle
+    time is spent."""
+    import oracle
+    total_groups = wl.B * wl.Hkv
+    done, t_oracle = 0, 0.0
+    while done < total_groups and t_oracle < budget_s:
+        n = min(chunk, total_groups - done)
+        qs, Ks, Vs, keys, _ = _oracle_sample_range(wl, done, n)
+        t0 = time.perf_counter()
+        oracle.attend(qs, Ks, Vs, keys, wl.scale)
+        t_oracle += time.perf_counter() - t0
+        done += n
+    nbytes = done * wl.L * wl.d * 2 * 2
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(groups)} of {wl.B * wl.Hkv} KV groups of {wl.name}, full traversal, "
-                      f"fp64, {dt:.2f} s"}
+    return {"value": nbytes / t_oracle / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {total_groups} KV groups of {wl.name}, full traversal, fp64 "
+                      f"oracle time {t_oracle:.2f} s"}
+
+
+def _oracle_sample_range(wl, g0, n):
+    import numpy as np
+    import skvgen
+    q = skvgen.host_q(wl)
+    Ks, Vs, qs = [], [], []
+    for g in range(g0, g0 + n):
+        b, kvh = g // wl.Hkv, g % wl.Hkv
+        K, V = skvgen.host_kv_group(wl, b, kvh, q=q)
+        Ks.append(K)
+        Vs.append(V)
+        qs.append(q[b, 0, kvh * wl.G:(kvh + 1) * wl.G])
+    keys = [[np.arange(wl.L)] * wl.G for _ in range(n)]
+    return np.stack(qs), np.stack(Ks), np.stack(Vs), keys, None
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle on the host cores (rank 0 only)."""
+    """--impl reference: the CPU oracle, as it stands, on the host cores (rank
+    0 only).  Each step is the oracle's full-traversal attention over a bounded
+    sample of the workload (4 of its KV groups), so that the run ends within a
+    few minutes."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import oracle
     import skvgen
     wl = skvgen.WORKLOADS[args.workload]
-    times, val = [], None
     n_groups = 4
-    for i in range(args.warmup + args.steps):
-        r = cpu_baseline(wl, max_groups=n_groups)
-        if i >= args.warmup:
-            times.append(r)
-    vals = [r["value"] for r in times]
-    v = statistics.median(vals)
+    qs, Ks, Vs, keys, groups = _oracle_sample(wl, n_groups)
+    for _ in range(args.warmup):
+        oracle.attend(qs, Ks, Vs, keys, wl.scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attend(qs, Ks, Vs, keys, wl.scale)
+    dt = (time.perf_counter() - t0) / args.steps
     nbytes = n_groups * wl.L * wl.d * 4
-    ms = nbytes / (v * 1e9) * 1e3
+    v = nbytes / dt / 1e9
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = f"{n_groups} of {wl.B * wl.Hkv} KV groups of {wl.name} per step, full traversal, fp64"
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": wl.name, "sample_groups": n_groups},
-           "cpu_baseline": {"value": v, "unit": "GB/s", "kind": "oracle", "cores": times[0]["cores"],
-                            "sample": times[0]["sample"]},
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": wl.name, "sample_groups": n_groups},
+           "cpu_baseline": {"value": v, "unit": "GB/s", "kind": "oracle", "cores": cores,
+                            "sample": sample},
            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 

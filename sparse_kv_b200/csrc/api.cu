@@ -18,19 +18,23 @@ struct Plan {
   int G = 0;
   int mode = TRAV_NATURAL;
   bool art = false;
+  int sched = SCHED_GROUP;
+  int n_ctas = 0;
   int splits = 1;
+  int nw = 0;
+  size_t hdr_bytes = 0;
   size_t ws_bytes = 0;
 };
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 // Split count for traversals of up to n_tiles tiles per group: minimise
 // (waves x tiles per CTA) plus a per-wave fill cost, one resident CTA per SM.
-int choose_splits(long long groups, int n_tiles) {
+int choose_splits(long long groups, long long n_tiles) {
   if (n_tiles <= 1 || groups <= 0) return 1;
   const int sms = num_sms();
-  const int s_max = std::max(1, std::min(64, n_tiles / 4));
+  const int s_max = (int)std::max<long long>(1, std::min<long long>(64, n_tiles / 4));
   int best = 1;
   long long best_cost = -1;
   for (int s = 1; s <= s_max; ++s) {
@@ -77,33 +81,38 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
   pl->G = G;
   pl->art = a->art.enable != 0;
   pl->mode = has_order ? TRAV_ORDER : has_seg ? TRAV_SEGMENTS : has_win ? TRAV_WINDOW : TRAV_NATURAL;
+  pl->nw = decode_consumer_warps(G, pl->art);
   pl->splits = 1;
+  pl->n_ctas = 0;
+  pl->hdr_bytes = 0;
   pl->ws_bytes = 0;
-  if (!pl->art) {
-    const long long L = a->max_seq_len;
-    int n_tiles = 0;
-    switch (pl->mode) {
-      case TRAV_NATURAL:
-        if (has_range) {
-          const long long e = std::min<long long>(a->kv_end, L);
-          n_tiles = (e > a->kv_begin) ? cdiv(e, kBlock) - a->kv_begin / kBlock : 0;
-        } else {
-          n_tiles = cdiv(L, kBlock);
-        }
-        break;
-      case TRAV_ORDER: n_tiles = a->order_len; break;
-      case TRAV_WINDOW:
-        n_tiles = cdiv(std::min<long long>(a->window.sink_tokens, L), kBlock) +
-                  cdiv(std::min<long long>(a->window.recent_tokens, L), kBlock) + 1;
-        break;
-      default: n_tiles = a->n_seg; break;
-    }
-    pl->splits = choose_splits((long long)a->batch * a->kv_heads, n_tiles);
-    if (pl->splits > 1) {
-      const size_t rows = (size_t)a->batch * a->q_heads;
-      pl->ws_bytes = (size_t)pl->splits * rows * (kHeadDim + 1) * sizeof(float);
-    }
+  if (pl->art) {
+    pl->sched = SCHED_GROUP;
+    return SKV_OK;
   }
+  const long long groups = (long long)a->batch * a->kv_heads;
+  long long slots = 0;
+  if (pl->mode != TRAV_SEGMENTS && a->batch <= kMaxPersistentBatch) {
+    DecodeParams probe{};
+    probe.mode = pl->mode;
+    probe.range_begin = a->kv_begin;
+    probe.range_end = a->kv_end;
+    probe.sink = a->window.sink_tokens;
+    probe.recent = a->window.recent_tokens;
+    probe.order_len = a->order_len;
+    const long long t_est = groups * group_tiles(probe, a->max_seq_len);
+    if (t_est >= (1ll << 31)) return SKV_EUNSUPPORTED;
+    pl->sched = SCHED_PERSISTENT;
+    const long long max_ctas = (long long)num_sms() * decode_ctas_per_sm(G, false);
+    pl->n_ctas = (int)std::max<long long>(1, std::min<long long>(max_ctas, cdiv(t_est, 4)));
+    slots = pl->n_ctas + groups;
+    pl->hdr_bytes = (size_t)cdiv((a->batch + 2) * 4ll, 256) * 256;
+  } else {
+    pl->sched = SCHED_SPLIT;
+    pl->splits = choose_splits(groups, pl->mode == TRAV_SEGMENTS ? a->n_seg : cdiv(a->max_seq_len, kBlock));
+    slots = groups * pl->splits;
+  }
+  pl->ws_bytes = pl->hdr_bytes + (size_t)slots * pl->nw * G * kRecFloats * sizeof(float);
   return SKV_OK;
 }
 
@@ -150,6 +159,8 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
   p.sink = a->window.sink_tokens;
   p.recent = a->window.recent_tokens;
   p.mode = pl.mode;
+  p.sched = pl.sched;
+  p.n_ctas = pl.n_ctas;
   p.n_splits = pl.splits;
   p.qscale = a->scale * 1.4426950408889634f;
   p.tau = a->art.tau;
@@ -159,21 +170,14 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
   p.lse = a->lse;
   p.blocks_consumed = a->blocks_consumed;
   p.status = a->status_word;
-  const size_t rows = (size_t)a->batch * a->q_heads;
-  if (pl.splits > 1) {
-    p.ws_o = static_cast<float*>(a->workspace);
-    p.ws_lse = p.ws_o + (size_t)pl.splits * rows * kHeadDim;
+  p.rec_nw = pl.nw;
+  if (!pl.art) {
+    p.ws_hdr = static_cast<int*>(a->workspace);
+    p.ws_rec = reinterpret_cast<float*>(static_cast<char*>(a->workspace) + pl.hdr_bytes);
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (a->blocks_consumed && !pl.art) {
-    if (cudaMemsetAsync(a->blocks_consumed, 0, rows * sizeof(int32_t), s) != cudaSuccess)
-      return SKV_ECUDA;
-  }
   if (launch_decode(p, pl.G, pl.art, s) != 0) return SKV_ECUDA;
-  if (pl.splits > 1) {
-    if (launch_merge(p.ws_o, p.ws_lse, pl.splits, (int)rows, kHeadDim, a->out, a->lse, s) != 0)
-      return SKV_ECUDA;
-  }
+  if (!pl.art && launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
   return SKV_OK;
 }
 

@@ -13,6 +13,15 @@ enum TravMode : int {
   TRAV_SEGMENTS = 3,  // caller's token segments
 };
 
+enum Schedule : int {
+  SCHED_PERSISTENT = 0,  // one CTA per SM walks an even share of all tiles of all groups
+  SCHED_SPLIT = 1,       // grid (splits, kv_heads, batch), each CTA one piece of one group
+  SCHED_GROUP = 2,       // grid (1, kv_heads, batch), one CTA walks a whole group (ART)
+};
+
+constexpr int kMaxPersistentBatch = 1024;  // batch prefix kept in shared memory
+constexpr int kRecFloats = 132;            // partial record: O[128], m (base 2), l, tiles, pad
+
 struct DecodeParams {
   const uint16_t* q;
   const uint16_t* k_pool;
@@ -28,7 +37,9 @@ struct DecodeParams {
   int range_begin, range_end;  // token range (range_end > 0 => active)
   int sink, recent;
   int mode;
-  int n_splits;
+  int sched;
+  int n_ctas;    // SCHED_PERSISTENT: grid size
+  int n_splits;  // SCHED_SPLIT: pieces per group
   float qscale;  // softmax scale * log2(e): scores are kept in base-2 units
   float tau, phi;
   int patience;
@@ -36,14 +47,43 @@ struct DecodeParams {
   float* lse;
   int* blocks_consumed;
   uint32_t* status;
-  float* ws_o;    // [n_splits][B*Hq][128] when n_splits > 1
-  float* ws_lse;  // [n_splits][B*Hq]
+  // Non-ART workspace: header (total tiles, batch prefix) and per-warp partial
+  // records [slots][rec_nw][G][kRecFloats], merged by launch_merge_records.
+  int* ws_hdr;
+  float* ws_rec;
+  int rec_nw;
 };
+
+// Tiles of one KV group for the index-based traversals (natural / range /
+// window / order), given the sequence length L.
+__host__ __device__ inline int group_tiles(const DecodeParams& p, int L) {
+  const int nb = (L + 63) / 64;
+  switch (p.mode) {
+    case TRAV_NATURAL: {
+      int ra = 0, re = L;
+      if (p.range_end > 0) {
+        ra = p.range_begin > 0 ? p.range_begin : 0;
+        re = p.range_end < L ? p.range_end : L;
+      }
+      return (re > ra) ? (re + 63) / 64 - ra / 64 : 0;
+    }
+    case TRAV_WINDOW: {
+      const int A = p.sink < L ? p.sink : L;
+      const int Rs = (L - p.recent > A) ? L - p.recent : A;
+      return (A + 63) / 64 + ((L > Rs) ? nb - Rs / 64 : 0);
+    }
+    case TRAV_ORDER: return p.order_len;
+    default: return 0;
+  }
+}
 
 // Host-side launchers (decode.cu / merge.cu / select.cu).
 int launch_decode(const DecodeParams& p, int G, bool art, void* stream);
+int decode_consumer_warps(int G, bool art);
+int decode_ctas_per_sm(int G, bool art);
 int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int d, float* out,
                  float* lse, void* stream);
+int launch_merge_records(const DecodeParams& p, int G, void* stream);
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int* ids, int* ss, int* se, void* stream);
 int num_sms();

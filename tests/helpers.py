@@ -92,7 +92,8 @@ def check_close(O_gpu, lse_gpu, O_ref, lse_ref, what=""):
     assert np.all(np.isfinite(O_gpu)), f"{what}: non-finite output"
     err = np.abs(O_gpu - O_ref).max() if O_ref.size else 0.0
     assert err <= ATOL_O, f"{what}: max |dO| = {err:.3e}"
-    ok = both_empty | (np.abs(lse_gpu - lse_ref) <= RTOL_LSE * np.maximum(1.0, np.abs(lse_ref)))
+    with np.errstate(invalid="ignore"):
+        ok = both_empty | (np.abs(lse_gpu - lse_ref) <= RTOL_LSE * np.maximum(1.0, np.abs(lse_ref)))
     assert np.all(ok), f"{what}: LSE mismatch {lse_gpu[~ok][:4]} vs {lse_ref[~ok][:4]}"
     return err
 

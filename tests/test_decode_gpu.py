@@ -200,7 +200,7 @@ def test_art_structured_small(tau, phi, p):
     assert flagged <= 2
 
 
-@pytest.mark.parametrize("p", [1, 4])
+@pytest.mark.parametrize("p", [1, 2, 3, 4])
 def test_art_always_passing_stops_after_one_plus_p_blocks(p):
     # thresholds no probe change can reach (d_scale < 10, 1 - cos < 2.5): every
     # test passes, so each head stops after block 0 and p more blocks
@@ -216,6 +216,21 @@ def test_art_always_passing_stops_after_one_plus_p_blocks(p):
     for b in range(2):
         for kvh in range(2):
             check_art(wl, res, b, kvh, q=q, tau=10.0, phi=2.5, patience=p)
+
+
+@pytest.mark.parametrize("G", [1, 2, 8])
+def test_art_other_group_sizes(G):
+    lens = [64 * 21 + 9, 64 * 6]
+    wl = skvgen.Workload("ag", B=2, Hq=2 * G, Hkv=2, L=max(lens), lens=lens, structured=True,
+                         paging="perm", seed=44 + G, softmax_scale=0.3)
+    dev = device_workload(wl)
+    q = skvgen.host_q(wl)
+    for tau, phi, p in [(10.0, 2.5, 2), (0.0, 0.0, 1), (3e-2, 3e-3, 2)]:
+        res = run_decode(wl, dev, art=(tau, phi, p))
+        assert res[3] == 0
+        for b in range(2):
+            for kvh in range(2):
+                check_art(wl, res, b, kvh, q=q, tau=tau, phi=phi, patience=p)
 
 
 def test_art_with_caller_order_skips_block0_in_list():
