@@ -151,6 +151,30 @@ SKV_API size_t skv_decode_workspace_size(const skv_decode_args* args);
  * `order` traversal. */
 SKV_API skv_status attn_decode(const skv_decode_args* args, skv_stream_t stream);
 
+/* attn_decode without any allocation -- for callers that cannot allocate.
+ * The pages have no counterpart of this call; it is a deployment aid.
+ *
+ * attn_decode needs device scratch (skv_decode_workspace_size bytes) that the
+ * caller normally allocates.  Some callers cannot allocate at the point where
+ * they decode (an allocator that must not be re-entered, a hook running
+ * inside another library, device memory reserved in full up front).  This
+ * call computes exactly what attn_decode computes, with the same arguments
+ * (args->workspace and args->workspace_bytes are ignored), but takes its
+ * scratch from a fixed array of SKV_STATIC_WORKSPACE_BYTES inside the
+ * library's device image, which every GPU that loads the library holds until
+ * the process exits.  It calls no allocator.
+ *  - Arguments needing more scratch than SKV_STATIC_WORKSPACE_BYTES (see
+ *    skv_decode_workspace_size) return SKV_EWORKSPACE and launch nothing.
+ *  - The first call on each device looks up the array's device address, with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents.
+ *    Nothing in it needs to start at zero (every byte read is written earlier
+ *    in the same call), but calls that can overlap on the GPU (other streams,
+ *    other host threads) race on it: serialise them.
+ * Errors: as attn_decode, plus SKV_ECUDA if the address lookup fails. */
+#define SKV_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)
+SKV_API skv_status attn_decode_static_ws(const skv_decode_args* args, skv_stream_t stream);
+
 /* Centroid selection ("Squeezed Attention" Q2 step 2) for each KV group
  * (b, kvh): score_c = (sum over the group's q_heads/kv_heads query heads of
  * q_h) . centroid_c, c in [0, n_clusters); keep the `topk` largest, ties to the

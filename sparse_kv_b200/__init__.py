@@ -13,7 +13,8 @@ import os
 
 from . import _build
 
-__all__ = ["attn_decode", "attn_select_centroids", "attn_merge_lse", "decode_workspace_size",
+__all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_merge_lse",
+           "decode_workspace_size",
            "strerror", "SkvError", "lib", "DEV_BITS"]
 
 SKV_OK, SKV_EINVAL, SKV_EUNSUPPORTED, SKV_ECUDA, SKV_ETIMEOUT, SKV_EWORKSPACE = range(6)
@@ -65,6 +66,8 @@ def lib():
         L.skv_decode_workspace_size.restype = ctypes.c_size_t
         L.attn_decode.argtypes = [ctypes.POINTER(DecodeArgs), _p]
         L.attn_decode.restype = _i
+        L.attn_decode_static_ws.argtypes = [ctypes.POINTER(DecodeArgs), _p]
+        L.attn_decode_static_ws.restype = _i
         L.attn_select_centroids.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p]
         L.attn_select_centroids.restype = _i
         L.attn_merge_lse.argtypes = [_p, _p, _i, _i, _i, _p, _p, _p]
@@ -141,6 +144,18 @@ def attn_decode(*args, stream=None, **kw):
     st = lib().attn_decode(ctypes.byref(a), _stream(stream))
     if st != SKV_OK:
         raise SkvError(st, "attn_decode")
+
+
+def attn_decode_static_ws(*args, stream=None, **kw):
+    """attn_decode for callers that cannot allocate device memory: same
+    arguments (any workspace is ignored), scratch taken from a fixed array in
+    the library (SKV_STATIC_WORKSPACE_BYTES).  Calls share that array, so they
+    must not overlap on the GPU.  Raises SkvError."""
+    kw.pop("workspace", None)
+    a = make_decode_args(*args, **kw)
+    st = lib().attn_decode_static_ws(ctypes.byref(a), _stream(stream))
+    if st != SKV_OK:
+        raise SkvError(st, "attn_decode_static_ws")
 
 
 def attn_decode_args(a, stream=None):
