@@ -197,12 +197,158 @@ def run_reference(args):
 
 # --------------------------------------------------------------------------- our arm
 
+class Step:
+    """One benchmark step: `run()` launches it on the current stream; `nbytes`
+    are the algorithmic bytes it moves; `launches` our kernels per step."""
+
+    def __init__(self, run, nbytes, launches, extra=None):
+        self.run, self.nbytes, self.launches, self.extra = run, nbytes, launches, extra or {}
+
+
+def _paged_inputs(torch, skvgen, wl, layer=0):
+    bt_host, num_pages = skvgen.block_table_host(wl, layer)
+    q = skvgen.device_q(wl, layer)
+    k_pool = torch.empty((max(num_pages, 1), wl.Hkv, wl.bs, wl.d), dtype=torch.bfloat16, device="cuda")
+    v_pool = torch.empty_like(k_pool)
+    block_table = torch.tensor(bt_host, device="cuda")
+    seq_lens = torch.tensor([wl.seq_len(b) for b in range(wl.B)], dtype=torch.int32, device="cuda")
+    return q, k_pool, v_pool, block_table, seq_lens
+
+
+def build_decode(torch, skv, skvgen, wl, status, art=False):
+    """Full-traversal (or ART) decode of one paged workload."""
+    q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, wl)
+    skvgen.device_kv_paged(wl, q, k_pool, v_pool, bt, sl)
+    out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
+    consumed = torch.zeros((wl.B, wl.Hq), dtype=torch.int32, device="cuda")
+    common = (q, k_pool, v_pool, bt, sl, out, lse)
+    kw = dict(max_seq_len=wl.Lmax, scale=wl.scale, status=status, blocks_consumed=consumed)
+    if art:
+        kw["art"] = (wl.tau, wl.phi, wl.patience)
+    n = skv.decode_workspace_size(*common, **kw)
+    ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda") if n else None
+    a = skv.make_decode_args(*common, workspace=ws, **kw)
+    L = skv.lib()
+
+    def run():
+        st = L.attn_decode(ctypes.byref(a), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise skv.SkvError(st, "attn_decode")
+
+    step = Step(run, wl.kv_bytes(), 1 if (art or not n) else 2)
+    # keep every tensor the raw pointers in `a` refer to alive with the step
+    step.tensors = dict(q=q, k_pool=k_pool, v_pool=v_pool, bt=bt, sl=sl, out=out, lse=lse,
+                        consumed=consumed, ws=ws, kw=kw, common=common)
+    return step
+
+
+def build_select(torch, skv, skvgen, wl, status):
+    """Centroid scoring + top-k, then attention over the chosen clusters' keys."""
+    q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, wl)
+    off, cent = skvgen.device_mixture(wl, k_pool, bt)
+    skvgen.device_kv_paged(wl, q, k_pool, v_pool, bt, sl, keys=False)
+    shape = (wl.B, wl.Hkv, wl.topk)
+    ids = torch.empty(shape, dtype=torch.int32, device="cuda")
+    ss = torch.empty(shape, dtype=torch.int32, device="cuda")
+    se = torch.empty(shape, dtype=torch.int32, device="cuda")
+    out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
+    kw = dict(max_seq_len=wl.Lmax, scale=wl.scale, status=status, segments=(ss, se))
+    n = skv.decode_workspace_size(q, k_pool, v_pool, bt, sl, out, lse, **kw)
+    ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda")
+    a = skv.make_decode_args(q, k_pool, v_pool, bt, sl, out, lse, workspace=ws, **kw)
+    L = skv.lib()
+    B, Hq, Hkv, C, k = wl.B, wl.Hq, wl.Hkv, 1 << wl.c_log2, wl.topk
+    qp, cp, op = ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(cent.data_ptr()), ctypes.c_void_p(off.data_ptr())
+    ip, sp_, ep = (ctypes.c_void_p(t.data_ptr()) for t in (ids, ss, se))
+
+    def run():
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        st = L.attn_select_centroids(qp, cp, op, B, Hq, Hkv, wl.d, C, k, ip, sp_, ep, stream)
+        if st != 0:
+            raise skv.SkvError(st, "attn_select_centroids")
+        st = L.attn_decode(ctypes.byref(a), stream)
+        if st != 0:
+            raise skv.SkvError(st, "attn_decode")
+
+    run()
+    torch.cuda.synchronize()
+    sel_tokens = int((se - ss).sum().item())
+    nbytes = sel_tokens * wl.d * 4 + cent.numel() * 2 + off.numel() * 4
+    step = Step(run, nbytes, 3, {"selected_tokens": sel_tokens,
+                                 "selected_frac": sel_tokens / (wl.B * wl.Hkv * wl.L),
+                                 "centroid_bytes": cent.numel() * 2})
+    # keep every tensor the raw pointers above refer to alive with the step
+    step.tensors = dict(q=q, k_pool=k_pool, v_pool=v_pool, bt=bt, sl=sl, off=off, cent=cent, ids=ids,
+                        ss=ss, se=se, out=out, lse=lse, ws=ws)
+    return step
+
+
+def build_routed(torch, skv, skvgen, wl, status):
+    """32 independent attention layers; layer l runs full attention with ART
+    when its seeded route bit is 1, else the sink + recent window only, whose
+    cache holds just those blocks."""
+    layers = []
+    for l in range(wl.n_layers):
+        fa = skvgen.route_bit(wl.seed, l) == 1
+        lw = wl.with_(paging="identity" if fa else "window")
+        q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, lw, layer=l)
+        skvgen.device_kv_paged(lw, q, k_pool, v_pool, bt, sl, layer=l)
+        out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
+        lse = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
+        consumed = torch.zeros((wl.B, wl.Hq), dtype=torch.int32, device="cuda")
+        kw = dict(max_seq_len=wl.Lmax, scale=wl.scale, status=status, blocks_consumed=consumed)
+        if fa:
+            kw["art"] = (wl.tau, wl.phi, wl.patience)
+        else:
+            kw["window"] = (wl.sink, wl.recent)
+        n = skv.decode_workspace_size(q, k_pool, v_pool, bt, sl, out, lse, **kw)
+        ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda") if n else None
+        a = skv.make_decode_args(q, k_pool, v_pool, bt, sl, out, lse, workspace=ws, **kw)
+        layers.append(dict(fa=fa, a=a, keep=(q, k_pool, v_pool, bt, sl, out, lse, consumed, ws),
+                           consumed=consumed, launches=1 if (fa or not n) else 2))
+    L = skv.lib()
+
+    def run():
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        for ly in layers:
+            st = L.attn_decode(ctypes.byref(ly["a"]), stream)
+            if st != 0:
+                raise skv.SkvError(st, "attn_decode")
+
+    run()
+    torch.cuda.synchronize()
+    nbytes, fa_n, fa_bytes_full, skipped = 0, 0, 0, []
+    win_tokens = len(__import__("oracle").keys_window(wl.L, wl.sink, wl.recent))
+    for ly in layers:
+        if ly["fa"]:
+            fa_n += 1
+            grp = ly["consumed"].cpu().numpy().reshape(wl.B, wl.Hkv, wl.G).max(axis=2)
+            nbytes += int(grp.sum()) * wl.bs * wl.d * 4
+            fa_bytes_full += wl.kv_bytes()
+            skipped.append(1.0 - float(grp.sum()) / (wl.B * wl.Hkv * wl.nb(0)))
+        else:
+            nbytes += wl.B * wl.Hkv * win_tokens * wl.d * 4
+    step = Step(run, nbytes, sum(ly["launches"] for ly in layers),
+                {"fa_layers": fa_n, "sa_layers": wl.n_layers - fa_n,
+                 "art_blocks_skipped_frac_mean": float(np.mean(skipped)) if skipped else 0.0,
+                 "dense_equivalent_bytes": fa_bytes_full + (wl.n_layers - fa_n) * wl.kv_bytes()})
+    step.tensors = dict(layers=layers)
+    return step
+
+
+np = None
+
+
 def main():
+    global np
     args = parse()
     if args.impl == "reference":
         run_reference(args)
         return
-    import numpy as np
+    import numpy
+    np = numpy
     import torch
     import torch.distributed as dist
 
@@ -215,54 +361,44 @@ def main():
 
     import skvgen
     import sparse_kv_b200 as skv
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
     wl = skvgen.WORKLOADS[args.workload]
     hbm_peak, peak_kind = peaks()
-
-    # ---- inputs resident in HBM
-    bt_host, num_pages = skvgen.block_table_host(wl)
-    q = skvgen.device_q(wl)
-    k_pool = torch.empty((num_pages, wl.Hkv, wl.bs, wl.d), dtype=torch.bfloat16, device="cuda")
-    v_pool = torch.empty_like(k_pool)
-    block_table = torch.tensor(bt_host, device="cuda")
-    seq_lens = torch.full((wl.B,), wl.L, dtype=torch.int32, device="cuda")
-    skvgen.device_kv_paged(wl, q, k_pool, v_pool, block_table, seq_lens)
-    out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
-    lse = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
-    consumed = torch.zeros((wl.B, wl.Hq), dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    common = (q, k_pool, v_pool, block_table, seq_lens, out, lse)
-    kw = dict(max_seq_len=wl.L, scale=wl.scale, status=status)
-    ws_n = skv.decode_workspace_size(*common, **kw)
-    ws = torch.empty(max(ws_n, 16) // 4 + 4, dtype=torch.float32, device="cuda")
-    a_full = skv.make_decode_args(*common, workspace=ws, **kw)
-    a_art = skv.make_decode_args(*common, art=(wl.tau, wl.phi, wl.patience), blocks_consumed=consumed,
-                                 **kw)
+
+    kind = args.workload.split("_")[0]
+    if kind in ("cfg1", "cfg2"):
+        step = build_decode(torch, skv, skvgen, wl, status)
+    elif kind == "cfg3":
+        step = build_select(torch, skv, skvgen, wl, status)
+    elif kind == "cfg5":
+        step = build_routed(torch, skv, skvgen, wl, status)
+    else:
+        raise SystemExit(f"workload {args.workload}: no bench step")
+    art_step = build_decode(torch, skv, skvgen, wl, status, art=True) if (kind == "cfg2" and not args.no_art) else None
     stream = torch.cuda.current_stream()
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    L = skv.lib()
-    kv_bytes = wl.kv_bytes()
-    head_tokens = wl.B * wl.L * wl.Hq
 
-    def launch(a):
-        st = L.attn_decode(ctypes.byref(a), sp)
-        if st != 0:
-            raise skv.SkvError(st, "attn_decode")
-
-    def timed(a, steps, warmup):
+    def timed(st, steps, warmup):
+        """CUDA-graph replay of `steps` steps, each bracketed by events."""
         for _ in range(warmup):
-            launch(a)
+            st.run()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            st.run()
+        for _ in range(2):
+            g.replay()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for e0, e1 in evs:
             e0.record(stream)
-            launch(a)
+            g.replay()
             e1.record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
@@ -272,57 +408,63 @@ def main():
             t = torch.tensor([total_ms], device="cuda")
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             total_ms = float(t.item())
+        del g
         return total_ms, per
 
     uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     with ClockSampler(uuid) as clk:
-        total_ms, per = timed(a_full, args.steps, args.warmup)
-        art_ms, art_per = (None, None)
-        if not args.no_art:
-            art_ms, art_per = timed(a_art, args.steps, args.warmup)
+        total_ms, per = timed(step, args.steps, args.warmup)
+        art_ms = None
+        if art_step is not None:
+            art_ms, _ = timed(art_step, args.steps, args.warmup)
     clocks = clk.summary()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status word {int(status.item()):#x}")
 
     ms_step = total_ms / args.steps
-    value = kv_bytes * world / (ms_step * 1e-3) / 1e9
+    value = step.nbytes * world / (ms_step * 1e-3) / 1e9
     per_launch_ms = statistics.mean(per)
-    achieved = kv_bytes / (per_launch_ms * 1e-3) / 1e9
+    achieved = step.nbytes / (per_launch_ms * 1e-3) / 1e9
 
-    # ---- end to end through the public API: q, tables in from pinned host, O/LSE out
-    q_h = q.cpu().pin_memory()
-    bt_h = block_table.cpu().pin_memory()
-    sl_h = seq_lens.cpu().pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    # ---- end to end through the public API: q (and tables) in from pinned host, O/LSE out
+    e2e = None
+    if kind in ("cfg1", "cfg2"):
+        T = step.tensors
+        q_h, bt_h, sl_h = (T[k].cpu().pin_memory() for k in ("q", "bt", "sl"))
+        out_h = torch.empty(T["out"].shape, dtype=torch.float32).pin_memory()
+        lse_h = torch.empty(T["lse"].shape, dtype=torch.float32).pin_memory()
 
-    def e2e_step():
-        q.copy_(q_h, non_blocking=True)
-        block_table.copy_(bt_h, non_blocking=True)
-        seq_lens.copy_(sl_h, non_blocking=True)
-        skv.attn_decode(*common, workspace=ws, stream=stream, **kw)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        def e2e_step():
+            T["q"].copy_(q_h, non_blocking=True)
+            T["bt"].copy_(bt_h, non_blocking=True)
+            T["sl"].copy_(sl_h, non_blocking=True)
+            skv.attn_decode(*T["common"], workspace=T["ws"], stream=stream, **T["kw"])
+            out_h.copy_(T["out"], non_blocking=True)
+            lse_h.copy_(T["lse"], non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    h2d = q.numel() * 2 + block_table.numel() * 4 + seq_lens.numel() * 4
-    d2h = out.numel() * 4 + lse.numel() * 4
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
+        d2h = out_h.numel() * 4 + lse_h.numel() * 4
+        e2e = {"value": step.nbytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "KV cache resident in HBM; per step q, block table and seq_lens copied in "
+                       "from pinned host memory and O, LSE copied out"}
 
     res = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -330,40 +472,59 @@ def main():
         "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
                    "head_dim": wl.d, "context": wl.L, "page_tokens": wl.bs, "paging": wl.paging,
-                   "traversal": "full", "l2": "inputs larger than L2 (2 GiB KV per step), no flush",
+                   "l2": "inputs larger than L2 (GBs of KV per step), no flush",
+                   "timing": "CUDA-graph replay per step, CUDA events",
                    "parallelism": f"replicas x{world}"},
-        "attended_tokens_per_s": head_tokens * world / (ms_step * 1e-3),
-        "kv_tokens_per_s": wl.B * wl.L * wl.Hkv * world / (ms_step * 1e-3),
+        "attended_tokens_per_s": step.nbytes / (wl.d * 4) * wl.G * world / (ms_step * 1e-3),
+        "kv_tokens_per_s": step.nbytes / (wl.d * 4) * world / (ms_step * 1e-3),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
-                     "frac_of_8000": achieved / 8000.0, "traffic": None,
-                     "kernel": "decode_kernel + split merge (one attn_decode call)"},
+                     "frac_of_8000": achieved / 8000.0, "traffic": traffic_for(kind),
+                     "kernel": "one step of our kernels (decode + merge; per-kernel shares in profiles/)"},
         "clocks": clocks,
-        "gpu_launches": args.steps * (2 if ws_n > 0 else 1) + (args.steps if not args.no_art else 0),
+        "gpu_launches": args.steps * step.launches,
     }
+    if step.extra:
+        res["step_detail"] = step.extra
+    if kind in ("cfg1", "cfg2"):
+        res["config"]["traversal"] = "full"
     if art_ms is not None:
-        cons = consumed.cpu().numpy()
-        # loads stop per KV group when all of its heads stopped: bytes = max over the group
+        cons = art_step.tensors["consumed"].cpu().numpy()
         grp = cons.reshape(wl.B, wl.Hkv, wl.G).max(axis=2)
         art_bytes = int(grp.sum()) * wl.bs * wl.d * 4
-        art_step = art_ms / args.steps
-        res["art"] = {"ms_per_step": art_step, "kv_gbs": art_bytes / (art_step * 1e-3) / 1e9,
+        art_step_ms = art_ms / args.steps
+        res["art"] = {"ms_per_step": art_step_ms, "kv_gbs": art_bytes / (art_step_ms * 1e-3) / 1e9,
                       "blocks_consumed_mean": float(cons.mean()), "blocks_total": wl.nb(0),
                       "blocks_skipped_frac": 1.0 - float(grp.sum()) / (wl.B * wl.Hkv * wl.nb(0)),
-                      "time_vs_full": art_step / ms_step,
-                      "attended_tokens_per_s": float(cons.sum()) * wl.bs / (art_step * 1e-3),
+                      "time_vs_full": art_step_ms / ms_step,
+                      "attended_tokens_per_s": float(cons.sum()) * wl.bs / (art_step_ms * 1e-3),
                       "tau": wl.tau, "phi": wl.phi, "patience": wl.patience}
-    res["e2e"] = {"value": kv_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                  "note": "KV cache resident in HBM; per step q, block table and seq_lens copied in "
-                          "from pinned host memory and O, LSE copied out"}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["gpu_launches"] += args.steps
+    if e2e is not None:
+        res["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and kind in ("cfg1", "cfg2"):
         res["cpu_baseline"] = cpu_baseline(wl)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(res), flush=True)
+
+
+def traffic_for(kind):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/traffic.json), if it was taken on the current kernel
+    source; else None."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "sparse_kv_b200", "csrc", "decode.cu")
+    if not os.path.exists(p):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    rec = json.load(open(p)).get(kind)
+    if not rec or rec.get("decode_cu_sha") != h:
+        return None
+    return rec.get("dram_bytes_per_launch")
 
 
 if __name__ == "__main__":

@@ -30,10 +30,10 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 // Split count for traversals of up to n_tiles tiles per group: minimise
-// (waves x tiles per CTA) plus a per-wave fill cost, one resident CTA per SM.
-int choose_splits(long long groups, long long n_tiles) {
+// (waves x tiles per CTA) plus a per-wave fill cost, given the resident CTAs per SM.
+int choose_splits(long long groups, long long n_tiles, int ctas_per_sm) {
   if (n_tiles <= 1 || groups <= 0) return 1;
-  const int sms = num_sms();
+  const int sms = num_sms() * ctas_per_sm;
   const int s_max = (int)std::max<long long>(1, std::min<long long>(64, n_tiles / 4));
   int best = 1;
   long long best_cost = -1;
@@ -109,7 +109,8 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     pl->hdr_bytes = (size_t)cdiv((a->batch + 2) * 4ll, 256) * 256;
   } else {
     pl->sched = SCHED_SPLIT;
-    pl->splits = choose_splits(groups, pl->mode == TRAV_SEGMENTS ? a->n_seg : cdiv(a->max_seq_len, kBlock));
+    pl->splits = choose_splits(groups, pl->mode == TRAV_SEGMENTS ? a->n_seg : cdiv(a->max_seq_len, kBlock),
+                               decode_ctas_per_sm(G, false));
     slots = groups * pl->splits;
   }
   pl->ws_bytes = pl->hdr_bytes + (size_t)slots * pl->nw * G * kRecFloats * sizeof(float);

@@ -134,6 +134,35 @@ struct Trav {
     }
   }
 
+  // Segment lists: the next piece = up to 64 consecutive tokens inside one
+  // page (page, first row, rows).  Used to pack several segments into one tile.
+  __device__ bool next_piece(int& page, int& r0, int& cnt, uint32_t* status) {
+    while (true) {
+      if (seg_pos >= seg_stop) {
+        if (seg_i >= seg_end_i) return false;
+        const int s = ss[seg_i], t = se[seg_i];
+        ++seg_i;
+        if (s > t) {
+          dev_error(status, SKV_DEV_BAD_SEGMENT);
+          continue;
+        }
+        seg_pos = max(s, 0);
+        seg_stop = min(t, L);
+        continue;
+      }
+      const int blk = seg_pos / kBlock;
+      r0 = seg_pos % kBlock;
+      cnt = min(kBlock - r0, seg_stop - seg_pos);
+      seg_pos += cnt;
+      page = bt[blk];
+      if (page < 0 || page >= num_pages) {
+        dev_error(status, SKV_DEV_BAD_PAGE);
+        continue;
+      }
+      return true;
+    }
+  }
+
   __device__ bool next(int& t0, int& n, int& pg1, int& pg2, int& n1, uint32_t* status) {
     while (true) {
       int a, e;
@@ -498,9 +527,78 @@ __global__ void __launch_bounds__(Cfg<G, NW, ART, MINB>::THREADS, MINB) decode_k
       }
       return true;
     };
+    // Segment lists: rows of several segments are packed into full 64-row
+    // tiles (attention over a key set does not depend on the keys' order);
+    // one bulk copy per piece (<= 64 consecutive tokens of one page).
+    constexpr int kMaxPieces = 8;
+    auto emit_packed = [&](int n, const int* pg, const int* r0, const int* cnt, int np, int g,
+                           int slot, int kvh) -> bool {
+      if (round >= 1) {
+        const uint32_t par = (round - 1) & 1;
+        uint64_t t_start = 0;
+        while (!mbar_try_wait(&empty[ps], par)) {
+          if (flags[0] != 0 || flags[1] != 0) return false;
+          const uint64_t now = globaltimer();
+          if (t_start == 0) t_start = now;
+          else if (now - t_start > kWaitLimitNs) {
+            dev_error(p.status, SKV_DEV_TIMEOUT);
+            flags[1] = 1;
+            aborted = true;
+            return false;
+          }
+        }
+      }
+      meta[ps] = make_int4(n, g, slot, 0);
+      unsigned char* sK = smem + ps * C::STAGE_BYTES;
+      unsigned char* sV = sK + kTileBytes;
+      mbar_arrive_expect_tx(&full[ps], (uint32_t)n * kRowBytes * 2);
+      int row = 0;
+      for (int i = 0; i < np; ++i) {
+        const size_t src = ((size_t)pg[i] * p.Hkv + kvh) * head_stride + (size_t)r0[i] * kHeadDim;
+        bulk_load(sK + row * kRowBytes, p.k_pool + src, (uint32_t)cnt[i] * kRowBytes, &full[ps], pol);
+        bulk_load(sV + row * kRowBytes, p.v_pool + src, (uint32_t)cnt[i] * kRowBytes, &full[ps], pol);
+        row += cnt[i];
+      }
+      ++e;
+      if (++ps == ST) {
+        ps = 0;
+        ++round;
+      }
+      return true;
+    };
+    auto run_segments = [&](Trav& tr, int g, int slot, int kvh) -> bool {
+      int pg[kMaxPieces], r0[kMaxPieces], cnt[kMaxPieces];
+      int np = 0, rows = 0, tiles = 0;
+      int page = 0, first = 0, c = 0;
+      while (flags[0] == 0 && tr.next_piece(page, first, c, p.status)) {
+        while (c > 0) {
+          const int take = min(c, kBlock - rows);
+          pg[np] = page;
+          r0[np] = first;
+          cnt[np] = take;
+          ++np;
+          rows += take;
+          first += take;
+          c -= take;
+          if (rows == kBlock || np == kMaxPieces) {
+            if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
+            ++tiles;
+            np = rows = 0;
+          }
+        }
+      }
+      if (flags[0] != 0) return false;
+      if (rows > 0) {
+        if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
+        ++tiles;
+      }
+      if (tiles == 0 && !emit(0, g, slot, kvh, 0, 0, 0, 0)) return false;
+      return true;
+    };
     // All entries of one group segment; a segment without valid tiles still
     // issues a marker so that the consumers account for the group.
     auto run_group = [&](Trav& tr, int g, int slot, int kvh) -> bool {
+      if (tr.mode == TRAV_SEGMENTS) return run_segments(tr, g, slot, kvh);
       int t0 = 0, n = 0, pg1 = 0, pg2 = 0, n1 = 0, cnt = 0;
       while (flags[0] == 0 && tr.next(t0, n, pg1, pg2, n1, p.status)) {
         if (!emit(n, g, slot, kvh, t0, pg1, pg2, n1)) return false;
@@ -916,9 +1014,16 @@ int launch_t(const DecodeParams& p, cudaStream_t st) {
   constexpr int MINB = minb_for<G, ART>();
   using C = Cfg<G, NW, ART, MINB>;
   auto kern = decode_kernel<G, ART, NW, MINB>;
-  cudaError_t err =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::TOTAL);
-  if (err != cudaSuccess) return (int)err;
+  // Set the shared-memory attribute once per device (not inside a capture).
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::TOTAL);
+    if (err != cudaSuccess) return (int)err;
+    attr_set[dev] = true;
+  }
   dim3 grid;
   if (!ART && p.sched == SCHED_PERSISTENT) grid = dim3(p.n_ctas, 1, 1);
   else grid = dim3(ART ? 1 : p.n_splits, p.Hkv, p.B);

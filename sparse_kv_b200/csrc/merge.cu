@@ -83,13 +83,18 @@ int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int
 namespace skv {
 namespace {
 
-constexpr int kMaxRecords = 256;  // records per row handled by one warp (slots x warps)
-
+// One CTA of kMergeWarps warps per output row.  Records are spread over all
+// threads for the per-record scalars (m, l, tiles) and over the warps for the
+// O vectors (lane j owns dims 4j..4j+3), so many independent loads are in
+// flight; the warps' partial sums are combined through shared memory.
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_records_kernel(const DecodeParams p, int G,
                                                                         int NW) {
-  const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= p.B * p.Hq) return;
+  extern __shared__ float fw[];  // [nrec] weights
+  __shared__ float red[kMergeWarps][2];
+  __shared__ float4 part[kMergeWarps][32];
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NT = kMergeWarps * 32;
   const int b = row / p.Hq, h = row % p.Hq, kvh = h / G, gh = h % G;
   const int g = b * p.Hkv + kvh;
   int s0 = 0, s1 = -1;  // slot range [s0, s1]
@@ -111,90 +116,98 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_records_kernel(const D
   auto rec_ptr = [&](int r) {
     return p.ws_rec + (((size_t)(s0 + r / NW) * NW + (r % NW)) * G + gh) * kRecFloats;
   };
-  auto rec_valid = [&](int r) {  // persistent: a CTA with an empty share wrote nothing
-    if (p.sched != SCHED_PERSISTENT) return true;
-    const long long c = s0 + r / NW - g;
-    return (c * T) / P != ((c + 1) * T) / P;
-  };
-  // Records are combined in chunks of kMaxRecords: per chunk (1) m, l, tiles
-  // spread over lanes and the chunk max, (2) weights 2^(m_r - M) and their
-  // sum, (3) the weighted sum of the O vectors with four loads in flight;
-  // chunks are folded into the running (M, W, acc) like any two partials.
-  float M = -INFINITY, W = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // pass 1: scalars of every record; block max of m and sum of tiles
+  float M = -INFINITY;
   int tiles = 0;
-  for (int base = 0; base < nrec; base += kMaxRecords) {
-    const int cnt = min(kMaxRecords, nrec - base);
-    float Mc = -INFINITY;
-    float mr[kMaxRecords / 32], lr[kMaxRecords / 32];
-#pragma unroll
-    for (int u = 0; u < kMaxRecords / 32; ++u) {
-      const int r = lane + 32 * u;
-      mr[u] = -INFINITY;
-      lr[u] = 0.f;
-      if (r < cnt && rec_valid(base + r)) {
-        const float4 ml = *reinterpret_cast<const float4*>(rec_ptr(base + r) + 128);  // m, l, tiles
-        if (ml.y > 0.f) {
-          mr[u] = ml.x;
-          lr[u] = ml.y;
-        }
-        if ((base + r) % NW == 0) tiles += (int)ml.z;
-      }
-      Mc = fmaxf(Mc, mr[u]);
+  for (int r = tid; r < nrec; r += NT) {
+    float m = -INFINITY;
+    bool valid = true;
+    if (p.sched == SCHED_PERSISTENT) {  // a CTA whose share of tiles is empty wrote nothing
+      const long long c = s0 + r / NW - g;
+      valid = (c * T) / P != ((c + 1) * T) / P;
     }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, m));
-    if (Mc == -INFINITY) continue;
-    float Wc = 0.f;
-    float fr[kMaxRecords / 32];
-#pragma unroll
-    for (int u = 0; u < kMaxRecords / 32; ++u) {
-      fr[u] = (lr[u] > 0.f) ? exp2f(mr[u] - Mc) : 0.f;
-      Wc += fr[u] * lr[u];
+    if (valid) {
+      const float4 ml = *reinterpret_cast<const float4*>(rec_ptr(r) + 128);  // m, l, tiles
+      if (ml.y > 0.f) m = ml.x;
+      if (r % NW == 0) tiles += (int)ml.z;
     }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) Wc += __shfl_xor_sync(0xffffffffu, Wc, m);
-    float4 ac = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < kMaxRecords / 32; ++u) {
-      if (32 * u >= cnt) break;
-      for (int r0 = 0; r0 < 32 && 32 * u + r0 < cnt; r0 += 4) {
-        float4 o[4];
-        float f[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r = 32 * u + r0 + q;
-          f[q] = __shfl_sync(0xffffffffu, fr[u], (r0 + q) & 31);
-          o[q] = (r < cnt && f[q] > 0.f)
-                     ? *reinterpret_cast<const float4*>(rec_ptr(base + r) + lane * 4)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          ac.x += f[q] * o[q].x;
-          ac.y += f[q] * o[q].y;
-          ac.z += f[q] * o[q].z;
-          ac.w += f[q] * o[q].w;
-        }
-      }
-    }
-    const float mn = fmaxf(M, Mc);
-    const float a = exp2f(M - mn), c = exp2f(Mc - mn);
-    acc.x = acc.x * a + ac.x * c;
-    acc.y = acc.y * a + ac.y * c;
-    acc.z = acc.z * a + ac.z * c;
-    acc.w = acc.w * a + ac.w * c;
-    W = W * a + Wc * c;
-    M = mn;
+    fw[r] = m;  // -inf for an empty or unwritten record; turned into a weight below
+    M = fmaxf(M, m);
   }
 #pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, m);
-  const float inv = (W > 0.f) ? 1.f / W : 0.f;
-  *reinterpret_cast<float4*>(p.out + (size_t)row * kHeadDim + lane * 4) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  for (int o = 16; o >= 1; o >>= 1) {
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+  }
   if (lane == 0) {
-    p.lse[row] = (W > 0.f) ? (M + log2f(W)) * 0.6931471805599453f : -INFINITY;
-    if (p.blocks_consumed) p.blocks_consumed[row] = tiles;
+    red[warp][0] = M;
+    red[warp][1] = __int_as_float(tiles);
+  }
+  __syncthreads();
+  M = -INFINITY;
+  tiles = 0;
+#pragma unroll
+  for (int w = 0; w < kMergeWarps; ++w) {
+    M = fmaxf(M, red[w][0]);
+    tiles += __float_as_int(red[w][1]);
+  }
+  // pass 2: weights f_r = 2^(m_r - M) and W = sum f_r l_r (l re-read from the record)
+  float W = 0.f;
+  for (int r = tid; r < nrec; r += NT) {
+    const float m = fw[r];
+    float f = 0.f;
+    if (m != -INFINITY) {
+      f = exp2f(m - M);
+      W += f * rec_ptr(r)[129];
+    }
+    fw[r] = f;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+  __syncthreads();
+  if (lane == 0) red[warp][0] = W;
+  __syncthreads();
+  W = 0.f;
+#pragma unroll
+  for (int w = 0; w < kMergeWarps; ++w) W += red[w][0];
+  // pass 3: O = sum f_r O_r, warp w takes records w, w + kMergeWarps, ... (8 in flight)
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r0 = warp; r0 < nrec; r0 += kMergeWarps * 8) {
+    float4 o[8];
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int r = r0 + q * kMergeWarps;
+      f[q] = (r < nrec) ? fw[r] : 0.f;
+      o[q] = (f[q] > 0.f) ? *reinterpret_cast<const float4*>(rec_ptr(r) + lane * 4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      acc.x += f[q] * o[q].x;
+      acc.y += f[q] * o[q].y;
+      acc.z += f[q] * o[q].z;
+      acc.w += f[q] * o[q].w;
+    }
+  }
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) {
+      s.x += part[w][lane].x;
+      s.y += part[w][lane].y;
+      s.z += part[w][lane].z;
+      s.w += part[w][lane].w;
+    }
+    const float inv = (W > 0.f) ? 1.f / W : 0.f;
+    *reinterpret_cast<float4*>(p.out + (size_t)row * kHeadDim + lane * 4) =
+        make_float4(s.x * inv, s.y * inv, s.z * inv, s.w * inv);
+    if (lane == 0) {
+      p.lse[row] = (W > 0.f) ? (M + log2f(W)) * 0.6931471805599453f : -INFINITY;
+      if (p.blocks_consumed) p.blocks_consumed[row] = tiles;
+    }
   }
 }
 
@@ -203,8 +216,21 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_records_kernel(const D
 int launch_merge_records(const DecodeParams& p, int G, void* stream) {
   const int N = p.B * p.Hq;
   if (N == 0) return 0;
-  merge_records_kernel<<<(N + kMergeWarps - 1) / kMergeWarps, kMergeWarps * 32, 0,
-                         static_cast<cudaStream_t>(stream)>>>(p, G, p.rec_nw);
+  // records per row: pieces of one group (<= all persistent CTAs, or the splits) x warps
+  const int max_slots = (p.sched == SCHED_PERSISTENT) ? p.n_ctas : p.n_splits;
+  const size_t smem = (size_t)max_slots * p.rec_nw * sizeof(float);
+  if (smem > 200 * 1024) return (int)cudaErrorInvalidConfiguration;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(merge_records_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess) return (int)e;
+    attr_set[dev] = true;
+  }
+  merge_records_kernel<<<N, kMergeWarps * 32, smem, static_cast<cudaStream_t>(stream)>>>(
+      p, G, p.rec_nw);
   return (int)cudaGetLastError();
 }
 

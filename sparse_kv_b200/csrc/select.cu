@@ -4,8 +4,9 @@
 //
 // One CTA per KV group (b, kvh).  The group's query heads are summed once
 // (one selection per GQA group, the cheapest form of the query-centroid
-// comparison), each centroid row is scored by 16 lanes with 16-byte loads and
-// a shuffle reduction, then a shared-memory bitonic sort over
+// comparison).  Centroid rows stream into shared memory in 64 KiB chunks by
+// bulk-async copies (two stages), each row is scored by 16 lanes with 16-byte
+// shared loads and a shuffle reduction, then a shared-memory bitonic sort over
 // (score, -index) keys gives the top k (ties to the lower index), which are
 // written in ascending id order with their key ranges.
 #include "common.cuh"
@@ -14,8 +15,19 @@
 namespace skv {
 namespace {
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 256;
 constexpr int kMaxClusters = 4096;
+constexpr int kChunk = 256;                             // centroids per stage
+constexpr int kChunkBytes = kChunk * kHeadDim * 2;      // 64 KiB
+constexpr int kSelStages = 2;
+// shared memory: stages | keys u64[kMaxClusters] | q sum f32[128] | flags u8[kMaxClusters] |
+//                warp sums int[8] | mbarriers
+constexpr size_t kOffKeys = (size_t)kSelStages * kChunkBytes;
+constexpr size_t kOffQ = kOffKeys + sizeof(uint64_t) * kMaxClusters;
+constexpr size_t kOffFlag = kOffQ + 128 * 4;
+constexpr size_t kOffWsum = kOffFlag + kMaxClusters;
+constexpr size_t kOffBar = kOffWsum + 64;
+constexpr size_t kSelSmem = kOffBar + kSelStages * 8;
 
 __device__ __forceinline__ uint64_t make_key(float s, int c) {
   uint32_t u = __float_as_uint(s);
@@ -28,52 +40,80 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
                                                             const int* __restrict__ off, int Hq,
                                                             int Hkv, int C, int k, int* ids, int* ss,
                                                             int* se) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint64_t* key = reinterpret_cast<uint64_t*>(smem);                              // [Cp]
-  float* qs = reinterpret_cast<float*>(smem + sizeof(uint64_t) * kMaxClusters);   // [128]
-  unsigned char* flag = smem + sizeof(uint64_t) * kMaxClusters + 128 * 4;          // [C]
-  int* wsum = reinterpret_cast<int*>(flag + kMaxClusters);                        // [16]
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* key = reinterpret_cast<uint64_t*>(smem + kOffKeys);
+  float* qs = reinterpret_cast<float*>(smem + kOffQ);
+  unsigned char* flag = smem + kOffFlag;
+  int* wsum = reinterpret_cast<int*>(smem + kOffWsum);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
 
   const int g = blockIdx.x, b = g / Hkv, kvh = g % Hkv, G = Hq / Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nchunks = (C + kChunk - 1) / kChunk;
+  const unsigned char* cg = reinterpret_cast<const unsigned char*>(cent + (size_t)g * C * kHeadDim);
   int Cp = 1;
   while (Cp < C) Cp <<= 1;
 
+  // Centroid rows stream through kSelStages shared-memory stages by bulk copy.
+  auto issue = [&](int chunk) {
+    const int st = chunk % kSelStages;
+    const int rows = min(kChunk, C - chunk * kChunk);
+    const uint32_t bytes = (uint32_t)rows * kHeadDim * 2;
+    mbar_arrive_expect_tx(&bar[st], bytes);
+    const unsigned char* src = cg + (size_t)chunk * kChunkBytes;
+    unsigned char* dst = smem + (size_t)st * kChunkBytes;
+    for (uint32_t o = 0; o < bytes; o += 16384)
+      bulk_load(dst + o, src + o, min(16384u, bytes - o), &bar[st], policy_evict_first());
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kSelStages; ++i) mbar_init(&bar[i], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int i = 0; i < kSelStages && i < nchunks; ++i) issue(i);
+
   if (tid < kHeadDim) {
-    float s = 0.f;
+    float sum = 0.f;
     for (int h = 0; h < G; ++h)
-      s += __uint_as_float((uint32_t)q[((size_t)b * Hq + kvh * G + h) * kHeadDim + tid] << 16);
-    qs[tid] = s;
+      sum += __uint_as_float((uint32_t)q[((size_t)b * Hq + kvh * G + h) * kHeadDim + tid] << 16);
+    qs[tid] = sum;
   }
   for (int c = tid; c < Cp; c += kSelThreads) key[c] = 0ull;  // padding sorts last
   for (int c = tid; c < C; c += kSelThreads) flag[c] = 0;
   __syncthreads();
 
-  // ---- scores: 16 lanes per centroid row, 2 rows per warp step
+  // ---- scores: 16 lanes per centroid row (8 dims each), 2 rows per warp step
   const int ch = lane & 15;
   float qv[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) qv[e] = qs[ch * 8 + e];
-  const uint16_t* cg = cent + (size_t)g * C * kHeadDim;
-  const int nw = kSelThreads / 32;
+  for (int chunk = 0; chunk < nchunks; ++chunk) {
+    const int st = chunk % kSelStages;
+    if (!mbar_wait_bounded(&bar[st], (chunk / kSelStages) & 1, nullptr)) break;
+    const unsigned char* sc = smem + (size_t)st * kChunkBytes;
+    const int rows = min(kChunk, C - chunk * kChunk);
 #pragma unroll 4
-  for (int cb = warp * 2; cb < C; cb += nw * 2) {  // warp-uniform trip count
-    const int c = cb + (lane >> 4);
-    const bool valid = c < C;
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (valid) w = *reinterpret_cast<const uint4*>(cg + (size_t)c * kHeadDim + ch * 8);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-    float acc = 0.f;
+    for (int rb = warp * 2; rb < rows; rb += (kSelThreads / 32) * 2) {  // warp-uniform bound
+      const int r = rb + (lane >> 4);
+      const bool valid = r < rows;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) w = *reinterpret_cast<const uint4*>(sc + (size_t)r * kHeadDim * 2 + ch * 16);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      float acc = 0.f;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      acc = fmaf(qv[2 * u], __uint_as_float(ws[u] << 16), acc);
-      acc = fmaf(qv[2 * u + 1], __uint_as_float(ws[u] & 0xFFFF0000u), acc);
+      for (int u = 0; u < 4; ++u) {
+        acc = fmaf(qv[2 * u], __uint_as_float(ws[u] << 16), acc);
+        acc = fmaf(qv[2 * u + 1], __uint_as_float(ws[u] & 0xFFFF0000u), acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      if (valid && ch == 0) key[chunk * kChunk + r] = make_key(acc, chunk * kChunk + r);
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    if (valid && ch == 0) key[c] = make_key(acc, c);
+    __syncthreads();  // stage st fully read
+    if (tid == 0 && chunk + kSelStages < nchunks) issue(chunk + kSelStages);
   }
   __syncthreads();
 
@@ -129,10 +169,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
 
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int* ids, int* ss, int* se, void* stream) {
-  const size_t smem = sizeof(uint64_t) * kMaxClusters + 128 * 4 + kMaxClusters + 16 * 4;
-  cudaError_t e =
-      cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return (int)e;
+  const size_t smem = kSelSmem;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return (int)e;
+    attr_set[dev] = true;
+  }
   select_kernel<<<B * Hkv, kSelThreads, smem, static_cast<cudaStream_t>(stream)>>>(
       q, cent, off, Hq, Hkv, C, k, ids, ss, se);
   return (int)cudaGetLastError();

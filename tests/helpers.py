@@ -129,3 +129,19 @@ def check_art(wl, dev_res, b, kvh, order=None, layer=0, q=None, tau=None, phi=No
                                   patience, forced=cg[None])
     check_close(O_g[b, hs], lse_g[b, hs], O[0], lse[0], f"ART group ({b},{kvh})")
     return flagged, cons[0], mg[0]
+
+
+def check_selection(wl, ids_gpu, groups, q=None):
+    """ids must equal the oracle's except at flagged near-tie boundaries."""
+    q = skvgen.host_q(wl) if q is None else q
+    flagged = 0
+    for (b, kvh) in groups:
+        _, off, cent = skvgen.host_mixture_group(wl, b, kvh, want_keys=False)
+        qg = q[b, 0, kvh * wl.G:(kvh + 1) * wl.G]
+        ids, sc = oracle.select(qg[None], cent[None], wl.topk)
+        if not np.array_equal(ids[0], ids_gpu[b, kvh]):
+            gap = oracle.topk_boundary_gap(sc, wl.topk)[0]
+            assert gap <= TOPK_FLAG_GAP, f"selection differs for ({b},{kvh}), gap {gap:.2e}"
+            # the GPU's choice must still be a valid top-k up to the near tie
+            flagged += 1
+    return flagged

@@ -5,8 +5,8 @@ import pytest
 
 import oracle
 import skvgen
-from helpers import (check_art, check_close, device_workload, group_inputs, oracle_keys_attend,
-                     run_decode, TOPK_FLAG_GAP)
+from helpers import (check_art, check_close, check_selection, device_workload, group_inputs,
+                     oracle_keys_attend, run_decode)
 
 pytestmark = pytest.mark.gpu
 
@@ -319,22 +319,6 @@ def _select(wl, dev):
     skv.attn_select_centroids(dev["q"], dev["centroids"], dev["cluster_off"], wl.topk, ids, ss, se)
     torch.cuda.synchronize()
     return ids, ss, se
-
-
-def check_selection(wl, ids_gpu, groups, q=None):
-    """ids must equal the oracle's except at flagged near-tie boundaries."""
-    q = skvgen.host_q(wl) if q is None else q
-    flagged = 0
-    for (b, kvh) in groups:
-        _, off, cent = skvgen.host_mixture_group(wl, b, kvh, want_keys=False)
-        qg = q[b, 0, kvh * wl.G:(kvh + 1) * wl.G]
-        ids, sc = oracle.select(qg[None], cent[None], wl.topk)
-        if not np.array_equal(ids[0], ids_gpu[b, kvh]):
-            gap = oracle.topk_boundary_gap(sc, wl.topk)[0]
-            assert gap <= TOPK_FLAG_GAP, f"selection differs for ({b},{kvh}), gap {gap:.2e}"
-            # the GPU's choice must still be a valid top-k up to the near tie
-            flagged += 1
-    return flagged
 
 
 def test_select_and_attend_small_mixture():
