@@ -44,6 +44,13 @@ def parse():
     return ap.parse_args()
 
 
+def tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return json.load(open(p))["bf16_tflops_sustained"], "measured sustained bf16"
+    return 1400.0, "fallback sustained bf16"
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -338,6 +345,43 @@ def build_routed(torch, skv, skvgen, wl, status):
     return step
 
 
+def build_chunk(torch, skv, skvgen, wl, status):
+    """Query chunk of Tq tokens: 8 context shards (one launch, one partial per
+    shard), the chunk's own keys under a causal mask, and the exact merge."""
+    q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, wl)
+    skvgen.device_kv_paged(wl, q, k_pool, v_pool, bt, sl)
+    ctx, S = wl.L - wl.chunk, wl.shards
+    parts_o = torch.empty((S + 1, wl.B, wl.Tq, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
+    parts_l = torch.empty((S + 1, wl.B, wl.Tq, wl.Hq), dtype=torch.float32, device="cuda")
+    N = wl.B * wl.Tq * wl.Hq
+    out = torch.empty((N, wl.d), dtype=torch.float32, device="cuda")
+    lse = torch.empty(N, dtype=torch.float32, device="cuda")
+    kw = dict(max_seq_len=wl.Lmax, scale=wl.scale, status=status)
+    a_ctx = skv.make_decode_args(q, k_pool, v_pool, bt, sl, parts_o[:S], parts_l[:S],
+                                 kv_range=(0, ctx), kv_shards=S, **kw)
+    a_tail = skv.make_decode_args(q, k_pool, v_pool, bt, sl, parts_o[S:], parts_l[S:],
+                                  kv_range=(ctx, wl.L), causal=True, **kw)
+    L = skv.lib()
+    po, pl_, op, lp = (ctypes.c_void_p(t.data_ptr()) for t in (parts_o, parts_l, out, lse))
+
+    def run():
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        for a in (a_ctx, a_tail):
+            st = L.attn_decode(ctypes.byref(a), stream)
+            if st != 0:
+                raise skv.SkvError(st, "attn_decode")
+        st = L.attn_merge_lse(po, pl_, S + 1, N, wl.d, op, lp, stream)
+        if st != 0:
+            raise skv.SkvError(st, "attn_merge_lse")
+
+    rows = wl.B * wl.Hq * wl.Tq
+    flops = 4.0 * wl.d * rows * ctx + 4.0 * wl.d * wl.B * wl.Hq * (wl.Tq * (wl.Tq + 1) // 2)
+    step = Step(run, wl.kv_bytes(), 3, {"flop": flops, "shards": S, "chunk_tokens": wl.Tq})
+    step.tensors = dict(q=q, k_pool=k_pool, v_pool=v_pool, bt=bt, sl=sl, parts_o=parts_o,
+                        parts_l=parts_l, out=out, lse=lse)
+    return step
+
+
 np = None
 
 
@@ -372,6 +416,8 @@ def main():
         step = build_select(torch, skv, skvgen, wl, status)
     elif kind == "cfg5":
         step = build_routed(torch, skv, skvgen, wl, status)
+    elif kind == "cfg4":
+        step = build_chunk(torch, skv, skvgen, wl, status)
     else:
         raise SystemExit(f"workload {args.workload}: no bench step")
     art_step = build_decode(torch, skv, skvgen, wl, status, art=True) if (kind == "cfg2" and not args.no_art) else None
@@ -486,6 +532,13 @@ def main():
     }
     if step.extra:
         res["step_detail"] = step.extra
+    if kind == "cfg4":  # a dense contraction: tensor-core roofline (sustained bf16 peak)
+        tf = step.extra["flop"] / (per_launch_ms * 1e-3) / 1e12
+        peak_tf, tf_kind = tensor_peak()
+        res["metric_tflops"] = step.extra["flop"] * world / (ms_step * 1e-3) / 1e12
+        res["roofline"] = {"bound": "tensor", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
+                           "frac": tf / peak_tf, "peak_kind": tf_kind, "traffic": None,
+                           "kernel": "one step: chunk kernel x2 + merge"}
     if kind in ("cfg1", "cfg2"):
         res["config"]["traversal"] = "full"
     if art_ms is not None:

@@ -43,7 +43,11 @@
  *    status_word is non-NULL; the affected rows are computed as if the bad
  *    entry were absent.  The caller reads the word back after synchronising.
  *  - Supported shapes: head_dim 128, block_size 64, q_heads / kv_heads in
- *    {1, 2, 4, 8}, q_tokens == 1.  Other values return SKV_EUNSUPPORTED.
+ *    {1, 2, 4, 8}.  q_tokens == 1 is decode (all options below); q_tokens > 1
+ *    is a query chunk computed on the tensor cores (tcgen05): natural
+ *    traversal or a [kv_begin, kv_end) range starting on a 64-token block,
+ *    optional causal mask over the chunk's own keys, optional equal shards;
+ *    no ART, order, window or segments.  Other values return SKV_EUNSUPPORTED.
  *  - Alignment: q, out, k_pool and v_pool 16-byte aligned.
  */
 #ifndef SPARSEKV_H
@@ -133,6 +137,12 @@ typedef struct {
   float scale;      /* softmax scale, e.g. 1/sqrt(head_dim) */
   skv_art art;
   skv_window window;
+  int causal;       /* q_tokens > 1: the chunk's own keys are the last q_tokens tokens of
+                       each sequence; query token t sees positions <= seq_len - q_tokens + t */
+  int kv_shards;    /* q_tokens > 1: split [kv_begin, kv_end) (or the whole sequence) into
+                       this many equal shards and write one partial per shard: out and lse
+                       gain a leading [kv_shards] dimension ("Pulsar Attention" Phase 2
+                       local attention per host); 0 or 1 = a single result */
   float* out;               /* fp32 [batch][q_tokens][q_heads][head_dim] */
   float* lse;               /* fp32 [batch][q_tokens][q_heads], natural log of sum exp(scale q.k);
                                -inf (with out = 0) when no key is attended */

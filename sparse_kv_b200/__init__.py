@@ -40,7 +40,8 @@ class DecodeArgs(ctypes.Structure):
         ("batch", _i), ("q_tokens", _i), ("q_heads", _i), ("kv_heads", _i), ("head_dim", _i),
         ("block_size", _i), ("max_blocks", _i), ("num_pages", _i), ("max_seq_len", _i),
         ("kv_begin", _i), ("kv_end", _i), ("scale", ctypes.c_float), ("art", _Art),
-        ("window", _Window), ("out", _p), ("lse", _p), ("blocks_consumed", _p),
+        ("window", _Window), ("causal", _i), ("kv_shards", _i), ("out", _p), ("lse", _p),
+        ("blocks_consumed", _p),
         ("status_word", _p), ("workspace", _p), ("workspace_bytes", ctypes.c_size_t),
     ]
 
@@ -97,13 +98,14 @@ def _stream(stream):
 
 def make_decode_args(q, k_pool, v_pool, block_table, seq_lens, out, lse, *, max_seq_len,
                      scale=None, order=None, segments=None, window=None, kv_range=None, art=None,
-                     blocks_consumed=None, status=None, workspace=None):
+                     causal=False, kv_shards=0, blocks_consumed=None, status=None, workspace=None):
     """Fill a DecodeArgs from tensors.
 
     q [B, Tq, Hq, 128] bf16; k_pool/v_pool [P, Hkv, 64, 128] bf16; block_table [B, MB]
     int32; seq_lens [B] int32; out [B, Tq, Hq, 128] fp32; lse [B, Tq, Hq] fp32.
     order: int32 [B, Hkv, n]; segments: (start, end) int32 [B, Hkv, n] each;
-    window: (sink, recent); kv_range: (begin, end); art: (tau, phi, patience)."""
+    window: (sink, recent); kv_range: (begin, end); art: (tau, phi, patience);
+    causal / kv_shards: query chunks (q_tokens > 1), see include/sparsekv.h."""
     B, Tq, Hq, d = q.shape
     P, Hkv, bs, d2 = k_pool.shape
     a = DecodeArgs()
@@ -124,6 +126,8 @@ def make_decode_args(q, k_pool, v_pool, block_table, seq_lens, out, lse, *, max_
         a.kv_begin, a.kv_end = int(kv_range[0]), int(kv_range[1])
     if art is not None:
         a.art = _Art(1, float(art[0]), float(art[1]), int(art[2]))
+    a.causal = 1 if causal else 0
+    a.kv_shards = int(kv_shards)
     a.out, a.lse = _ptr(out), _ptr(lse)
     a.blocks_consumed = _ptr(blocks_consumed)
     a.status_word = _ptr(status)

@@ -16,6 +16,7 @@ namespace {
 
 struct Plan {
   int G = 0;
+  bool chunk = false;
   int mode = TRAV_NATURAL;
   bool art = false;
   int sched = SCHED_GROUP;
@@ -62,7 +63,7 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
   if (!isfinite(a->scale)) return SKV_EINVAL;
   const int G = a->q_heads / a->kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return SKV_EUNSUPPORTED;
-  if (a->q_tokens != 1) return SKV_EUNSUPPORTED;
+  if (a->kv_shards < 0) return SKV_EINVAL;
 
   const bool has_order = a->order != nullptr;
   const bool has_seg = a->seg_start != nullptr || a->seg_end != nullptr;
@@ -77,6 +78,16 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     if (!(a->art.tau >= 0.f) || !(a->art.phi >= 0.f) || a->art.patience < 1) return SKV_EINVAL;
     if (has_seg || has_win || has_range) return SKV_EUNSUPPORTED;
   }
+  if (a->q_tokens > 1) {  // query chunk on the tensor cores
+    if (a->art.enable || has_order || has_seg || has_win) return SKV_EUNSUPPORTED;
+    pl->G = G;
+    pl->chunk = true;
+    pl->art = false;
+    pl->mode = TRAV_NATURAL;
+    pl->ws_bytes = 0;
+    return SKV_OK;
+  }
+  if (a->kv_shards > 1) return SKV_EUNSUPPORTED;  // decode: one result (use kv ranges)
 
   pl->G = G;
   pl->art = a->art.enable != 0;
@@ -177,6 +188,10 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
     p.ws_rec = reinterpret_cast<float*>(static_cast<char*>(a->workspace) + pl.hdr_bytes);
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (pl.chunk) {
+    if (launch_chunk(p, a->q_tokens, a->causal, a->kv_shards, s) != 0) return SKV_ECUDA;
+    return SKV_OK;
+  }
   if (launch_decode(p, pl.G, pl.art, s) != 0) return SKV_ECUDA;
   if (!pl.art && launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
   return SKV_OK;

@@ -116,6 +116,11 @@ __device__ __forceinline__ void unpack2(f2 x, float& a, float& b) {
 __device__ __forceinline__ void ffma2(f2& acc, f2 a, f2 b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc.v) : "l"(a.v), "l"(b.v));
 }
+__device__ __forceinline__ f2 fadd2(f2 a, f2 b) {
+  f2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
 __device__ __forceinline__ f2 fmul2(f2 a, f2 b) {
   f2 r;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));

@@ -84,6 +84,7 @@ int decode_ctas_per_sm(int G, bool art);
 int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int d, float* out,
                  float* lse, void* stream);
 int launch_merge_records(const DecodeParams& p, int G, void* stream);
+int launch_chunk(const DecodeParams& p, int Tq, int causal, int n_shards, void* stream);
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int* ids, int* ss, int* se, void* stream);
 int num_sms();

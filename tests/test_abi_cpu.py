@@ -68,7 +68,10 @@ def status(a):
     (dict(q_heads=24), skv.SKV_EUNSUPPORTED),      # GQA group of 3
     (dict(head_dim=64), skv.SKV_EUNSUPPORTED),
     (dict(block_size=32), skv.SKV_EUNSUPPORTED),
-    (dict(q_tokens=2), skv.SKV_EUNSUPPORTED),
+    (dict(q_tokens=2, art=_Art(1, 1e-3, 1e-4, 4)), skv.SKV_EUNSUPPORTED),  # chunk + ART
+    (dict(q_tokens=2, window=_Window(64, 4096)), skv.SKV_EUNSUPPORTED),   # chunk + window
+    (dict(kv_shards=-1), skv.SKV_EINVAL),
+    (dict(kv_shards=4), skv.SKV_EUNSUPPORTED),                            # shards need a chunk
     (dict(q=FAKE + 8), skv.SKV_EINVAL),            # misaligned
     (dict(k_pool=FAKE + 4), skv.SKV_EINVAL),
     (dict(max_blocks=100), skv.SKV_EINVAL),        # table narrower than max_seq_len
