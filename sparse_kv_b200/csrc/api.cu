@@ -19,12 +19,15 @@ struct Plan {
   bool chunk = false;
   int mode = TRAV_NATURAL;
   bool art = false;
-  int sched = SCHED_GROUP;
+  int sched = SCHED_PERSISTENT;
   int n_ctas = 0;
   int splits = 1;
   int nw = 0;
-  size_t hdr_bytes = 0;
+  size_t hdr_bytes = 0;   // plain: header; ART: zeroed control words
+  size_t lb_bytes = 0;    // ART look-back records
+  size_t scratch_bytes = 0;  // ART per-CTA scratch
   size_t ws_bytes = 0;
+  int art_chunk = 0, art_maxc = 0;
 };
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -92,16 +95,31 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
   pl->G = G;
   pl->art = a->art.enable != 0;
   pl->mode = has_order ? TRAV_ORDER : has_seg ? TRAV_SEGMENTS : has_win ? TRAV_WINDOW : TRAV_NATURAL;
-  pl->nw = decode_consumer_warps(G, pl->art);
   pl->splits = 1;
   pl->n_ctas = 0;
   pl->hdr_bytes = 0;
   pl->ws_bytes = 0;
+  const long long groups = (long long)a->batch * a->kv_heads;
   if (pl->art) {
-    pl->sched = SCHED_GROUP;
+    // (chunk, group) items; one record per (group, chunk, head)
+    DecodeParams probe{};
+    probe.mode = pl->mode;
+    probe.order_len = a->order_len;
+    pl->sched = SCHED_ART;
+    pl->nw = 1;
+    pl->art_chunk = art_chunk_blocks(G);
+    pl->art_maxc = (int)cdiv(art_positions(probe, a->max_seq_len), pl->art_chunk);
+    const long long items = groups * pl->art_maxc;
+    if (items >= (1ll << 30) || pl->art_maxc > 32768) return SKV_EUNSUPPORTED;
+    pl->n_ctas = num_sms() * art_ctas_per_sm(G);
+    pl->hdr_bytes = (size_t)cdiv(art_ctl_words(groups, pl->art_maxc, G) * 4, 256) * 256;
+    pl->lb_bytes = (size_t)cdiv(items * G * kLbFloats * 4, 256) * 256;
+    pl->scratch_bytes = (size_t)pl->n_ctas * art_scratch_bytes_per_cta(G);
+    pl->ws_bytes = pl->hdr_bytes + pl->lb_bytes + pl->scratch_bytes +
+                   (size_t)items * G * kRecFloats * sizeof(float);
     return SKV_OK;
   }
-  const long long groups = (long long)a->batch * a->kv_heads;
+  pl->nw = decode_consumer_warps(G);
   long long slots = 0;
   if (pl->mode != TRAV_SEGMENTS && a->batch <= kMaxPersistentBatch) {
     DecodeParams probe{};
@@ -114,14 +132,14 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     const long long t_est = groups * group_tiles(probe, a->max_seq_len);
     if (t_est >= (1ll << 31)) return SKV_EUNSUPPORTED;
     pl->sched = SCHED_PERSISTENT;
-    const long long max_ctas = (long long)num_sms() * decode_ctas_per_sm(G, false);
+    const long long max_ctas = (long long)num_sms() * decode_ctas_per_sm(G);
     pl->n_ctas = (int)std::max<long long>(1, std::min<long long>(max_ctas, cdiv(t_est, 4)));
     slots = pl->n_ctas + groups;
     pl->hdr_bytes = (size_t)cdiv((a->batch + 2) * 4ll, 256) * 256;
   } else {
     pl->sched = SCHED_SPLIT;
     pl->splits = choose_splits(groups, pl->mode == TRAV_SEGMENTS ? a->n_seg : cdiv(a->max_seq_len, kBlock),
-                               decode_ctas_per_sm(G, false));
+                               decode_ctas_per_sm(G));
     slots = groups * pl->splits;
   }
   pl->ws_bytes = pl->hdr_bytes + (size_t)slots * pl->nw * G * kRecFloats * sizeof(float);
@@ -183,17 +201,27 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
   p.blocks_consumed = a->blocks_consumed;
   p.status = a->status_word;
   p.rec_nw = pl.nw;
-  if (!pl.art) {
-    p.ws_hdr = static_cast<int*>(a->workspace);
-    p.ws_rec = reinterpret_cast<float*>(static_cast<char*>(a->workspace) + pl.hdr_bytes);
-  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pl.chunk) {
     if (launch_chunk(p, a->q_tokens, a->causal, a->kv_shards, s) != 0) return SKV_ECUDA;
     return SKV_OK;
   }
-  if (launch_decode(p, pl.G, pl.art, s) != 0) return SKV_ECUDA;
-  if (!pl.art && launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
+  char* ws = static_cast<char*>(a->workspace);
+  if (pl.art) {
+    p.art_chunk = pl.art_chunk;
+    p.art_maxc = pl.art_maxc;
+    p.art_ctl = reinterpret_cast<int*>(ws);
+    p.art_lb = reinterpret_cast<float*>(ws + pl.hdr_bytes);
+    p.art_scratch = reinterpret_cast<float*>(ws + pl.hdr_bytes + pl.lb_bytes);
+    p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes + pl.lb_bytes + pl.scratch_bytes);
+    if (cudaMemsetAsync(ws, 0, pl.hdr_bytes, s) != cudaSuccess) return SKV_ECUDA;
+    if (launch_art(p, pl.G, s) != 0) return SKV_ECUDA;
+  } else {
+    p.ws_hdr = reinterpret_cast<int*>(ws);
+    p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes);
+    if (launch_decode(p, pl.G, s) != 0) return SKV_ECUDA;
+  }
+  if (launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
   return SKV_OK;
 }
 

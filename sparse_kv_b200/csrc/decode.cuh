@@ -16,11 +16,12 @@ enum TravMode : int {
 enum Schedule : int {
   SCHED_PERSISTENT = 0,  // one CTA per SM walks an even share of all tiles of all groups
   SCHED_SPLIT = 1,       // grid (splits, kv_heads, batch), each CTA one piece of one group
-  SCHED_GROUP = 2,       // grid (1, kv_heads, batch), one CTA walks a whole group (ART)
+  SCHED_ART = 2,         // persistent CTAs take (chunk, group) items (art.cu)
 };
 
 constexpr int kMaxPersistentBatch = 1024;  // batch prefix kept in shared memory
 constexpr int kRecFloats = 132;            // partial record: O[128], m (base 2), l, tiles, pad
+constexpr int kLbFloats = 12;              // ART look-back record per head: m, l, O[0:8], run, state
 
 struct DecodeParams {
   const uint16_t* q;
@@ -52,7 +53,32 @@ struct DecodeParams {
   int* ws_hdr;
   float* ws_rec;
   int rec_nw;
+  // ART (SCHED_ART): chunk length in blocks, chunks per group (the longest
+  // sequence's), control words zeroed before every launch (item counter, stop
+  // chunk per group, ready flag per chunk, blocks consumed and stop chunk per
+  // head) and the
+  // look-back records [group][chunk][G][kLbFloats]; ws_rec holds one record
+  // per (group, chunk, head) (rec_nw = 1).
+  int art_chunk;
+  int art_maxc;
+  int* art_ctl;
+  float* art_lb;
+  float* art_scratch;  // per-CTA probe slots and state area (stays in L2)
 };
+
+// ART traversal positions of a sequence of L tokens: block 0, then the
+// caller's list (with block 0 skipped) or the other blocks most recent first.
+__host__ __device__ inline int art_positions(const DecodeParams& p, int L) {
+  const int nb = (L + 63) / 64;
+  if (nb == 0) return 0;
+  return p.mode == TRAV_ORDER ? 1 + p.order_len : nb;
+}
+
+// Control words of the ART schedule: counter (4), stop chunk per group, ready
+// flag per chunk, blocks consumed and stop chunk per head.
+inline long long art_ctl_words(long long groups, long long maxc, int G) {
+  return 4 + groups + groups * maxc + 2 * groups * G;
+}
 
 // Tiles of one KV group for the index-based traversals (natural / range /
 // window / order), given the sequence length L.
@@ -78,9 +104,13 @@ __host__ __device__ inline int group_tiles(const DecodeParams& p, int L) {
 }
 
 // Host-side launchers (decode.cu / merge.cu / select.cu).
-int launch_decode(const DecodeParams& p, int G, bool art, void* stream);
-int decode_consumer_warps(int G, bool art);
-int decode_ctas_per_sm(int G, bool art);
+int launch_decode(const DecodeParams& p, int G, void* stream);
+int decode_consumer_warps(int G);
+int decode_ctas_per_sm(int G);
+int launch_art(const DecodeParams& p, int G, void* stream);
+int art_chunk_blocks(int G);
+int art_ctas_per_sm(int G);
+size_t art_scratch_bytes_per_cta(int G);
 int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int d, float* out,
                  float* lse, void* stream);
 int launch_merge_records(const DecodeParams& p, int G, void* stream);

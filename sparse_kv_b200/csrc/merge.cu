@@ -73,12 +73,13 @@ int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int
 }  // namespace skv
 
 // ---------------------------------------------------------------------------
-// Merge of the decode kernel's per-warp partial records (split-KV schedules).
-// Row (b, h) of group g = b*Hkv + h/G collects the records of every piece of
-// g: persistent schedule -> slots c + g for the CTAs c whose tile share meets
-// g's tiles [T_g, T_g + n_g); split schedule -> slots g*S .. g*S + S-1.  Each
-// record holds (O unnormalised, m in base 2, l, tiles); the merge is the same
-// exact online-softmax combination as above, in base 2.
+// Merge of the decode kernels' partial records.  Row (b, h) of group
+// g = b*Hkv + h/G collects the records of every piece of g: persistent
+// schedule -> slots c + g for the CTAs c whose tile share meets g's tiles
+// [T_g, T_g + n_g); split schedule -> slots g*S .. g*S + S-1; ART -> the
+// chunks of g up to the one where the row's head stopped.  Each record holds
+// (O unnormalised, m in base 2, l, tiles); the merge is the same exact
+// online-softmax combination as above, in base 2.
 // ---------------------------------------------------------------------------
 namespace skv {
 namespace {
@@ -99,7 +100,21 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_records_kernel(const D
   const int g = b * p.Hkv + kvh;
   int s0 = 0, s1 = -1;  // slot range [s0, s1]
   long long T = 0, P = p.n_ctas;
-  if (p.sched == SCHED_PERSISTENT) {
+  int art_used = 0;
+  if (p.sched == SCHED_ART) {
+    const int groups = p.B * p.Hkv;
+    const int* stop_chunk = p.art_ctl + 4;
+    const int* consumed = stop_chunk + groups + (size_t)groups * p.art_maxc;
+    const int* head_stop = consumed + (size_t)groups * G;
+    int L = p.seq_lens[b];
+    if (L < 0 || L > p.max_seq_len) L = 0;
+    int nch = (art_positions(p, L) + p.art_chunk - 1) / p.art_chunk;
+    const int sc = head_stop[(size_t)g * G + gh];  // the head's stop chunk + 1
+    if (sc != 0 && sc < nch) nch = sc;
+    s0 = g * p.art_maxc;
+    s1 = s0 + nch - 1;
+    art_used = consumed[(size_t)g * G + gh];
+  } else if (p.sched == SCHED_PERSISTENT) {
     T = p.ws_hdr[0];
     const int pb = p.ws_hdr[1 + b], pb1 = p.ws_hdr[2 + b];
     const int nt = (pb1 - pb) / p.Hkv;
@@ -206,7 +221,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_records_kernel(const D
         make_float4(s.x * inv, s.y * inv, s.z * inv, s.w * inv);
     if (lane == 0) {
       p.lse[row] = (W > 0.f) ? (M + log2f(W)) * 0.6931471805599453f : -INFINITY;
-      if (p.blocks_consumed) p.blocks_consumed[row] = tiles;
+      if (p.blocks_consumed) p.blocks_consumed[row] = (p.sched == SCHED_ART) ? art_used : tiles;
     }
   }
 }
@@ -217,7 +232,9 @@ int launch_merge_records(const DecodeParams& p, int G, void* stream) {
   const int N = p.B * p.Hq;
   if (N == 0) return 0;
   // records per row: pieces of one group (<= all persistent CTAs, or the splits) x warps
-  const int max_slots = (p.sched == SCHED_PERSISTENT) ? p.n_ctas : p.n_splits;
+  const int max_slots = (p.sched == SCHED_PERSISTENT) ? p.n_ctas
+                        : (p.sched == SCHED_ART)      ? p.art_maxc
+                                                      : p.n_splits;
   const size_t smem = (size_t)max_slots * p.rec_nw * sizeof(float);
   if (smem > 200 * 1024) return (int)cudaErrorInvalidConfiguration;
   static bool attr_set[64] = {};
