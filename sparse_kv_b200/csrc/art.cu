@@ -18,26 +18,28 @@
 //              (bulk copies, no multicast), exactly like the plain decode
 //              kernel, and ends each chunk with a marker entry;
 //   consumers  NW warps fold every block into their online-softmax states
-//              (tile.cuh) and hand the judge, through a small ring of probe
-//              slots, (m, l, O[0:8]) of their state after every block and
-//              their whole state at the end of every chunk.  They never wait
-//              for a decision;
-//   judge      one warp combines the consumer warps' probes into the chunk-
-//              local prefix after every block and the end-of-chunk states
-//              into the chunk's record; then it waits for the previous
-//              chunk's published prefix (m, l, O[0:8], run of passing tests,
-//              blocks consumed or the stop) -- a decoupled look-back, as in
-//              single-pass parallel prefix scans -- evaluates the test for all
-//              CB blocks at once (lane t: block t; the patience run by warp
-//              ballots) and publishes the inclusive prefix.
-// The probe slots and the state area are a small per-CTA scratch in global
-// memory (rewritten in place, so it stays in L2), which leaves the shared
-// memory to a 3-stage ring at two CTAs per SM.
+//              (tile.cuh) and leave (m, l, O[0:8]) of their state after every
+//              block in a per-CTA scratch area.  At the end of a chunk they
+//              meet once; each warp combines its share of the blocks into the
+//              chunk-local prefixes, writes its whole state, and posts the
+//              chunk to the judge.  They never wait for a decision;
+//   judge      one warp combines the states into the chunk's record, waits for
+//              the previous chunk's published prefix (m, l, O[0:8], run of
+//              passing tests, blocks consumed or the stop) -- a decoupled
+//              look-back, as in single-pass parallel prefix scans --
+//              evaluates the test for all CB blocks at once (lane t: block t;
+//              the patience run by warp ballots) and publishes the inclusive
+//              prefix.
+// Posts alternate between two buffers, so the consumers run a chunk ahead of
+// the judge.  The probes, states and chunk-local prefixes live in global
+// memory rewritten in place (they stay in L2), which leaves the shared memory
+// to a 3-stage ring at two
+// CTAs per SM.
 // A head that stops inside a chunk needs its state after the stop block, which
-// the consumers have already passed: the judge posts a request, and at their
-// next chunk boundary the consumers re-fold that chunk's blocks up to the stop
-// for the stopping heads straight from the pool in global memory (once per
-// head; the pages are usually still in L2); the judge overwrites the record.
+// the consumers have already passed: the judge posts a request, and at a later
+// chunk boundary the consumers re-fold that chunk's blocks up to the stop for
+// the stopping heads straight from the pool in global memory (once per head;
+// the pages are usually still in L2); the judge overwrites the record.
 // Chunks taken after every head of a group has stopped issue no loads.
 // attn_decode's merge combines each head's records up to its stop chunk,
 // which is exact.
@@ -50,7 +52,7 @@
 #define SKV_ART_WARPS 8
 #endif
 #ifndef SKV_ART_CHUNK
-#define SKV_ART_CHUNK 16
+#define SKV_ART_CHUNK 32
 #endif
 #ifndef SKV_ART_CTAS_PER_SM
 #define SKV_ART_CTAS_PER_SM 2
@@ -60,17 +62,22 @@ namespace skv {
 namespace {
 
 constexpr int kProbeFloats = 12;  // per (block, warp, head): m, l, pad, pad, O[0:8]
-constexpr int kSlots = 8;         // probe ring depth (entries the consumers may run ahead)
-constexpr int kReqs = 32;         // re-run requests in flight (at most one per chunk in the ring lag)
-enum SlotKind : int { SLOT_TILE = 0, SLOT_END = 1, SLOT_FIX = 2, SLOT_QUIT = 3, SLOT_DONE = 4 };
+constexpr int kReqs = 32;         // re-run requests in flight (a few chunks' worth)
+enum PostKind : int { POST_END = 1, POST_FIX = 2, POST_QUIT = 3, POST_DONE = 4 };
 
 constexpr size_t up16(size_t x) { return (x + 15) / 16 * 16; }
 
-// Per-CTA scratch in global memory: probe slots [kSlots][NW][G][12] and the
-// state area [NW][G][kRecFloats].
-template <int G, int NW>
+// Per-CTA scratch in global memory, two buffers (post parity): probes
+// [2][CB][NW][G][12], states [2][NW][G][kRecFloats] and chunk-local prefixes
+// [2][CB][G][12].
+template <int G, int NW, int CB>
+__host__ __device__ constexpr size_t probe_floats() {
+  return (size_t)CB * NW * G * kProbeFloats;
+}
+template <int G, int NW, int CB>
 __host__ __device__ constexpr size_t scratch_floats() {
-  return (size_t)kSlots * NW * G * kProbeFloats + (size_t)NW * G * kRecFloats;
+  return 2 * probe_floats<G, NW, CB>() + 2 * (size_t)NW * G * kRecFloats +
+         2 * (size_t)CB * G * kProbeFloats;
 }
 
 template <int G, int NW, int CB, int ST>
@@ -78,20 +85,21 @@ struct ArtCfg {  // shared-memory layout
   using Ln = Lanes<G, NW>;
   static constexpr int RPW = Ln::RPW;
   static constexpr int THREADS = (NW + 2) * 32;  // consumers, producer, judge
-  static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes;
-  static constexpr int NBAR = 2 * ST + 1 + 2 * kSlots + 1;  // full, empty, fin, pfull, pfree, sfree
+  // a stage: K rows, V rows, and the group's q rows (loaded with a chunk's first block)
+  static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes + (size_t)G * kRowBytes;
+  static constexpr int NBAR = 2 * ST + 6;  // full, empty, fin, consumer barrier, posted[2], free[2]
   static constexpr size_t OFF_BAR = ST * STAGE_BYTES;
   static constexpr size_t OFF_META = up16(OFF_BAR + NBAR * 8);        // int4 [ST]
   static constexpr size_t OFF_FLAGS = up16(OFF_META + ST * 16);       // int [4]
-  static constexpr size_t OFF_TAG = OFF_FLAGS + 16;                   // int [kSlots][4]
-  static constexpr size_t OFF_RTAG = OFF_TAG + kSlots * 16;           // int [kSlots]
-  static constexpr size_t OFF_REQ = up16(OFF_RTAG + kSlots * 4);      // int [kReqs][4] + int [kReqs][G]
+  static constexpr size_t OFF_TAG = OFF_FLAGS + 16;                   // int [2][4]
+  static constexpr size_t OFF_RTAG = OFF_TAG + 32;                    // int [2] (+ pad)
+  static constexpr size_t OFF_REQ = OFF_RTAG + 16;                    // int [kReqs][4] + int [kReqs][G]
   static constexpr size_t OFF_P = up16(OFF_REQ + kReqs * 16 + (size_t)kReqs * G * 4);  // float2 [NW][RPW][G]
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;   // float2 [NW][G]
-  static constexpr size_t OFF_LOCAL = up16(OFF_A + (size_t)NW * G * 8);  // float [CB][G][12]
-  static constexpr size_t TOTAL = OFF_LOCAL + (size_t)CB * G * kProbeFloats * 4;
+  static constexpr size_t OFF_WCTL = up16(OFF_A + (size_t)NW * G * 8);  // int [NW][8]
+  static constexpr size_t TOTAL = OFF_WCTL + (size_t)NW * 8 * 4;
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_P % 16 == 0, "alignment");
-  static_assert(OFF_A % 16 == 0 && OFF_LOCAL % 16 == 0, "alignment");
+  static_assert(OFF_A % 16 == 0 && OFF_WCTL % 16 == 0, "alignment");
   static_assert(OFF_TAG % 16 == 0 && OFF_REQ % 16 == 0, "alignment");
   static_assert((RPW * G * 8) % 16 == 0 || G == 1, "pbuf rows");
   static_assert(CB >= 1 && CB <= 32, "one judge lane per block of a chunk");
@@ -148,20 +156,20 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + ST;
   uint64_t* fin_bar = empty + ST;
-  uint64_t* pfull = fin_bar + 1;      // [kSlots], one arrival per consumer warp
-  uint64_t* pfree = pfull + kSlots;   // [kSlots], the judge's arrival
-  uint64_t* sfree = pfree + kSlots;   // the judge has read the state area
+  uint64_t* cbar = fin_bar + 1;     // consumer warps meet at the end of a chunk
+  uint64_t* posted = cbar + 1;      // [2] a post is ready (one arrival per consumer warp)
+  uint64_t* freed = posted + 2;     // [2] the judge is done with a post
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows | 0 = end of chunk, group, chunk, block in chunk | blocks}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   // flags[1]: abort (a bounded wait expired); flags[2]: consumers finished
   // (entries consumed + 1)
-  volatile int* tag = reinterpret_cast<volatile int*>(smem + C::OFF_TAG);  // [kSlots][4]: kind, group, chunk, a
-  volatile int* rtag = reinterpret_cast<volatile int*>(smem + C::OFF_RTAG);  // requests posted, per slot
+  volatile int* tag = reinterpret_cast<volatile int*>(smem + C::OFF_TAG);    // [2][4]: kind, group, chunk, a
+  volatile int* rtag = reinterpret_cast<volatile int*>(smem + C::OFF_RTAG);  // [2] requests posted
   volatile int* req = reinterpret_cast<volatile int*>(smem + C::OFF_REQ);  // [kReqs][4]: group, chunk, vmask, stopmask
   volatile int* req_t = reinterpret_cast<volatile int*>(smem + C::OFF_REQ + kReqs * 16);  // [kReqs][G]
-  float* local = reinterpret_cast<float*>(smem + C::OFF_LOCAL);
-  float* probe = p.art_scratch + (size_t)blockIdx.x * scratch_floats<G, NW>();
-  float* state = probe + (size_t)kSlots * NW * G * kProbeFloats;
+  float* probe = p.art_scratch + (size_t)blockIdx.x * scratch_floats<G, NW, CB>();  // [2][CB][NW][G][12]
+  float* state = probe + 2 * probe_floats<G, NW, CB>();                            // [2][NW][G][132]
+  float* local = state + 2 * (size_t)NW * G * kRecFloats;                          // [2][CB][G][12]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int groups = p.B * p.Hkv;
@@ -172,11 +180,11 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       mbar_init(&empty[s], NW);
     }
     mbar_init(fin_bar, NW);
-    for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&pfull[s], NW);
-      mbar_init(&pfree[s], 1);
+    mbar_init(cbar, NW);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&posted[i], NW);
+      mbar_init(&freed[i], 1);
     }
-    mbar_init(sfree, 1);
     flags[0] = flags[1] = flags[2] = flags[3] = 0;
     fence_barrier_init();
   }
@@ -190,12 +198,14 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
 
   // ------------------------------------------------------------------ producer
   if (warp == NW) {
-    if (lane != 0) return;
+    // The whole warp looks up a chunk's pages (lane i: block i); lane 0 issues
+    // the copies.  The next item is taken one ahead, so the atomic's latency
+    // overlaps the current chunk.
     const uint64_t pol = policy_evict_first();
     const size_t head_stride = (size_t)kBlock * kHeadDim;
     int e = 0, ps = 0, round = 0;
     bool ok = true;
-    auto emit = [&](int n, int g, int c, int w, int page, int kvh) -> bool {
+    auto emit = [&](int n, int g, int c, int w, int page, int kvh, const uint16_t* qsrc) -> bool {
       if (round >= 1 && !mbar_wait_bounded(&empty[ps], (round - 1) & 1, &flags[1])) {
         fail();
         return false;
@@ -204,9 +214,11 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       if (n > 0) {
         unsigned char* sK = smem + ps * C::STAGE_BYTES;
         const size_t src = ((size_t)page * p.Hkv + kvh) * head_stride;
-        mbar_arrive_expect_tx(&full[ps], (uint32_t)n * kRowBytes * 2);
+        const uint32_t qbytes = qsrc ? (uint32_t)G * kRowBytes : 0u;
+        mbar_arrive_expect_tx(&full[ps], (uint32_t)n * kRowBytes * 2 + qbytes);
         bulk_load(sK, p.k_pool + src, (uint32_t)n * kRowBytes, &full[ps], pol);
         bulk_load(sK + kTileBytes, p.v_pool + src, (uint32_t)n * kRowBytes, &full[ps], pol);
+        if (qsrc) bulk_load(sK + 2 * kTileBytes, qsrc, qbytes, &full[ps], pol);
       } else {
         mbar_arrive(&full[ps]);
       }
@@ -218,37 +230,61 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       return true;
     };
     const long long items = (long long)groups * p.art_maxc;
-    while (ok) {
-      const long long w = atomicAdd(ctl.counter, 1);
-      if (w >= items) break;
+    long long w = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
+    w = __shfl_sync(0xffffffffu, w, 0);
+    while (ok && w < items) {
+      const long long w_next = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
       const int c = (int)(w / groups), g = (int)(w % groups);
       const int b = g / p.Hkv, kvh = g % p.Hkv;
       int L = p.seq_lens[b];
       if (L < 0 || L > p.max_seq_len) {
-        if (c == 0 && kvh == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
+        if (c == 0 && kvh == 0 && lane == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
         L = 0;
       }
       const int nb = (L + kBlock - 1) / kBlock;
       const int N = art_positions(p, L);
-      if (c * CB >= N) continue;
-      const int sc = *reinterpret_cast<volatile int*>(ctl.stop_chunk + g);
-      if (sc != 0 && c >= sc) continue;  // every head stopped in an earlier chunk
-      const int* ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)g * p.order_len : nullptr;
-      const int* bt = p.block_table + (size_t)b * p.max_blocks;
-      const int pos0 = c * CB, npos = min(CB, N - pos0);
-      for (int i = 0; i < npos && ok; ++i) {
-        const int blk = art_block(p, ord, nb, pos0 + i, p.status);
-        if (blk < 0) continue;
-        const int page = bt[blk];
-        if (page < 0 || page >= p.num_pages) {
-          dev_error(p.status, SKV_DEV_BAD_PAGE);
-          continue;
-        }
-        ok = emit(min(kBlock, L - blk * kBlock), g, c, i, page, kvh);
+      bool skip = c * CB >= N;
+      if (!skip) {
+        const int sc = *reinterpret_cast<volatile int*>(ctl.stop_chunk + g);
+        skip = sc != 0 && c >= sc;  // every head stopped in an earlier chunk
+        skip = __shfl_sync(0xffffffffu, skip, 0);
       }
-      if (ok) ok = emit(0, g, c, npos, 0, 0);  // end of chunk
+      if (!skip) {
+        const int* ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)g * p.order_len : nullptr;
+        const int* bt = p.block_table + (size_t)b * p.max_blocks;
+        const int pos0 = c * CB, npos = min(CB, N - pos0);
+        int blk = -1, n = 0, page = 0;
+        if (lane < npos) {
+          blk = art_block(p, ord, nb, pos0 + lane, p.status);
+          if (blk >= 0) {
+            page = bt[blk];
+            if (page < 0 || page >= p.num_pages) {
+              dev_error(p.status, SKV_DEV_BAD_PAGE);
+              blk = -1;
+            } else {
+              n = min(kBlock, L - blk * kBlock);
+            }
+          }
+        }
+        const uint32_t vm = __ballot_sync(0xffffffffu, blk >= 0);
+        const uint16_t* qsrc = p.q + ((size_t)b * p.Hq + (size_t)kvh * G) * kHeadDim;
+        for (int i = 0; i < npos && ok; ++i) {
+          if (!((vm >> i) & 1u)) continue;
+          const int ni = __shfl_sync(0xffffffffu, n, i), pgi = __shfl_sync(0xffffffffu, page, i);
+          int r = 1;
+          if (lane == 0) r = emit(ni, g, c, i, pgi, kvh, (vm & ((1u << i) - 1u)) ? nullptr : qsrc);
+          ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+        }
+        if (ok) {
+          int r = 1;
+          if (lane == 0) r = emit(0, g, c, npos, 0, 0, nullptr);  // end of chunk
+          ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+        }
+      }
+      w = __shfl_sync(0xffffffffu, w_next, 0);
     }
-    if (ok) emit(-1, -1, 0, 0, 0, 0);
+    if (lane != 0) return;
+    if (ok) emit(-1, -1, 0, 0, 0, 0, nullptr);
     // Copies the consumers never waited for (abort) must land before the CTA
     // exits: learn how many entries they consumed, then drain the rest.
     const uint64_t t_start = globaltimer();
@@ -263,28 +299,33 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
 
   // ------------------------------------------------------------------ judge
   if (warp == NW + 1) {
-    int kj = 0;     // probe-ring entries consumed
+    int kj = 0;     // posts consumed
     int n_req = 0;  // re-run requests posted
     int n_fix = 0;  // re-runs received back
     // combine the state area into the records of `heads` of chunk (g, c)
-    auto reduce_states = [&](int g, int c, uint32_t heads) {
+    auto reduce_states = [&](const float* st_area, int g, int c, uint32_t heads) {
       const size_t item = (size_t)g * p.art_maxc + c;
       for (int h = 0; h < G; ++h) {
         if (!((heads >> h) & 1u)) continue;
+        // every load up front: one round trip to L2
         float2 ml[NW];
-        float M = -INFINITY;
+        float4 xs[NW];
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-          ml[w] = *reinterpret_cast<const float2*>(state + (w * G + h) * kRecFloats + 128);
-          if (ml[w].y > 0.f) M = fmaxf(M, ml[w].x);
+          ml[w] = *reinterpret_cast<const float2*>(st_area + (w * G + h) * kRecFloats + 128);
+          xs[w] = *reinterpret_cast<const float4*>(st_area + (w * G + h) * kRecFloats + lane * 4);
         }
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+          if (ml[w].y > 0.f) M = fmaxf(M, ml[w].x);
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
         float Ls = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
           for (int w = 0; w < NW; ++w) {
             const float f = (ml[w].y > 0.f) ? exp2f(ml[w].x - M) : 0.f;
-            const float4 x = *reinterpret_cast<const float4*>(state + (w * G + h) * kRecFloats + lane * 4);
+            const float4 x = xs[w];
             Ls += ml[w].y * f;
             o.x += x.x * f;
             o.y += x.y * f;
@@ -296,19 +337,21 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         *reinterpret_cast<float4*>(rec + lane * 4) = o;
         if (lane == 0) *reinterpret_cast<float4*>(rec + 128) = make_float4(M, Ls, 0.f, 0.f);
       }
-      __syncwarp();
-      mbar_arrive_if(sfree, lane == 0);
     };
 
     // Look-back and the stopping rule for chunk (g, c): publishes the chunk's
     // inclusive prefix; returns the heads that stop in the chunk, their stop
-    // blocks in st_out (-1: none).
-    auto evaluate = [&](int g, int c, uint32_t vmask, int* st_out) -> uint32_t {
+    // blocks in st_out (-1: none).  SEG lanes per head (lane t: block t), so
+    // 32 / SEG heads per pass.
+    auto evaluate = [&](const float* loc, int g, int c, uint32_t vmask, int* st_out) -> uint32_t {
+      constexpr int SEG = CB <= 8 ? 8 : (CB <= 16 ? 16 : 32);
+      constexpr int HPP = 32 / SEG;
       const size_t item = (size_t)g * p.art_maxc + c;
       const int b = g / p.Hkv;
       int L = p.seq_lens[b];
       if (L < 0 || L > p.max_seq_len) L = 0;
       const int nch = (art_positions(p, L) + CB - 1) / CB;
+#pragma unroll
       for (int h = 0; h < G; ++h) st_out[h] = -1;
       // (1) the previous chunk's prefix: ready, or the group already stopped
       int lb = 1;
@@ -330,129 +373,142 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       }
       lb = __shfl_sync(0xffffffffu, lb, 0);
       if (lb == 2) return 0;  // nothing to publish: the group stopped before this chunk
-      // every head's previous record in one round trip: word k of the group at lane k % 32
-      float pw0 = 0.f, pw1 = 0.f, pw2 = 0.f;
-      if (c > 0) {
-        const float* src = p.art_lb + (item - 1) * G * kProbeFloats;
-        if (lane < G * kProbeFloats) pw0 = __ldcg(src + lane);
-        if (lane + 32 < G * kProbeFloats) pw1 = __ldcg(src + lane + 32);
-        if (lane + 64 < G * kProbeFloats) pw2 = __ldcg(src + lane + 64);
-      }
+      const int sub = lane / SEG, t = lane % SEG, base = sub * SEG;
+      const uint32_t segmask = (SEG == 32) ? 0xffffffffu : ((1u << SEG) - 1u);
       uint32_t stopmask = 0;
       bool all = true;
-      for (int h = 0; h < G; ++h) {
-        float Pv[kProbeFloats];
-#pragma unroll
-        for (int k = 0; k < kProbeFloats; ++k) {
-          const int idx = h * kProbeFloats + k;
-          const float v = __shfl_sync(0xffffffffu, idx < 32 ? pw0 : (idx < 64 ? pw1 : pw2), idx & 31);
-          Pv[k] = (c > 0) ? v : (k == 0 ? -INFINITY : 0.f);
+      for (int h0 = 0; h0 < G; h0 += HPP) {
+        const int h = h0 + sub;
+        const bool hv = h < G;
+        // previous inclusive prefix of head h: m, l, x[8], run, blocks or -(used + 1)
+        float4 P0 = make_float4(-INFINITY, 0.f, 0.f, 0.f), P1 = make_float4(0.f, 0.f, 0.f, 0.f),
+               P2 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c > 0 && hv) {
+          const float4* src = reinterpret_cast<const float4*>(p.art_lb + ((item - 1) * G + h) * kProbeFloats);
+          P0 = __ldcg(src);
+          P1 = __ldcg(src + 1);
+          P2 = __ldcg(src + 2);
         }
-        const int P_run = __float_as_int(Pv[10]), P_state = __float_as_int(Pv[11]);
-        float out[kProbeFloats];
+        const float Pm = P0.x, Pl = P0.y;
+        const float Px[8] = {P0.z, P0.w, P1.x, P1.y, P1.z, P1.w, P2.x, P2.y};
+        const int P_run = __float_as_int(P2.z), P_state = __float_as_int(P2.w);
+        const bool live = hv && P_state >= 0;
+        // chunk-local prefix after block t, then the global prefix
+        const bool valid = live && t < CB && ((vmask >> t) & 1u);
+        float M = -INFINITY, Ls = 0.f, X[8];
 #pragma unroll
-        for (int k = 0; k < kProbeFloats; ++k) out[k] = Pv[k];
-        if (P_state >= 0) {
-          // chunk-local prefix after block t (lane t), then the global prefix
-          const int t = lane;
-          const bool valid = t < CB && ((vmask >> t) & 1u);
-          float M = -INFINITY, Ls = 0.f, X[8];
+        for (int d = 0; d < 8; ++d) X[d] = 0.f;
+        if (valid) {
+          const float* q = loc + ((size_t)t * G + h) * kProbeFloats;
+          const float2 ml = *reinterpret_cast<const float2*>(q);
+          const float4 x0 = *reinterpret_cast<const float4*>(q + 4);
+          const float4 x1 = *reinterpret_cast<const float4*>(q + 8);
+          M = ml.x;
+          Ls = ml.y;
+          X[0] = x0.x; X[1] = x0.y; X[2] = x0.z; X[3] = x0.w;
+          X[4] = x1.x; X[5] = x1.y; X[6] = x1.z; X[7] = x1.w;
+        }
+        const float Mg = fmaxf(Pm, M);
+        const float fa = (Pm == -INFINITY) ? 0.f : exp2f(Pm - Mg);
+        const float fb = (M == -INFINITY) ? 0.f : exp2f(M - Mg);
+        const float Lg = Pl * fa + Ls * fb;
+        const float invL = (Lg > 0.f) ? 1.f / Lg : 0.f;
+        const float invP = (Pl > 0.f) ? 1.f / Pl : 0.f;
+        float Xg[8], xn[8], xp[8];
 #pragma unroll
-          for (int d = 0; d < 8; ++d) X[d] = 0.f;
-          if (valid) {
-            const float* q = local + ((size_t)t * G + h) * kProbeFloats;
-            M = q[0];
-            Ls = q[1];
-            const float4 x0 = *reinterpret_cast<const float4*>(q + 4);
-            const float4 x1 = *reinterpret_cast<const float4*>(q + 8);
-            X[0] = x0.x; X[1] = x0.y; X[2] = x0.z; X[3] = x0.w;
-            X[4] = x1.x; X[5] = x1.y; X[6] = x1.z; X[7] = x1.w;
-          }
-          const float Mg = fmaxf(Pv[0], M);
-          const float fa = (Pv[0] == -INFINITY) ? 0.f : exp2f(Pv[0] - Mg);
-          const float fb = (M == -INFINITY) ? 0.f : exp2f(M - Mg);
-          const float Lg = Pv[1] * fa + Ls * fb;
-          const float invL = (Lg > 0.f) ? 1.f / Lg : 0.f;
-          const float invP = (Pv[1] > 0.f) ? 1.f / Pv[1] : 0.f;
-          float Xg[8], xn[8], xp[8];
+        for (int d = 0; d < 8; ++d) {
+          Xg[d] = Px[d] * fa + X[d] * fb;
+          xn[d] = Xg[d] * invL;
+        }
+        // probe of the previous consumed block: the last valid lane below in
+        // this head's segment, else the previous prefix
+        const uint32_t below = vmask & ((1u << t) - 1u);
+        const int pl = base + (below ? 31 - __clz(below) : 0);
 #pragma unroll
-          for (int d = 0; d < 8; ++d) {
-            Xg[d] = Pv[2 + d] * fa + X[d] * fb;
-            xn[d] = Xg[d] * invL;
-          }
-          // probe of the previous consumed block: the last valid lane below,
-          // else the previous prefix
-          const uint32_t below = vmask & ((1u << t) - 1u);
-          const int pl = below ? 31 - __clz(below) : 0;
+        for (int d = 0; d < 8; ++d) {
+          const float v = __shfl_sync(0xffffffffu, xn[d], pl);
+          xp[d] = below ? v : Px[d] * invP;
+        }
+        const int gidx = P_state + __popc(below);  // consumed blocks before this one
+        float nx = 0.f, np = 0.f, dd = 0.f;
 #pragma unroll
-          for (int d = 0; d < 8; ++d) {
-            const float v = __shfl_sync(0xffffffffu, xn[d], pl);
-            xp[d] = below ? v : Pv[2 + d] * invP;
-          }
-          const int gidx = P_state + __popc(below);  // consumed blocks before this one
-          float nx = 0.f, np = 0.f, dd = 0.f;
+        for (int d = 0; d < 8; ++d) {
+          nx += xn[d] * xn[d];
+          np += xp[d] * xp[d];
+        }
+        const float a = sqrtf(nx), bp = sqrtf(np);
+        const float ia = (a > 0.f) ? 1.f / a : 0.f, ib = (bp > 0.f) ? 1.f / bp : 0.f;
 #pragma unroll
-          for (int d = 0; d < 8; ++d) {
-            nx += xn[d] * xn[d];
-            np += xp[d] * xp[d];
-          }
-          const float a = sqrtf(nx), bp = sqrtf(np);
-          const float ia = (a > 0.f) ? 1.f / a : 0.f, ib = (bp > 0.f) ? 1.f / bp : 0.f;
-#pragma unroll
-          for (int d = 0; d < 8; ++d) {
-            const float du = xn[d] * ia - xp[d] * ib;
-            dd += du * du;
-          }
-          float d_s, d_c;
-          if (bp == 0.f) d_s = (a == 0.f) ? 0.f : INFINITY;
-          else d_s = fabsf(a - bp) * ib;
-          if (a == 0.f || bp == 0.f) d_c = (a == 0.f && bp == 0.f) ? 0.f : 1.f;
-          else d_c = 0.5f * dd;  // 1 - cos(x, x') = |x/|x| - x'/|x'||^2 / 2
-          const bool pass = valid && gidx >= 1 && d_s < p.tau && d_c < p.phi;
-          const uint32_t passm = __ballot_sync(0xffffffffu, pass);
-          const uint32_t failm = __ballot_sync(0xffffffffu, valid && !pass);
-          const uint32_t upto = (2u << t) - 1u;  // lanes 0..t (wraps to all for t = 31)
-          const uint32_t ff = failm & upto;
-          int run;
-          if (ff) {
-            const int f = 31 - __clz(ff);
-            run = __popc(passm & upto & ~((2u << f) - 1u));
-          } else {
-            run = P_run + __popc(passm & upto);
-          }
-          const uint32_t stopm = __ballot_sync(0xffffffffu, valid && run >= p.patience);
-          const int total = P_state + __popc(vmask);
-          if (stopm) {
-            const int ts = __ffs(stopm) - 1;
+        for (int d = 0; d < 8; ++d) {
+          const float du = xn[d] * ia - xp[d] * ib;
+          dd += du * du;
+        }
+        float d_s, d_c;
+        if (bp == 0.f) d_s = (a == 0.f) ? 0.f : INFINITY;
+        else d_s = fabsf(a - bp) * ib;
+        if (a == 0.f || bp == 0.f) d_c = (a == 0.f && bp == 0.f) ? 0.f : 1.f;
+        else d_c = 0.5f * dd;  // 1 - cos(x, x') = |x/|x| - x'/|x'||^2 / 2
+        const bool pass = valid && gidx >= 1 && d_s < p.tau && d_c < p.phi;
+        const uint32_t passm = (__ballot_sync(0xffffffffu, pass) >> base) & segmask;
+        const uint32_t failm = (__ballot_sync(0xffffffffu, valid && !pass) >> base) & segmask;
+        const uint32_t upto = (2u << t) - 1u;  // blocks 0..t (wraps to all for t = 31)
+        const uint32_t ff = failm & upto;
+        int run;
+        if (ff) {
+          const int f = 31 - __clz(ff);
+          run = __popc(passm & upto & ~((2u << f) - 1u));
+        } else {
+          run = P_run + __popc(passm & upto);
+        }
+        const uint32_t stopm = (__ballot_sync(0xffffffffu, valid && run >= p.patience) >> base) & segmask;
+        const int total = P_state + __popc(vmask);
+        // the record of this chunk, written by one lane of the segment
+        const int ts = stopm ? __ffs(stopm) - 1 : -1;
+        const int last = vmask ? 31 - __clz(vmask) : -1;
+        float4 R0 = P0, R1 = P1, R2 = P2;  // a head stopped earlier passes its record on
+        int wl = 0;
+        if (live) {
+          if (ts >= 0) {
             const int used = P_state + __popc(vmask & ((2u << ts) - 1u));
-            out[10] = __int_as_float(0);
-            out[11] = __int_as_float(-(used + 1));
-            st_out[h] = ts;
-            stopmask |= 1u << h;
-            if (lane == 0) {
+            R2.z = __int_as_float(0);
+            R2.w = __int_as_float(-(used + 1));
+            wl = ts;
+            if (t == ts) {
               ctl.consumed[(size_t)g * G + h] = used;
               ctl.head_stop[(size_t)g * G + h] = c + 1;
             }
           } else {
-            all = false;
-            const int last = vmask ? 31 - __clz(vmask) : -1;
             if (last >= 0) {
-              out[0] = __shfl_sync(0xffffffffu, Mg, last);
-              out[1] = __shfl_sync(0xffffffffu, Lg, last);
-#pragma unroll
-              for (int d = 0; d < 8; ++d) out[2 + d] = __shfl_sync(0xffffffffu, Xg[d], last);
-              out[10] = __int_as_float(__shfl_sync(0xffffffffu, run, last));
+              wl = last;
+              R0 = make_float4(Mg, Lg, Xg[0], Xg[1]);
+              R1 = make_float4(Xg[2], Xg[3], Xg[4], Xg[5]);
+              R2 = make_float4(Xg[6], Xg[7], __int_as_float(run), __int_as_float(total));
+            } else {
+              R2.w = __int_as_float(total);
             }
-            out[11] = __int_as_float(total);
-            if (lane == 0 && c == nch - 1) ctl.consumed[(size_t)g * G + h] = total;
+            if (t == wl && c == nch - 1) ctl.consumed[(size_t)g * G + h] = total;
           }
         }
-        float* dst = p.art_lb + (item * G + h) * kProbeFloats;
-        float mine = 0.f;
+        if (hv && t == wl) {
+          float4* dst = reinterpret_cast<float4*>(p.art_lb + (item * G + h) * kProbeFloats);
+          dst[0] = R0;
+          dst[1] = R1;
+          dst[2] = R2;
+        }
+        // per-head outcome to every lane
 #pragma unroll
-        for (int k = 0; k < kProbeFloats; ++k)
-          if (lane == k) mine = out[k];
-        if (lane < kProbeFloats) dst[lane] = mine;
+        for (int s2 = 0; s2 < HPP; ++s2) {
+          const int hh = h0 + s2;
+          const int ts_h = __shfl_sync(0xffffffffu, live ? ts : -2, s2 * SEG);  // -2: stopped before
+          if (hh < G) {
+            if (ts_h >= 0) {
+              stopmask |= 1u << hh;
+              st_out[hh] = ts_h;
+            } else if (ts_h == -1) {
+              all = false;
+            }
+          }
+        }
       }
       __threadfence();
       __syncwarp();
@@ -467,50 +523,19 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     };
 
     while (true) {
-      const int slot = kj % kSlots;
-      if (!mbar_wait_bounded(&pfull[slot], (kj / kSlots) & 1, &flags[1])) {
+      const int par = kj & 1;
+      if (!mbar_wait_bounded(&posted[par], (kj >> 1) & 1, &flags[1])) {
         if (lane == 0) fail();
         break;
       }
-      const int kind = tag[slot * 4], tg_g = tag[slot * 4 + 1], tg_c = tag[slot * 4 + 2],
-                tg_a = tag[slot * 4 + 3];
-      if (kind == SLOT_TILE) {
-        // chunk-local prefix after block tg_a: combine the warps' states (lane: head, dim)
-        const float* pr = probe + (size_t)slot * NW * G * kProbeFloats;
-#pragma unroll
-        for (int r = 0; r < (G * 8 + 31) / 32; ++r) {
-          const int h = r * 4 + (lane >> 3), d = lane & 7;
-          if (h < G) {
-            float m[NW];
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-              m[w] = pr[(w * G + h) * kProbeFloats];
-              M = fmaxf(M, m[w]);
-            }
-            float Ls = 0.f, X = 0.f;
-            if (M != -INFINITY) {
-#pragma unroll
-              for (int w = 0; w < NW; ++w) {
-                const float* q = pr + (w * G + h) * kProbeFloats;
-                const float f = exp2f(m[w] - M);  // 0 for an empty warp state
-                Ls += q[1] * f;
-                X += q[4 + d] * f;
-              }
-            }
-            float* dst = local + ((size_t)tg_a * G + h) * kProbeFloats;
-            dst[4 + d] = X;
-            if (d == 0) {
-              dst[0] = M;
-              dst[1] = Ls;
-            }
-          }
-        }
-      } else if (kind == SLOT_END) {
-        reduce_states(tg_g, tg_c, (1u << G) - 1u);
-        __syncwarp();  // every lane's local prefixes are visible
+      const int kind = tag[par * 4], tg_g = tag[par * 4 + 1], tg_c = tag[par * 4 + 2],
+                tg_a = tag[par * 4 + 3];
+      const float* st_area = state + (size_t)par * NW * G * kRecFloats;
+      if (kind == POST_END) {
+        reduce_states(st_area, tg_g, tg_c, (1u << G) - 1u);
         int st[G];
-        const uint32_t stopmask = evaluate(tg_g, tg_c, (uint32_t)tg_a, st);
+        const uint32_t stopmask =
+            evaluate(local + (size_t)par * CB * G * kProbeFloats, tg_g, tg_c, (uint32_t)tg_a, st);
         if (stopmask) {
           if (n_req - n_fix >= kReqs) {
             if (lane == 0) fail();  // cannot happen: the consumers serve requests every chunk
@@ -527,16 +552,16 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
             ++n_req;
           }
         }
-      } else if (kind == SLOT_FIX) {
-        reduce_states(tg_g, tg_c, (uint32_t)tg_a);
+      } else if (kind == POST_FIX) {
+        reduce_states(st_area, tg_g, tg_c, (uint32_t)tg_a);
         ++n_fix;
       }
       __syncwarp();
-      if (lane == 0) rtag[slot] = n_req;
+      if (lane == 0) rtag[par] = n_req;
       __syncwarp();
-      mbar_arrive_if(&pfree[slot], lane == 0);
+      mbar_arrive_if(&freed[par], lane == 0);
       ++kj;
-      if (kind == SLOT_DONE) break;
+      if (kind == POST_DONE) break;
     }
     return;
   }
@@ -547,124 +572,175 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   const int rb = warp * C::RPW;
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P) + warp * C::RPW * G;
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
-  int ks = 0;          // probe-ring entries posted
-  int req_seen = 0;    // requests the judge had posted at the last slot handshake
-  int req_done = 0;    // requests served
-  int n_state = 0;     // uses of the state area
+  // Warp-uniform counters used at chunk boundaries live in shared memory (one
+  // block per warp): the fold loop is register-bound.
+  enum { W_KP = 0, W_RSEEN, W_RDONE, W_CBPH, W_DRAIN, W_CURG, W_CURC };
+  volatile int* wc = reinterpret_cast<volatile int*>(smem + C::OFF_WCTL) + warp * 8;
+  wc[W_KP] = 0;      // posts made
+  wc[W_RSEEN] = 0;   // requests the judge had posted when it freed our buffer
+  wc[W_RDONE] = 0;   // requests served
+  wc[W_CBPH] = 0;    // phase of the consumer barrier
+  wc[W_DRAIN] = 0;   // the producer's end entry has been seen
+  wc[W_CURG] = -1;   // chunk being folded
+  wc[W_CURC] = -1;
+  int kpar = 0;  // parity of the next post (its buffers hold the current chunk)
   bool ok = true;
 
-  // Post one probe-ring entry; `fill(slot)` writes this warp's part first.
-  // Every warp reads the judge's request count at the same handshake, so all
-  // take the same decisions.
-  auto post = [&](int kind, int g, int c, int a, auto&& fill) {
-    const int slot = ks % kSlots;
-    if (ks >= kSlots) {
-      if (!mbar_wait_bounded(&pfree[slot], ((ks / kSlots) - 1) & 1, &flags[1])) {
+  // Take the buffer of the next post (the judge is done with the post two
+  // back).  Every warp reads the judge's request count at the same handshake,
+  // so all take the same decisions.
+  auto acquire = [&]() {
+    const int kp = wc[W_KP];
+    if (kp >= 2) {
+      if (!mbar_wait_bounded(&freed[kp & 1], ((kp >> 1) - 1) & 1, &flags[1])) {
         if (lane == 0) fail();
         ok = false;
       }
-      req_seen = rtag[slot];
+      wc[W_RSEEN] = rtag[kp & 1];
     }
-    fill(slot);
+  };
+  auto publish = [&](int kind, int g, int c, int a) {
+    const int kp = wc[W_KP];
+    const int par = kp & 1;
     if (warp == 0 && lane == 0) {
-      tag[slot * 4] = kind;
-      tag[slot * 4 + 1] = g;
-      tag[slot * 4 + 2] = c;
-      tag[slot * 4 + 3] = a;
+      tag[par * 4] = kind;
+      tag[par * 4 + 1] = g;
+      tag[par * 4 + 2] = c;
+      tag[par * 4 + 3] = a;
     }
     __syncwarp();
-    mbar_arrive_if(&pfull[slot], lane == 0);
-    ++ks;
+    mbar_arrive_if(&posted[par], lane == 0);
+    wc[W_KP] = kp + 1;
+    kpar = (kp + 1) & 1;
   };
-  auto no_fill = [](int) {};
-  // this warp's whole state -> the state area (once the judge has read the last one)
+  // this warp's whole state -> the state area of the current post
   auto write_state = [&]() {
-    if (n_state >= 1 && !mbar_wait_bounded(sfree, (n_state - 1) & 1, &flags[1])) {
-      if (lane == 0) fail();
-      ok = false;
-    }
-    ++n_state;
+    float* st_area = state + (size_t)(wc[W_KP] & 1) * NW * G * kRecFloats;
 #pragma unroll
     for (int g2 = 0; g2 < G; ++g2) {
       float x0, x1, x2, x3;
       unpack2(W.acc[g2][0], x0, x1);
       unpack2(W.acc[g2][1], x2, x3);
-      *reinterpret_cast<float4*>(state + (warp * G + g2) * kRecFloats + lane * 4) =
+      *reinterpret_cast<float4*>(st_area + (warp * G + g2) * kRecFloats + lane * 4) =
           make_float4(x0, x1, x2, x3);
     }
     if (W.owner) {
 #pragma unroll
       for (int j = 0; j < Lanes<G, NW>::VPL; ++j)
-        *reinterpret_cast<float2*>(state + (warp * G + W.hd[j]) * kRecFloats + 128) =
+        *reinterpret_cast<float2*>(st_area + (warp * G + W.hd[j]) * kRecFloats + 128) =
             make_float2(W.m_st[j], W.l_st[j]);
+    }
+  };
+  // End of a chunk: once every warp's probes are written, this warp combines
+  // blocks warp, warp + NW, ... into the chunk-local prefixes (lane: head, dim).
+  auto merge_probes = [&](uint32_t vmask) {
+    __syncwarp();
+    mbar_arrive_if(cbar, lane == 0);
+    const int cb_ph = wc[W_CBPH];
+    if (!mbar_wait_bounded(cbar, cb_ph, &flags[1])) {
+      if (lane == 0) fail();
+      ok = false;
+    }
+    wc[W_CBPH] = cb_ph ^ 1;
+    const int par = wc[W_KP] & 1;
+    const float* pr0 = probe + (size_t)par * probe_floats<G, NW, CB>();
+    float* loc = local + (size_t)par * CB * G * kProbeFloats;
+    for (int t = warp; t < CB; t += NW) {
+      if (!((vmask >> t) & 1u)) continue;
+      const float* pr = pr0 + (size_t)t * NW * G * kProbeFloats;
+#pragma unroll
+      for (int r = 0; r < (G * 8 + 31) / 32; ++r) {
+        const int h = r * 4 + (lane >> 3), d = lane & 7;
+        if (h < G) {
+          float2 ml[NW];
+          float x[NW];
+#pragma unroll
+          for (int w = 0; w < NW; ++w) {
+            ml[w] = *reinterpret_cast<const float2*>(pr + (w * G + h) * kProbeFloats);
+            x[w] = pr[(w * G + h) * kProbeFloats + 4 + d];
+          }
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[w].x);
+          float Ls = 0.f, X = 0.f;
+          if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+              const float f = exp2f(ml[w].x - M);  // 0 for an empty warp state
+              Ls += ml[w].y * f;
+              X += x[w] * f;
+            }
+          }
+          float* dst = loc + ((size_t)t * G + h) * kProbeFloats;
+          dst[4 + d] = X;
+          if (d == 0) {
+            dst[0] = M;
+            dst[1] = Ls;
+          }
+        }
+      }
     }
   };
 
   // Re-fold of a chunk for the heads that stop in it (a request of the judge):
-  // the chunk's blocks up to each head's stop block, from the pool.
-  int rr = -1;  // request being served
-  int rr_t = 0, rr_tmax = 0, rr_g = 0, rr_c = 0, rr_L = 0, rr_nb = 0, rr_kvh = 0;
-  uint32_t rr_vm = 0, rr_stop = 0;
-  const int* rr_ord = nullptr;
-  const int* rr_bt = nullptr;
-  int rr_st[G];
+  // the chunk's blocks up to each head's stop block, from the pool.  Only the
+  // request index and the next block live in registers; the rest is re-read
+  // from the request slot (this path is rare, the fold loop is register-bound).
+  int rr = -1, rr_t = 0;
   uint32_t done_mask = 0;
   auto start_request = [&]() -> bool {
-    if (req_done >= req_seen || !ok) return false;
+    const int req_done = wc[W_RDONE];
+    if (req_done >= wc[W_RSEEN] || !ok) return false;
     rr = req_done % kReqs;
-    rr_g = req[rr * 4];
-    rr_c = req[rr * 4 + 1];
-    rr_vm = (uint32_t)req[rr * 4 + 2];
-    rr_stop = (uint32_t)req[rr * 4 + 3];
-    rr_tmax = -1;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      rr_st[h] = req_t[rr * G + h];
-      if ((rr_stop >> h) & 1u) rr_tmax = max(rr_tmax, rr_st[h]);
-    }
-    const int b = rr_g / p.Hkv;
-    rr_kvh = rr_g % p.Hkv;
-    rr_L = p.seq_lens[b];
-    if (rr_L < 0 || rr_L > p.max_seq_len) rr_L = 0;
-    rr_nb = (rr_L + kBlock - 1) / kBlock;
-    rr_ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)rr_g * p.order_len : nullptr;
-    rr_bt = p.block_table + (size_t)b * p.max_blocks;
     rr_t = 0;
+    const int g = req[rr * 4];
+    const int b = g / p.Hkv, kvh = g % p.Hkv;
     W.reset();
-    W.load_q(p.q, (size_t)b * p.Hq + (size_t)rr_kvh * G, p.qscale, lane);
-    done_mask = ~rr_stop;
+    W.load_q(p.q, (size_t)b * p.Hq + (size_t)kvh * G, p.qscale, lane);
+    done_mask = ~(uint32_t)req[rr * 4 + 3];
     return true;
   };
 
-  int e = 0, s = 0;
+  int s = 0, e = 0;  // ring stage, ring entries consumed
   uint32_t ph = 0;
-  int cur_g = -1, cur_c = -1;
   uint32_t vmask = 0;
-  bool draining = false;  // the producer's end entry has been seen
   while (ok) {
     const unsigned char* sK;
     const unsigned char* sV;
     int nv, pos = 0;
     const bool from_ring = rr < 0;
     if (!from_ring) {
-      while (rr_t <= rr_tmax && !((rr_vm >> rr_t) & 1u)) ++rr_t;
-      if (rr_t > rr_tmax) {  // request complete: its states go to the judge
+      const int rg = req[rr * 4], rc = req[rr * 4 + 1];
+      const uint32_t rvm = (uint32_t)req[rr * 4 + 2], rstop = (uint32_t)req[rr * 4 + 3];
+      int tmax = -1;
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        if ((rstop >> h) & 1u) tmax = max(tmax, req_t[rr * G + h]);
+      while (rr_t <= tmax && !((rvm >> rr_t) & 1u)) ++rr_t;
+      if (rr_t > tmax) {  // request complete: its states go to the judge
+        acquire();
         write_state();
-        post(SLOT_FIX, rr_g, rr_c, (int)rr_stop, no_fill);
-        ++req_done;
+        publish(POST_FIX, rg, rc, (int)rstop);
+        wc[W_RDONE] = wc[W_RDONE] + 1;
         rr = -1;
-        cur_g = -1;  // the registers were used: reload at the next block
-        if (!start_request() && draining) {
-          post(SLOT_DONE, 0, 0, 0, no_fill);
+        wc[W_CURG] = -1;  // the registers were used: reload at the next block
+        if (!start_request() && wc[W_DRAIN]) {
+          acquire();
+          publish(POST_DONE, 0, 0, 0);
           break;
         }
         continue;
       }
-      const int blk = art_block(p, rr_ord, rr_nb, rr_c * CB + rr_t, nullptr);
-      const size_t off = ((size_t)rr_bt[blk] * p.Hkv + rr_kvh) * kBlock * kHeadDim;  // page validated at load
+      const int b = rg / p.Hkv, kvh = rg % p.Hkv;
+      int L = p.seq_lens[b];
+      if (L < 0 || L > p.max_seq_len) L = 0;
+      const int* ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)rg * p.order_len : nullptr;
+      const int blk = art_block(p, ord, (L + kBlock - 1) / kBlock, rc * CB + rr_t, nullptr);
+      const int page = p.block_table[(size_t)b * p.max_blocks + blk];  // validated at load
+      const size_t off = ((size_t)page * p.Hkv + kvh) * kBlock * kHeadDim;
       sK = reinterpret_cast<const unsigned char*>(p.k_pool + off);
       sV = reinterpret_cast<const unsigned char*>(p.v_pool + off);
-      nv = min(kBlock, rr_L - blk * kBlock) - rb;
+      nv = min(kBlock, L - blk * kBlock) - rb;
     } else {
       if (!mbar_wait_bounded(&full[s], ph, &flags[1])) {
         if (lane == 0) fail();
@@ -675,28 +751,32 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       const int n = mt.x;
       if (n < 0) {
         // end of the traversal: once the judge has handled every chunk (the
-        // QUIT entry's handshake), serve the last requests, then release it
-        draining = true;
-        post(SLOT_QUIT, 0, 0, 0, no_fill);
-        const int slot = (ks - 1) % kSlots;
-        if (!mbar_wait_bounded(&pfree[slot], ((ks - 1) / kSlots) & 1, &flags[1])) {
+        // QUIT post's handshake), serve the last requests, then release it
+        wc[W_DRAIN] = 1;
+        acquire();
+        publish(POST_QUIT, 0, 0, 0);
+        const int kq = wc[W_KP] - 1;
+        if (!mbar_wait_bounded(&freed[kq & 1], (kq >> 1) & 1, &flags[1])) {
           if (lane == 0) fail();
           ok = false;
           break;
         }
-        req_seen = rtag[slot];
+        wc[W_RSEEN] = rtag[kq & 1];
         if (!start_request()) {
-          post(SLOT_DONE, 0, 0, 0, no_fill);
+          acquire();
+          publish(POST_DONE, 0, 0, 0);
           break;
         }
         continue;
       }
-      if (mt.y != cur_g || mt.z != cur_c) {
-        cur_g = mt.y;
-        cur_c = mt.z;
+      if (mt.y != wc[W_CURG] || mt.z != wc[W_CURC]) {  // a new chunk: take the next post's buffers
+        acquire();
+        wc[W_CURG] = mt.y;
+        wc[W_CURC] = mt.z;
         W.reset();
-        const int b = cur_g / p.Hkv, kvh = cur_g % p.Hkv;
-        W.load_q(p.q, (size_t)b * p.Hq + (size_t)kvh * G, p.qscale, lane);
+        if (n > 0)  // the chunk's first block carries the group's q rows
+          W.load_q(reinterpret_cast<const uint16_t*>(smem + s * C::STAGE_BYTES + 2 * kTileBytes), 0,
+                   p.qscale, lane);
         vmask = 0;
         done_mask = 0;
       }
@@ -707,8 +787,9 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
           s = 0;
           ph ^= 1u;
         }
+        merge_probes(vmask);
         write_state();
-        post(SLOT_END, cur_g, cur_c, (int)vmask, no_fill);
+        publish(POST_END, mt.y, mt.z, (int)vmask);
         start_request();
         continue;
       }
@@ -728,27 +809,26 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       }
       // this warp's running state after block `pos` of the chunk
       vmask |= 1u << pos;
-      post(SLOT_TILE, cur_g, cur_c, pos, [&](int slot) {
-        float* pw = probe + ((size_t)slot * NW + warp) * G * kProbeFloats;
-        if (W.owner) {
+      float* pw = probe + (size_t)kpar * probe_floats<G, NW, CB>() +
+                  ((size_t)pos * NW + warp) * G * kProbeFloats;
+      if (W.owner) {
 #pragma unroll
-          for (int j = 0; j < Lanes<G, NW>::VPL; ++j)
-            *reinterpret_cast<float2*>(pw + W.hd[j] * kProbeFloats) = make_float2(W.m_st[j], W.l_st[j]);
-        }
-        if (lane < 2) {
+        for (int j = 0; j < Lanes<G, NW>::VPL; ++j)
+          *reinterpret_cast<float2*>(pw + W.hd[j] * kProbeFloats) = make_float2(W.m_st[j], W.l_st[j]);
+      }
+      if (lane < 2) {
 #pragma unroll
-          for (int g2 = 0; g2 < G; ++g2) {
-            float x0, x1, x2, x3;
-            unpack2(W.acc[g2][0], x0, x1);
-            unpack2(W.acc[g2][1], x2, x3);
-            *reinterpret_cast<float4*>(pw + g2 * kProbeFloats + 4 + lane * 4) = make_float4(x0, x1, x2, x3);
-          }
+        for (int g2 = 0; g2 < G; ++g2) {
+          float x0, x1, x2, x3;
+          unpack2(W.acc[g2][0], x0, x1);
+          unpack2(W.acc[g2][1], x2, x3);
+          *reinterpret_cast<float4*>(pw + g2 * kProbeFloats + 4 + lane * 4) = make_float4(x0, x1, x2, x3);
         }
-      });
+      }
     } else {
 #pragma unroll
       for (int h = 0; h < G; ++h)
-        if (rr_st[h] == rr_t) done_mask |= 1u << h;
+        if (req_t[rr * G + h] == rr_t) done_mask |= 1u << h;
       ++rr_t;
     }
   }
@@ -778,6 +858,7 @@ int launch_art_t(const DecodeParams& p, cudaStream_t st) {
   constexpr int NW = SKV_ART_WARPS, CB = art_cb<G>(), ST = art_st<G, NW>(), MINB = art_minb<G>();
   using C = ArtCfg<G, NW, CB, ST>;
   static_assert(C::TOTAL <= (MINB == 2 ? 113 : 227) * 1024, "shared memory budget");
+  static_assert(ST >= 3, "a ring of at least three stages");
   auto kern = art_kernel<G, NW, CB, ST, MINB>;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -808,10 +889,10 @@ int art_chunk_blocks(int G) {
 size_t art_scratch_bytes_per_cta(int G) {
   constexpr int NW = SKV_ART_WARPS;
   switch (G) {
-    case 1: return scratch_floats<1, NW>() * 4;
-    case 2: return scratch_floats<2, NW>() * 4;
-    case 4: return scratch_floats<4, NW>() * 4;
-    default: return scratch_floats<8, NW>() * 4;
+    case 1: return scratch_floats<1, NW, art_cb<1>()>() * 4;
+    case 2: return scratch_floats<2, NW, art_cb<2>()>() * 4;
+    case 4: return scratch_floats<4, NW, art_cb<4>()>() * 4;
+    default: return scratch_floats<8, NW, art_cb<8>()>() * 4;
   }
 }
 

@@ -96,13 +96,14 @@ def test_workspace_size_query():
     n = L.skv_decode_workspace_size(ctypes.byref(full))
     # header (batch prefix) + per-warp partial records of 132 floats per head
     assert n > 0 and (n % 256) == 0 and n >= 16 * 8 * 16 * 4 * 132 * 4
-    # ART: per (chunk of 16 blocks, KV group): a look-back record of 12 floats
-    # and a partial record of 132 floats per head, plus zeroed control words
+    # ART: per (chunk of 32 blocks, KV group): a look-back record of 12 floats
+    # and a partial record of 132 floats per head, zeroed control words, and a
+    # scratch area of at most 192 KB per resident CTA (2 per SM)
     art = good_args(art=_Art(1, 1e-3, 1e-4, 4))
-    items = 16 * 8 * (512 // 16)
+    items = 16 * 8 * (512 // 32)
     na = L.skv_decode_workspace_size(ctypes.byref(art))
-    assert na >= items * 4 * (132 + 12) * 4 + (4 + 16 * 8 * (1 + 512 // 16 + 8)) * 4
-    assert na < items * 4 * (132 + 12) * 4 + 64 * 1024 + 2 * 148 * 8 * 4 * (8 * 12 + 132) * 4
+    assert na >= items * 4 * (132 + 12) * 4 + (4 + 16 * 8 * (1 + 512 // 32 + 8)) * 4
+    assert na < items * 4 * (132 + 12) * 4 + 64 * 1024 + 2 * 148 * 192 * 1024
     assert status(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == skv.SKV_EWORKSPACE
     assert L.skv_decode_workspace_size(ctypes.byref(good_args(head_dim=64))) == 0
     small = good_args(workspace=FAKE, workspace_bytes=n - 16)
