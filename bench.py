@@ -44,11 +44,16 @@ def parse():
     return ap.parse_args()
 
 
-def tensor_peak():
+def tensor_peak(power_capped):
+    """Dense bf16 peak: the burst figure while the clocks held (no power cap
+    seen during the timed region), else the sustained one."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        return json.load(open(p))["bf16_tflops_sustained"], "measured sustained bf16"
-    return 1400.0, "fallback sustained bf16"
+        d = json.load(open(p))
+        if power_capped:
+            return d["bf16_tflops_sustained"], "measured sustained bf16 (sw_power_cap seen)"
+        return d["bf16_tflops"], "measured burst bf16 (no power cap seen)"
+    return (1400.0, "fallback sustained bf16") if power_capped else (1590.0, "fallback burst bf16")
 
 
 def peaks():
@@ -243,7 +248,7 @@ def build_decode(torch, skv, skvgen, wl, status, art=False):
         if st != 0:
             raise skv.SkvError(st, "attn_decode")
 
-    step = Step(run, wl.kv_bytes(), 1 if (art or not n) else 2)
+    step = Step(run, wl.kv_bytes(), 2 if n else 1)  # decode or ART kernel, then the record merge
     # keep every tensor the raw pointers in `a` refer to alive with the step
     step.tensors = dict(q=q, k_pool=k_pool, v_pool=v_pool, bt=bt, sl=sl, out=out, lse=lse,
                         consumed=consumed, ws=ws, kw=kw, common=common)
@@ -314,7 +319,7 @@ def build_routed(torch, skv, skvgen, wl, status):
         ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda") if n else None
         a = skv.make_decode_args(q, k_pool, v_pool, bt, sl, out, lse, workspace=ws, **kw)
         layers.append(dict(fa=fa, a=a, keep=(q, k_pool, v_pool, bt, sl, out, lse, consumed, ws),
-                           consumed=consumed, launches=1 if (fa or not n) else 2))
+                           consumed=consumed, launches=2 if n else 1))
     L = skv.lib()
 
     def run():
@@ -534,10 +539,10 @@ def main():
         res["step_detail"] = step.extra
     if kind == "cfg4":  # a dense contraction: tensor-core roofline (sustained bf16 peak)
         tf = step.extra["flop"] / (per_launch_ms * 1e-3) / 1e12
-        peak_tf, tf_kind = tensor_peak()
+        peak_tf, tf_kind = tensor_peak("sw_power_cap" in clocks.get("reasons", []))
         res["metric_tflops"] = step.extra["flop"] * world / (ms_step * 1e-3) / 1e12
         res["roofline"] = {"bound": "tensor", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
-                           "frac": tf / peak_tf, "peak_kind": tf_kind, "traffic": None,
+                           "frac": tf / peak_tf, "peak_kind": tf_kind, "traffic": traffic_for(kind),
                            "kernel": "one step: chunk kernel x2 + merge"}
     if kind in ("cfg1", "cfg2"):
         res["config"]["traversal"] = "full"
@@ -552,7 +557,7 @@ def main():
                       "time_vs_full": art_step_ms / ms_step,
                       "attended_tokens_per_s": float(cons.sum()) * wl.bs / (art_step_ms * 1e-3),
                       "tau": wl.tau, "phi": wl.phi, "patience": wl.patience}
-        res["gpu_launches"] += args.steps
+        res["gpu_launches"] += args.steps * art_step.launches
     if e2e is not None:
         res["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline and kind in ("cfg1", "cfg2"):
@@ -564,18 +569,36 @@ def main():
         print(json.dumps(res), flush=True)
 
 
-def traffic_for(kind):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary (profiles/traffic.json), if it was taken on the current kernel
-    source; else None."""
+# dominant kernel of each workload's step and the sources it is built from
+KERNEL_SOURCES = {
+    "decode_kernel": ["decode.cu", "tile.cuh", "common.cuh", "decode.cuh"],
+    "art_kernel": ["art.cu", "tile.cuh", "common.cuh", "decode.cuh"],
+    "chunk_kernel": ["chunk.cu", "common.cuh", "decode.cuh"],
+    "select_kernel": ["select.cu", "common.cuh"],
+}
+DOMINANT = {"cfg1": "decode_kernel", "cfg2": "decode_kernel", "cfg3": "decode_kernel",
+            "cfg4": "chunk_kernel", "cfg5": "art_kernel"}
+
+
+def kernel_sha(kernel):
+    """Hash of the sources a kernel is compiled from (first 16 hex digits)."""
     import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "sparse_kv_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kind):
+    """DRAM bytes (read + write) per launch of the workload's dominant kernel
+    from the committed ncu summary (profiles/traffic.json), if it was taken on
+    the kernel's current sources; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "sparse_kv_b200", "csrc", "decode.cu")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or kind not in DOMINANT:
         return None
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    kernel = DOMINANT[kind]
     rec = json.load(open(p)).get(kind)
-    if not rec or rec.get("decode_cu_sha") != h:
+    if not rec or rec.get("kernel") != kernel or rec.get("sources_sha") != kernel_sha(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
