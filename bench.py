@@ -523,7 +523,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
                    "head_dim": wl.d, "context": wl.L, "page_tokens": wl.bs, "paging": wl.paging,
-                   "l2": "inputs larger than L2 (GBs of KV per step), no flush",
+                   "l2": ("KV cache of 4 MiB fits in L2 (launch-bound case), no flush" if kind == "cfg1"
+                          else "inputs larger than L2 (GBs of KV per step), no flush"),
                    "timing": "CUDA-graph replay per step, CUDA events",
                    "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": step.nbytes / (wl.d * 4) * wl.G * world / (ms_step * 1e-3),
@@ -533,6 +534,7 @@ def main():
                      "frac_of_8000": achieved / 8000.0, "traffic": traffic_for(kind),
                      "kernel": "one step of our kernels (decode + merge; per-kernel shares in profiles/)"},
         "clocks": clocks,
+        "step_ms_p10_p50_p90": [float(x) for x in np.percentile(per, [10, 50, 90])],
         "gpu_launches": args.steps * step.launches,
     }
     if step.extra:
