@@ -19,21 +19,20 @@
 //              kernel, and ends each chunk with a marker entry;
 //   consumers  NW warps fold every block into their online-softmax states
 //              (tile.cuh) and leave (m, l, O[0:8]) of their state after every
-//              block in a per-CTA scratch area.  At the end of a chunk they
-//              meet once; each warp combines its share of the blocks into the
-//              chunk-local prefixes, writes its whole state, and posts the
-//              chunk to the judge.  They never wait for a decision;
-//   judge      one warp combines the states into the chunk's record, waits for
-//              the previous chunk's published prefix (m, l, O[0:8], run of
-//              passing tests, blocks consumed or the stop) -- a decoupled
-//              look-back, as in single-pass parallel prefix scans --
-//              evaluates the test for all CB blocks at once (lane t: block t;
-//              the patience run by warp ballots) and publishes the inclusive
-//              prefix.
+//              block in a per-CTA scratch area; at the end of a chunk each
+//              warp writes its whole state and posts the chunk to the judge.
+//              They never meet and never wait for a decision;
+//   judge      one warp combines the warps' probes into the chunk-local prefix
+//              after every block (lane = (block, head)) and their states into
+//              the chunk's record, waits for the previous chunk's published
+//              prefix (m, l, O[0:8], run of passing tests, blocks consumed or
+//              the stop) -- a decoupled look-back, as in single-pass parallel
+//              prefix scans -- evaluates the test for all CB blocks at once
+//              (lane t: block t; the patience run by warp ballots) and
+//              publishes the inclusive prefix.
 // Posts alternate between two buffers, so the consumers run a chunk ahead of
-// the judge.  The probes, states and chunk-local prefixes live in global
-// memory rewritten in place (they stay in L2), which leaves the shared memory
-// to a 3-stage ring at two
+// the judge.  The probes and states live in global memory rewritten in place
+// (they stay in L2), which leaves the shared memory to a 3-stage ring at two
 // CTAs per SM.
 // A head that stops inside a chunk needs its state after the stop block, which
 // the consumers have already passed: the judge posts a request, and at a later
@@ -68,16 +67,14 @@ enum PostKind : int { POST_END = 1, POST_FIX = 2, POST_QUIT = 3, POST_DONE = 4 }
 constexpr size_t up16(size_t x) { return (x + 15) / 16 * 16; }
 
 // Per-CTA scratch in global memory, two buffers (post parity): probes
-// [2][CB][NW][G][12], states [2][NW][G][kRecFloats] and chunk-local prefixes
-// [2][CB][G][12].
+// [2][CB][NW][G][12] and states [2][NW][G][kRecFloats].
 template <int G, int NW, int CB>
 __host__ __device__ constexpr size_t probe_floats() {
   return (size_t)CB * NW * G * kProbeFloats;
 }
 template <int G, int NW, int CB>
 __host__ __device__ constexpr size_t scratch_floats() {
-  return 2 * probe_floats<G, NW, CB>() + 2 * (size_t)NW * G * kRecFloats +
-         2 * (size_t)CB * G * kProbeFloats;
+  return 2 * probe_floats<G, NW, CB>() + 2 * (size_t)NW * G * kRecFloats;
 }
 
 template <int G, int NW, int CB, int ST>
@@ -87,7 +84,7 @@ struct ArtCfg {  // shared-memory layout
   static constexpr int THREADS = (NW + 2) * 32;  // consumers, producer, judge
   // a stage: K rows, V rows, and the group's q rows (loaded with a chunk's first block)
   static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes + (size_t)G * kRowBytes;
-  static constexpr int NBAR = 2 * ST + 6;  // full, empty, fin, consumer barrier, posted[2], free[2]
+  static constexpr int NBAR = 2 * ST + 5;  // full, empty, fin, posted[2], free[2]
   static constexpr size_t OFF_BAR = ST * STAGE_BYTES;
   static constexpr size_t OFF_META = up16(OFF_BAR + NBAR * 8);        // int4 [ST]
   static constexpr size_t OFF_FLAGS = up16(OFF_META + ST * 16);       // int [4]
@@ -97,9 +94,10 @@ struct ArtCfg {  // shared-memory layout
   static constexpr size_t OFF_P = up16(OFF_REQ + kReqs * 16 + (size_t)kReqs * G * 4);  // float2 [NW][RPW][G]
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;   // float2 [NW][G]
   static constexpr size_t OFF_WCTL = up16(OFF_A + (size_t)NW * G * 8);  // int [NW][8]
-  static constexpr size_t TOTAL = OFF_WCTL + (size_t)NW * 8 * 4;
+  static constexpr size_t OFF_LOCAL = OFF_WCTL + (size_t)NW * 8 * 4;    // float [CB][G][12] (judge)
+  static constexpr size_t TOTAL = OFF_LOCAL + (size_t)CB * G * kProbeFloats * 4;
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_P % 16 == 0, "alignment");
-  static_assert(OFF_A % 16 == 0 && OFF_WCTL % 16 == 0, "alignment");
+  static_assert(OFF_A % 16 == 0 && OFF_WCTL % 16 == 0 && OFF_LOCAL % 16 == 0, "alignment");
   static_assert(OFF_TAG % 16 == 0 && OFF_REQ % 16 == 0, "alignment");
   static_assert((RPW * G * 8) % 16 == 0 || G == 1, "pbuf rows");
   static_assert(CB >= 1 && CB <= 32, "one judge lane per block of a chunk");
@@ -156,8 +154,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + ST;
   uint64_t* fin_bar = empty + ST;
-  uint64_t* cbar = fin_bar + 1;     // consumer warps meet at the end of a chunk
-  uint64_t* posted = cbar + 1;      // [2] a post is ready (one arrival per consumer warp)
+  uint64_t* posted = fin_bar + 1;   // [2] a post is ready (one arrival per consumer warp)
   uint64_t* freed = posted + 2;     // [2] the judge is done with a post
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows | 0 = end of chunk, group, chunk, block in chunk | blocks}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
@@ -169,7 +166,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   volatile int* req_t = reinterpret_cast<volatile int*>(smem + C::OFF_REQ + kReqs * 16);  // [kReqs][G]
   float* probe = p.art_scratch + (size_t)blockIdx.x * scratch_floats<G, NW, CB>();  // [2][CB][NW][G][12]
   float* state = probe + 2 * probe_floats<G, NW, CB>();                            // [2][NW][G][132]
-  float* local = state + 2 * (size_t)NW * G * kRecFloats;                          // [2][CB][G][12]
+  float* local = reinterpret_cast<float*>(smem + C::OFF_LOCAL);                    // [CB][G][12]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int groups = p.B * p.Hkv;
@@ -180,7 +177,6 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       mbar_init(&empty[s], NW);
     }
     mbar_init(fin_bar, NW);
-    mbar_init(cbar, NW);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&posted[i], NW);
       mbar_init(&freed[i], 1);
@@ -302,6 +298,56 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     int kj = 0;     // posts consumed
     int n_req = 0;  // re-run requests posted
     int n_fix = 0;  // re-runs received back
+    // Chunk-local prefix after every block of the chunk: combine the consumer
+    // warps' running states.  Lane = one (block, head) pair; every load of a
+    // half of the warps is issued at once (one L2 round trip per half).
+    auto merge_probes = [&](const float* pr0, uint32_t vmask) {
+      constexpr int NH = NW / 2;
+      for (int i0 = 0; i0 < CB * G; i0 += 32) {
+        const int i = i0 + lane, t = i / G, h = i % G;
+        const bool valid = i < CB * G && ((vmask >> t) & 1u);
+        float M = -INFINITY, Ls = 0.f, X[8];
+#pragma unroll
+        for (int d = 0; d < 8; ++d) X[d] = 0.f;
+        if (valid) {
+          const float* pr = pr0 + ((size_t)t * NW * G + h) * kProbeFloats;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float2 ml[NH];
+            float4 xa[NH], xb[NH];
+#pragma unroll
+            for (int w = 0; w < NH; ++w) {
+              const float* q = pr + (size_t)(half * NH + w) * G * kProbeFloats;
+              ml[w] = *reinterpret_cast<const float2*>(q);
+              xa[w] = *reinterpret_cast<const float4*>(q + 4);
+              xb[w] = *reinterpret_cast<const float4*>(q + 8);
+            }
+            float Mh = M;
+#pragma unroll
+            for (int w = 0; w < NH; ++w) Mh = fmaxf(Mh, ml[w].x);
+            if (Mh != -INFINITY) {
+              const float fo = exp2f(M - Mh);  // rescale what the first half gave (0 if none)
+              Ls *= fo;
+#pragma unroll
+              for (int d = 0; d < 8; ++d) X[d] *= fo;
+#pragma unroll
+              for (int w = 0; w < NH; ++w) {
+                const float f = exp2f(ml[w].x - Mh);  // 0 for an empty warp state
+                Ls += ml[w].y * f;
+                X[0] += xa[w].x * f; X[1] += xa[w].y * f; X[2] += xa[w].z * f; X[3] += xa[w].w * f;
+                X[4] += xb[w].x * f; X[5] += xb[w].y * f; X[6] += xb[w].z * f; X[7] += xb[w].w * f;
+              }
+              M = Mh;
+            }
+          }
+          float* dst = local + ((size_t)t * G + h) * kProbeFloats;
+          *reinterpret_cast<float4*>(dst) = make_float4(M, Ls, 0.f, 0.f);
+          *reinterpret_cast<float4*>(dst + 4) = make_float4(X[0], X[1], X[2], X[3]);
+          *reinterpret_cast<float4*>(dst + 8) = make_float4(X[4], X[5], X[6], X[7]);
+        }
+      }
+    };
+
     // combine the state area into the records of `heads` of chunk (g, c)
     auto reduce_states = [&](const float* st_area, int g, int c, uint32_t heads) {
       const size_t item = (size_t)g * p.art_maxc + c;
@@ -532,10 +578,11 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
                 tg_a = tag[par * 4 + 3];
       const float* st_area = state + (size_t)par * NW * G * kRecFloats;
       if (kind == POST_END) {
+        merge_probes(probe + (size_t)par * probe_floats<G, NW, CB>(), (uint32_t)tg_a);
         reduce_states(st_area, tg_g, tg_c, (1u << G) - 1u);
+        __syncwarp();  // the chunk-local prefixes are visible to every lane
         int st[G];
-        const uint32_t stopmask =
-            evaluate(local + (size_t)par * CB * G * kProbeFloats, tg_g, tg_c, (uint32_t)tg_a, st);
+        const uint32_t stopmask = evaluate(local, tg_g, tg_c, (uint32_t)tg_a, st);
         if (stopmask) {
           if (n_req - n_fix >= kReqs) {
             if (lane == 0) fail();  // cannot happen: the consumers serve requests every chunk
@@ -574,12 +621,11 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
   // Warp-uniform counters used at chunk boundaries live in shared memory (one
   // block per warp): the fold loop is register-bound.
-  enum { W_KP = 0, W_RSEEN, W_RDONE, W_CBPH, W_DRAIN, W_CURG, W_CURC };
+  enum { W_KP = 0, W_RSEEN, W_RDONE, W_DRAIN, W_CURG, W_CURC };
   volatile int* wc = reinterpret_cast<volatile int*>(smem + C::OFF_WCTL) + warp * 8;
   wc[W_KP] = 0;      // posts made
   wc[W_RSEEN] = 0;   // requests the judge had posted when it freed our buffer
   wc[W_RDONE] = 0;   // requests served
-  wc[W_CBPH] = 0;    // phase of the consumer barrier
   wc[W_DRAIN] = 0;   // the producer's end entry has been seen
   wc[W_CURG] = -1;   // chunk being folded
   wc[W_CURC] = -1;
@@ -631,57 +677,6 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
             make_float2(W.m_st[j], W.l_st[j]);
     }
   };
-  // End of a chunk: once every warp's probes are written, this warp combines
-  // blocks warp, warp + NW, ... into the chunk-local prefixes (lane: head, dim).
-  auto merge_probes = [&](uint32_t vmask) {
-    __syncwarp();
-    mbar_arrive_if(cbar, lane == 0);
-    const int cb_ph = wc[W_CBPH];
-    if (!mbar_wait_bounded(cbar, cb_ph, &flags[1])) {
-      if (lane == 0) fail();
-      ok = false;
-    }
-    wc[W_CBPH] = cb_ph ^ 1;
-    const int par = wc[W_KP] & 1;
-    const float* pr0 = probe + (size_t)par * probe_floats<G, NW, CB>();
-    float* loc = local + (size_t)par * CB * G * kProbeFloats;
-    for (int t = warp; t < CB; t += NW) {
-      if (!((vmask >> t) & 1u)) continue;
-      const float* pr = pr0 + (size_t)t * NW * G * kProbeFloats;
-#pragma unroll
-      for (int r = 0; r < (G * 8 + 31) / 32; ++r) {
-        const int h = r * 4 + (lane >> 3), d = lane & 7;
-        if (h < G) {
-          float2 ml[NW];
-          float x[NW];
-#pragma unroll
-          for (int w = 0; w < NW; ++w) {
-            ml[w] = *reinterpret_cast<const float2*>(pr + (w * G + h) * kProbeFloats);
-            x[w] = pr[(w * G + h) * kProbeFloats + 4 + d];
-          }
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[w].x);
-          float Ls = 0.f, X = 0.f;
-          if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-              const float f = exp2f(ml[w].x - M);  // 0 for an empty warp state
-              Ls += ml[w].y * f;
-              X += x[w] * f;
-            }
-          }
-          float* dst = loc + ((size_t)t * G + h) * kProbeFloats;
-          dst[4 + d] = X;
-          if (d == 0) {
-            dst[0] = M;
-            dst[1] = Ls;
-          }
-        }
-      }
-    }
-  };
-
   // Re-fold of a chunk for the heads that stop in it (a request of the judge):
   // the chunk's blocks up to each head's stop block, from the pool.  Only the
   // request index and the next block live in registers; the rest is re-read
@@ -787,7 +782,6 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
           s = 0;
           ph ^= 1u;
         }
-        merge_probes(vmask);
         write_state();
         publish(POST_END, mt.y, mt.z, (int)vmask);
         start_request();
