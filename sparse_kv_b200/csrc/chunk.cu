@@ -8,22 +8,30 @@
 // that partial's normalised O and log-sum-exp; partials combine exactly with
 // attn_merge_lse.
 //
-// Warp roles (7 warps):
-//   warps 0, 6  producers: TMA tensor loads (128B swizzle, no multicast) of the
-//               K rows (warp 0) and V rows (warp 6) of 128-key tiles into two
+// Warp roles (11 warps):
+//   warps 0, 10 producers: TMA tensor loads (128B swizzle, no multicast) of the
+//               K rows (warp 0) and V rows (warp 10) of 128-key tiles into two
 //               separate 2-stage rings (a K stage frees after Q K^T, a V stage
 //               after P V, so the next keys load while the softmax runs)
 //   warp 1      MMA: allocates 512 TMEM columns, issues tcgen05.mma for
 //               S = Q K^T (two ping-pong S buffers of 128 fp32 columns) and
-//               O += P V (O: 128 fp32 columns), commits to mbarriers
-//   warps 2..5  softmax: thread i owns row i (TMEM lane i), reads its S row
-//               with tcgen05.ld, masks, keeps the row max, rescales O in TMEM
-//               only when the max grows by more than 2^8 (the scale is applied
-//               consistently to O and l, so the result stays exact), writes P
-//               as bf16 into 128B-swizzled shared memory, and in the end
-//               normalises O.
-// Operands: Q, K, P K-major and V MN-major, all in the canonical 128B-swizzle
-// layout (8-row x 128-byte atoms, 1024-byte aligned); bf16 x bf16 -> fp32.
+//               O += P V (O: 128 fp32 columns; P, the A operand, read from
+//               TMEM: two ping-pong buffers of 64 columns, bf16 pairs),
+//               commits to mbarriers
+//   warps 2..9  softmax: two threads per row (TMEM lane), one per 64-column
+//               half (warps 2..5 the low half, 6..9 the high half; a warp may
+//               only read its own quarter of the TMEM lanes, and both warps of
+//               a pair sit on the same quarter).  A thread reads its half of
+//               the S row with tcgen05.ld, masks, and swaps its half's max with
+//               its partner through shared memory; both then keep the same row
+//               max, rescale their half of O in TMEM only when the max grows by
+//               more than 2^8 (the scale is applied consistently to O and l,
+//               so the result stays exact), write their half of P as bf16 pairs
+//               into their own TMEM lane with tcgen05.st, and in the end
+//               normalise O.
+// Operands: Q and K K-major, V MN-major, in the canonical 128B-swizzle layout
+// (8-row x 128-byte atoms, 1024-byte aligned) in shared memory; P in TMEM
+// (row = lane, two bf16 keys per 32-bit column); bf16 x bf16 -> fp32.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -35,26 +43,28 @@ namespace {
 
 constexpr int BM = 128;                         // rows per CTA
 constexpr int BN = 128;                         // keys per tile
-constexpr int kChunkWarps = 7;
+constexpr int kChunkWarps = 11;
 constexpr int kChunkThreads = kChunkWarps * 32;
 constexpr int kHalf = BM * 64 * 2;              // one 64-column half of a 128-row tile: 16 KiB
 constexpr int kTile = 2 * kHalf;                // 32 KiB
 constexpr int kStages = 2;
-constexpr uint32_t kTmemCols = 512;             // S0 [0,128), S1 [128,256), O [256,384)
+constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512)
 constexpr uint32_t kColO = 256;
+constexpr uint32_t kColP = 384;
 
 constexpr size_t OFF_Q = 0;
-constexpr size_t OFF_P = OFF_Q + kTile;            // two P buffers (tile j uses j & 1)
-constexpr size_t OFF_K = OFF_P + 2 * (size_t)kTile;  // K stage s at +s*kTile
+constexpr size_t OFF_K = OFF_Q + (size_t)kTile;      // K stage s at +s*kTile
 constexpr size_t OFF_V = OFF_K + (size_t)kStages * kTile;  // V stage s at +s*kTile
 constexpr size_t OFF_BAR = OFF_V + (size_t)kStages * kTile;
-// k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_free[2], p_full, o_done[2]
-constexpr int NBAR = 15;
-constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
+// k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_free[2], p_full, o_done[2],
+// xbar[4] (one per softmax warp pair)
+constexpr int NBAR = 19;
+constexpr size_t OFF_XCH = OFF_BAR + NBAR * 8;       // float [2 parity][2 halves][128 rows]
+constexpr size_t OFF_TMEM = OFF_XCH + 2 * 2 * BM * 4;
 constexpr size_t OFF_FLAG = OFF_TMEM + 16;
 constexpr size_t SMEM_USED = OFF_FLAG + 16;
 constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024 bytes
-static_assert(OFF_P % 1024 == 0 && OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && kTile % 1024 == 0,
+static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && kTile % 1024 == 0,
               "swizzle atoms");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
@@ -102,6 +112,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t da, uint64_t 
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(da), "l"(db), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
+// The same with the A operand in TMEM (M rows = lanes, K along the columns).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                            uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(db), "r"(idesc), "r"((uint32_t)accumulate)
       : "memory");
 }
 
@@ -155,6 +175,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
+// 32 consecutive 32-bit columns of this thread's TMEM lane, raw bits.
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -199,6 +232,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* s_free = bar + 10;
   uint64_t* p_full = bar + 12;
   uint64_t* o_done = bar + 13;  // [2]: P.V of tiles with j & 1 == b
+  uint64_t* xbar = bar + 15;    // [4]: the two softmax warps of a TMEM lane quarter
+  volatile float* xch = reinterpret_cast<volatile float*>(smem + OFF_XCH);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
 
@@ -235,11 +270,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     }
     mbar_init(&s_full[0], 1);    // tcgen05.commit after Q K^T
     mbar_init(&s_full[1], 1);
-    mbar_init(&s_free[0], 128);  // every softmax thread has read its S row
-    mbar_init(&s_free[1], 128);
-    mbar_init(p_full, 128);      // every softmax thread has written its P row
+    mbar_init(&s_free[0], 256);  // every softmax thread has read its half S row
+    mbar_init(&s_free[1], 256);
+    mbar_init(p_full, 256);      // every softmax thread has written its half P row
     mbar_init(&o_done[0], 1);    // tcgen05.commit after P V of even tiles
     mbar_init(&o_done[1], 1);    // ... and of odd tiles
+    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);  // one arrival per warp of the pair
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -250,26 +286,27 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // ---- Q rows -> shared memory (softmax threads, one row each)
-  const bool softmax_warp = warp >= 2 && warp < 6;
+  // ---- Q rows -> shared memory (softmax threads, a half row each)
+  const bool softmax_warp = warp >= 2 && warp < 10;
   const int srow = softmax_warp ? ((warp & 3) * 32 + lane) : -1;  // TMEM lane = row
+  const int ch = (warp - 2) >> 2;                                // column half of this thread
   const int grow = m_tile * BM + srow;                          // row within the group
   const int t_row = (srow >= 0) ? grow / p.G : 0;
   const bool row_valid = srow >= 0 && t_row < p.Tq;
   if (srow >= 0) {
-    uint4 chunks[16];
+    uint4 chunks[8];
     if (row_valid) {
       const uint4* src = reinterpret_cast<const uint4*>(
           p.q + (((size_t)b * p.Tq + t_row) * p.Hq + (size_t)kvh * p.G + grow % p.G) * kHeadDim);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) chunks[c] = src[c];
+      for (int c = 0; c < 8; ++c) chunks[c] = src[ch * 8 + c];
     } else {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) chunks[c] = make_uint4(0u, 0u, 0u, 0u);
+      for (int c = 0; c < 8; ++c) chunks[c] = make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
-      *reinterpret_cast<uint4*>(smem + OFF_Q + (c >> 3) * kHalf + swz(srow, c & 7)) = chunks[c];
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint4*>(smem + OFF_Q + ch * kHalf + swz(srow, c)) = chunks[c];
     fence_async_smem();
   }
   fence_before_sync();
@@ -277,8 +314,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 || warp == 6) {
-    // ------------------------------------------------------------ producers (K: warp 0, V: warp 6)
+  if (warp == 0 || warp == 10) {
+    // ------------------------------------------------------------ producers (K: warp 0, V: warp 10)
     const bool is_k = warp == 0;
     if (lane == 0 && n_tiles > 0) {
       const CUtensorMap* map = is_k ? &tmK : &tmV;
@@ -325,7 +362,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_tiles > 0) {
       const uint32_t idesc_qk = instr_desc(false), idesc_pv = instr_desc(true);
-      const uint32_t q_addr = smem_u32(smem + OFF_Q), p_addr = smem_u32(smem + OFF_P);
+      const uint32_t q_addr = smem_u32(smem + OFF_Q);
       auto issue_qk = [&](int j) -> bool {
         const int st = j & 1, sb = j & 1;
         if (!mbar_wait_bounded(&k_full[st], (j >> 1) & 1, abort_flag)) return false;
@@ -349,14 +386,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (!mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
         fence_after_sync();
         const uint32_t v_addr = smem_u32(smem + OFF_V + (size_t)(j & 1) * kTile);
-        const uint32_t pj_addr = p_addr + (uint32_t)(j & 1) * kTile;
+        const uint32_t pj = tmem + kColP + (uint32_t)(j & 1) * (BN / 2);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
-          // A = P rows x 16 keys (K-major); B = V 16 keys x 128 dims (MN-major)
-          const uint32_t a_off = (ks >> 2) * kHalf + (ks & 3) * 32;
+          // A = P rows x 16 keys (TMEM, 8 columns); B = V 16 keys x 128 dims (MN-major)
           const uint32_t b_off = ks * 16 * 128;
-          mma_bf16(tmem + kColO, smem_desc(pj_addr + a_off, 16, 1024),
-                   smem_desc(v_addr + b_off, kHalf, 1024), idesc_pv, j > 0 || ks > 0);
+          mma_bf16_ts(tmem + kColO, pj + ks * 8, smem_desc(v_addr + b_off, kHalf, 1024), idesc_pv,
+                      j > 0 || ks > 0);
         }
         mma_commit(&o_done[j & 1]);
         mma_commit(&v_empty[j & 1]);
@@ -368,35 +404,45 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    constexpr int HC = BN / 2;                                       // columns of a half
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;  // TMEM lane field
     const int q_pos = L - p.Tq + t_row;  // causal limit of this row
+    uint64_t* pair_bar = &xbar[warp & 3];
     float m_used = -INFINITY, l_sum = 0.f;
     bool o_live = false;  // O holds data (first P.V has run)
     bool ok = true;
+    // swap a value with the other half of this row (phase `ph` of the pair's barrier)
+    auto swap_half = [&](float mine, int ph) -> float {
+      xch[((ph & 1) * 2 + ch) * BM + srow] = mine;
+      __syncwarp();
+      mbar_arrive_if(pair_bar, lane == 0);
+      if (!mbar_wait_bounded(pair_bar, ph & 1, abort_flag)) ok = false;
+      return xch[((ph & 1) * 2 + (ch ^ 1)) * BM + srow];
+    };
     for (int j = 0; j < n_tiles && ok; ++j) {
       const int sb = j & 1;
       if (!mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       fence_after_sync();
-      float s[BN];
+      float s[HC];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < HC / 32; ++c) {
         float v[32];
-        tmem_ld32(tmem + lane_base + sb * BN + c * 32, v);
+        tmem_ld32(tmem + lane_base + sb * BN + ch * HC + c * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
       }
       tmem_wait_ld();
       fence_before_sync();
       mbar_arrive(&s_free[sb]);
-      // mask (boundary tiles only) and the tile max of the raw scores (the scale is
+      // mask (boundary tiles only) and the max of the raw scores (the scale is
       // positive, so max(s) * scale is the max of the base-2 logits); 8 chains
       const int kp0 = pos0 + j * BN;
       const bool interior = row_valid && kp0 >= k_lo && kp0 + BN <= k_hi &&
                             (!p.causal || kp0 + BN - 1 <= q_pos);
       if (!interior) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int kp = kp0 + c;
+        for (int c = 0; c < HC; ++c) {
+          const int kp = kp0 + ch * HC + c;
           bool valid = row_valid && kp >= k_lo && kp < k_hi;
           if (p.causal) valid = valid && kp <= q_pos;
           s[c] = valid ? s[c] : -INFINITY;
@@ -406,13 +452,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx[u] = fmaxf(s[u], s[u + 8]);
 #pragma unroll
-      for (int c = 16; c < BN; c += 16)
+      for (int c = 16; c < HC; c += 16)
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], fmaxf(s[c + u], s[c + 8 + u]));
-      const float tmax = p.qscale * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                          fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      // P buffer j & 1 was last read by the P.V of tile j - 2: it must be complete.
-      // (o_done[b] cannot run ahead by two phases: its next phase needs this P.)
+      const float hmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float tmax = p.qscale * fmaxf(hmax, swap_half(hmax, j));
+      if (!ok) break;
+      // P buffer j & 1 was last read by the P.V of tile j - 2: it must be complete
+      // (o_done[b] cannot run ahead by two phases: its next phase needs this P)
       if (j >= 2 && !mbar_wait_bounded(&o_done[j & 1], ((j >> 1) - 1) & 1, abort_flag)) {
         ok = false;
         break;
@@ -429,28 +477,29 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           }
           fence_after_sync();
 #pragma unroll
-          for (int c = 0; c < kHeadDim / 32; ++c) {
+          for (int c = 0; c < HC / 32; ++c) {
             float v[32];
-            tmem_ld32(tmem + lane_base + kColO + c * 32, v);
+            tmem_ld32(tmem + lane_base + kColO + ch * HC + c * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= alpha;
-            tmem_st32(tmem + lane_base + kColO + c * 32, v);
+            tmem_st32(tmem + lane_base + kColO + ch * HC + c * 32, v);
           }
           tmem_wait_st();
         }
         m_used = tmax;
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      // P = 2^(s * scale - m) as bf16 into the swizzled P tile; packed fp32x2 for the
-      // exponent argument and for l, which accumulates the unrounded values
+      // P = 2^(s * scale - m) as bf16 pairs into this half of P buffer j & 1 in
+      // TMEM (this thread's lane); packed fp32x2 for the exponent argument and
+      // for l, which sums the unrounded values
       const f2 sc2 = pack2(p.qscale, p.qscale), nm2 = pack2(-mu, -mu);
       f2 ls2[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) ls2[u] = pack2(0.f, 0.f);
+      uint32_t pw[HC / 2];
 #pragma unroll
-      for (int c8 = 0; c8 < BN / 8; ++c8) {
-        uint32_t w[4];
+      for (int c8 = 0; c8 < HC / 8; ++c8) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           f2 x = nm2;
@@ -461,11 +510,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           const f2 pp = pack2(p0, p1);
           ls2[u] = fadd2(ls2[u], pp);
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);  // p0 in the low half
-          w[u] = *reinterpret_cast<const uint32_t*>(&h2);
+          pw[c8 * 4 + u] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        *reinterpret_cast<uint4*>(smem + OFF_P + (size_t)(j & 1) * kTile + (c8 >> 3) * kHalf +
-                                  swz(srow, c8 & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      tmem_st32u(tmem + lane_base + kColP + (uint32_t)(j & 1) * (BN / 2) + ch * (HC / 2), pw);
+      tmem_wait_st();
       {
         const f2 t2 = fadd2(fadd2(ls2[0], ls2[1]), fadd2(ls2[2], ls2[3]));
         float a0, a1;
@@ -473,7 +522,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         l_sum += a0 + a1;
       }
       // keys outside the range on a boundary tile: zero their V rows (they may hold
-      // anything) so that 0 * V stays 0
+      // anything) so that 0 * V stays 0; each thread clears its half of the row
       const int key = kp0 + srow;
       if (kp0 < k_lo || kp0 + BN > k_hi) {
         // V(j) must have landed before its rows are cleared (v_full cannot run two
@@ -485,8 +534,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (key < k_lo || key >= k_hi) {
           unsigned char* sV = smem + OFF_V + (size_t)(j & 1) * kTile;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            *reinterpret_cast<uint4*>(sV + (c >> 3) * kHalf + swz(srow, c & 7)) = make_uint4(0u, 0u, 0u, 0u);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(sV + ch * kHalf + swz(srow, c)) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
       fence_async_smem();
@@ -494,22 +543,23 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       mbar_arrive(p_full);
       o_live = true;
     }
-    // ---- epilogue: O / l and log-sum-exp for this row
+    // ---- epilogue: O / l and log-sum-exp for this row (l summed over both halves)
     if (ok && n_tiles > 0) {  // the last P.V (the tensor core runs them in order)
       const int jl = n_tiles - 1;
       if (!mbar_wait_bounded(&o_done[jl & 1], (jl >> 1) & 1, abort_flag)) ok = false;
     }
+    if (ok) l_sum += swap_half(l_sum, n_tiles);
     if (!ok) {
       dev_error(p.status, SKV_DEV_TIMEOUT);
       *abort_flag = 1;
     }
     fence_after_sync();
-    float o[kHeadDim];
+    float o[HC];
     if (n_tiles > 0) {
 #pragma unroll
-      for (int c = 0; c < kHeadDim / 32; ++c) {
+      for (int c = 0; c < HC / 32; ++c) {
         float v[32];
-        tmem_ld32(tmem + lane_base + kColO + c * 32, v);
+        tmem_ld32(tmem + lane_base + kColO + ch * HC + c * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[c * 32 + i] = v[i];
       }
@@ -519,16 +569,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
       const size_t rows = (size_t)p.B * p.Tq * p.Hq;
       const size_t row = ((size_t)b * p.Tq + t_row) * p.Hq + (size_t)kvh * p.G + grow % p.G;
-      float4* dst = reinterpret_cast<float4*>(p.out + ((size_t)shard * rows + row) * kHeadDim);
+      float4* dst = reinterpret_cast<float4*>(p.out + ((size_t)shard * rows + row) * kHeadDim + ch * HC);
 #pragma unroll
-      for (int c = 0; c < kHeadDim / 4; ++c) {
+      for (int c = 0; c < HC / 4; ++c) {
         if (n_tiles > 0)
           dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
         else
           dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      p.lse[(size_t)shard * rows + row] =
-          (l_sum > 0.f) ? (m_used + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      if (ch == 0)
+        p.lse[(size_t)shard * rows + row] =
+            (l_sum > 0.f) ? (m_used + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
     }
   }
   // ---- teardown: every tcgen05 operation is complete; free TMEM
