@@ -14,21 +14,22 @@
 //               separate 2-stage rings (a K stage frees after Q K^T, a V stage
 //               after P V, so the next keys load while the softmax runs)
 //   warp 1      MMA: allocates 512 TMEM columns, issues tcgen05.mma for
-//               S = Q K^T (two ping-pong S buffers of 128 fp32 columns) and
-//               O += P V (O: 128 fp32 columns; P, the A operand, read from
-//               TMEM: two ping-pong buffers of 64 columns, bf16 pairs),
-//               commits to mbarriers
-//   warps 2..9  softmax: two threads per row (TMEM lane), one per 64-column
-//               half (warps 2..5 the low half, 6..9 the high half; a warp may
-//               only read its own quarter of the TMEM lanes, and both warps of
-//               a pair sit on the same quarter).  A thread reads its half of
-//               the S row with tcgen05.ld, masks, and swaps its half's max with
-//               its partner through shared memory; both then keep the same row
-//               max, rescale their half of O in TMEM only when the max grows by
-//               more than 2^8 (the scale is applied consistently to O and l,
-//               so the result stays exact), write their half of P as bf16 pairs
-//               into their own TMEM lane with tcgen05.st, and in the end
-//               normalise O.
+//               S = Q K^T into two ping-pong S buffers of 128 fp32 columns and,
+//               per key half h, O_h += P_h V_h (two accumulators of 128 fp32
+//               columns; the A operand P_h is read from TMEM, where the
+//               softmax wrote it over the S columns it came from), and commits
+//               to mbarriers
+//   warps 2..9  softmax: two threads per row (TMEM lane), one per 64-key half
+//               of every tile (warps 2..5 the low half, 6..9 the high half; a
+//               warp may only touch its own quarter of the TMEM lanes, and both
+//               warps of a pair sit on the same quarter).  Each thread runs its
+//               own online softmax over its half's keys: reads its half of the
+//               S row with tcgen05.ld, masks, keeps its running max, rescales
+//               its accumulator O_h in TMEM only when the max grows by more than
+//               2^8 (the scale is applied consistently to O_h and l_h, so the
+//               result stays exact), and writes P_h as bf16 pairs with
+//               tcgen05.st.  The two halves meet once, at the end, to combine
+//               (m, l, O) of the row exactly.
 // Operands: Q and K K-major, V MN-major, in the canonical 128B-swizzle layout
 // (8-row x 128-byte atoms, 1024-byte aligned) in shared memory; P in TMEM
 // (row = lane, two bf16 keys per 32-bit column); bf16 x bf16 -> fp32.
@@ -48,17 +49,16 @@ constexpr int kChunkThreads = kChunkWarps * 32;
 constexpr int kHalf = BM * 64 * 2;              // one 64-column half of a 128-row tile: 16 KiB
 constexpr int kTile = 2 * kHalf;                // 32 KiB
 constexpr int kStages = 2;
-constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512)
-constexpr uint32_t kColO = 256;
-constexpr uint32_t kColP = 384;
+constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O_0 [256,384), O_1 [384,512)
+constexpr uint32_t kColO = 256;       // O_h at kColO + h * 128
 
 constexpr size_t OFF_Q = 0;
 constexpr size_t OFF_K = OFF_Q + (size_t)kTile;      // K stage s at +s*kTile
 constexpr size_t OFF_V = OFF_K + (size_t)kStages * kTile;  // V stage s at +s*kTile
 constexpr size_t OFF_BAR = OFF_V + (size_t)kStages * kTile;
-// k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_free[2], p_full, o_done[2],
+// k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full, o_done[2],
 // xbar[4] (one per softmax warp pair)
-constexpr int NBAR = 19;
+constexpr int NBAR = 17;
 constexpr size_t OFF_XCH = OFF_BAR + NBAR * 8;       // float [2 parity][2 halves][128 rows]
 constexpr size_t OFF_TMEM = OFF_XCH + 2 * 2 * BM * 4;
 constexpr size_t OFF_FLAG = OFF_TMEM + 16;
@@ -229,10 +229,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* v_full = bar + 4;
   uint64_t* v_empty = bar + 6;
   uint64_t* s_full = bar + 8;
-  uint64_t* s_free = bar + 10;
-  uint64_t* p_full = bar + 12;
-  uint64_t* o_done = bar + 13;  // [2]: P.V of tiles with j & 1 == b
-  uint64_t* xbar = bar + 15;    // [4]: the two softmax warps of a TMEM lane quarter
+  uint64_t* p_full = bar + 10;
+  uint64_t* o_done = bar + 11;  // [2]: P.V of tiles with j & 1 == b
+  uint64_t* xbar = bar + 13;    // [4]: the two softmax warps of a TMEM lane quarter
   volatile float* xch = reinterpret_cast<volatile float*>(smem + OFF_XCH);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
@@ -270,8 +269,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     }
     mbar_init(&s_full[0], 1);    // tcgen05.commit after Q K^T
     mbar_init(&s_full[1], 1);
-    mbar_init(&s_free[0], 256);  // every softmax thread has read its half S row
-    mbar_init(&s_free[1], 256);
     mbar_init(p_full, 256);      // every softmax thread has written its half P row
     mbar_init(&o_done[0], 1);    // tcgen05.commit after P V of even tiles
     mbar_init(&o_done[1], 1);    // ... and of odd tiles
@@ -365,8 +362,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const uint32_t q_addr = smem_u32(smem + OFF_Q);
       auto issue_qk = [&](int j) -> bool {
         const int st = j & 1, sb = j & 1;
+        // S buffer sb last held P(j - 2), read by a P.V issued before this Q K^T: the
+        // tensor core runs them in order
         if (!mbar_wait_bounded(&k_full[st], (j >> 1) & 1, abort_flag)) return false;
-        if (j >= 2 && !mbar_wait_bounded(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag)) return false;
         fence_after_sync();
         const uint32_t k_addr = smem_u32(smem + OFF_K + (size_t)st * kTile);
 #pragma unroll
@@ -386,13 +384,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (!mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
         fence_after_sync();
         const uint32_t v_addr = smem_u32(smem + OFF_V + (size_t)(j & 1) * kTile);
-        const uint32_t pj = tmem + kColP + (uint32_t)(j & 1) * (BN / 2);
+        const uint32_t pj = tmem + (uint32_t)(j & 1) * BN;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
-          // A = P rows x 16 keys (TMEM, 8 columns); B = V 16 keys x 128 dims (MN-major)
+          // A = P_h rows x 16 keys (TMEM, 8 columns of the half's S columns);
+          // B = V 16 keys x 128 dims (MN-major); D = O_h
+          const int h = ks >> 2, kk = ks & 3;
           const uint32_t b_off = ks * 16 * 128;
-          mma_bf16_ts(tmem + kColO, pj + ks * 8, smem_desc(v_addr + b_off, kHalf, 1024), idesc_pv,
-                      j > 0 || ks > 0);
+          mma_bf16_ts(tmem + kColO + h * BM, pj + h * (BN / 2) + kk * 8,
+                      smem_desc(v_addr + b_off, kHalf, 1024), idesc_pv, j > 0 || kk > 0);
         }
         mma_commit(&o_done[j & 1]);
         mma_commit(&v_empty[j & 1]);
@@ -404,36 +404,27 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    constexpr int HC = BN / 2;                                       // columns of a half
+    constexpr int HC = BN / 2;                                       // keys of a half
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;  // TMEM lane field
+    const uint32_t col_o = kColO + (uint32_t)ch * BM;               // this half's O_h
     const int q_pos = L - p.Tq + t_row;  // causal limit of this row
-    uint64_t* pair_bar = &xbar[warp & 3];
     float m_used = -INFINITY, l_sum = 0.f;
-    bool o_live = false;  // O holds data (first P.V has run)
+    bool o_live = false;  // O_h holds data (first P.V has run)
     bool ok = true;
-    // swap a value with the other half of this row (phase `ph` of the pair's barrier)
-    auto swap_half = [&](float mine, int ph) -> float {
-      xch[((ph & 1) * 2 + ch) * BM + srow] = mine;
-      __syncwarp();
-      mbar_arrive_if(pair_bar, lane == 0);
-      if (!mbar_wait_bounded(pair_bar, ph & 1, abort_flag)) ok = false;
-      return xch[((ph & 1) * 2 + (ch ^ 1)) * BM + srow];
-    };
     for (int j = 0; j < n_tiles && ok; ++j) {
       const int sb = j & 1;
       if (!mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       fence_after_sync();
+      const uint32_t col_s = (uint32_t)sb * BN + (uint32_t)ch * HC;  // this half's S columns
       float s[HC];
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) {
         float v[32];
-        tmem_ld32(tmem + lane_base + sb * BN + ch * HC + c * 32, v);
+        tmem_ld32(tmem + lane_base + col_s + c * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
       }
       tmem_wait_ld();
-      fence_before_sync();
-      mbar_arrive(&s_free[sb]);
       // mask (boundary tiles only) and the max of the raw scores (the scale is
       // positive, so max(s) * scale is the max of the base-2 logits); 8 chains
       const int kp0 = pos0 + j * BN;
@@ -455,21 +446,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       for (int c = 16; c < HC; c += 16)
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], fmaxf(s[c + u], s[c + 8 + u]));
-      const float hmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float tmax = p.qscale * fmaxf(hmax, swap_half(hmax, j));
-      if (!ok) break;
-      // P buffer j & 1 was last read by the P.V of tile j - 2: it must be complete
-      // (o_done[b] cannot run ahead by two phases: its next phase needs this P)
-      if (j >= 2 && !mbar_wait_bounded(&o_done[j & 1], ((j >> 1) - 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      fence_after_sync();
+      const float tmax = p.qscale * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                          fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       if (tmax > m_used + 8.f) {  // lazy rescale: only when the max grows by more than 2^8
         const float alpha = exp2f(m_used - tmax);  // 0 when m_used is -inf
         l_sum *= alpha;
-        if (o_live) {  // O must hold every P.V so far: wait for the one of tile j - 1
+        if (o_live) {  // O_h must hold every P.V so far: wait for the one of tile j - 1
           const int jp = j - 1;
           if (!mbar_wait_bounded(&o_done[jp & 1], (jp >> 1) & 1, abort_flag)) {
             ok = false;
@@ -477,22 +459,22 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           }
           fence_after_sync();
 #pragma unroll
-          for (int c = 0; c < HC / 32; ++c) {
+          for (int c = 0; c < BM / 32; ++c) {
             float v[32];
-            tmem_ld32(tmem + lane_base + kColO + ch * HC + c * 32, v);
+            tmem_ld32(tmem + lane_base + col_o + c * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= alpha;
-            tmem_st32(tmem + lane_base + kColO + ch * HC + c * 32, v);
+            tmem_st32(tmem + lane_base + col_o + c * 32, v);
           }
           tmem_wait_st();
         }
         m_used = tmax;
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      // P = 2^(s * scale - m) as bf16 pairs into this half of P buffer j & 1 in
-      // TMEM (this thread's lane); packed fp32x2 for the exponent argument and
-      // for l, which sums the unrounded values
+      // P_h = 2^(s * scale - m_h) as bf16 pairs over the first 32 of this half's S
+      // columns (already read); packed fp32x2 for the exponent argument and for
+      // l, which sums the unrounded values
       const f2 sc2 = pack2(p.qscale, p.qscale), nm2 = pack2(-mu, -mu);
       f2 ls2[4];
 #pragma unroll
@@ -513,7 +495,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           pw[c8 * 4 + u] = *reinterpret_cast<const uint32_t*>(&h2);
         }
       }
-      tmem_st32u(tmem + lane_base + kColP + (uint32_t)(j & 1) * (BN / 2) + ch * (HC / 2), pw);
+      tmem_st32u(tmem + lane_base + col_s, pw);
       tmem_wait_st();
       {
         const f2 t2 = fadd2(fadd2(ls2[0], ls2[1]), fadd2(ls2[2], ls2[3]));
@@ -543,30 +525,47 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       mbar_arrive(p_full);
       o_live = true;
     }
-    // ---- epilogue: O / l and log-sum-exp for this row (l summed over both halves)
+    // ---- epilogue: combine the two halves' (m, l, O) of this row
     if (ok && n_tiles > 0) {  // the last P.V (the tensor core runs them in order)
       const int jl = n_tiles - 1;
       if (!mbar_wait_bounded(&o_done[jl & 1], (jl >> 1) & 1, abort_flag)) ok = false;
     }
-    if (ok) l_sum += swap_half(l_sum, n_tiles);
+    float m_o = -INFINITY, l_o = 0.f;  // the other half's
+    {
+      xch[(0 * 2 + ch) * BM + srow] = m_used;
+      xch[(1 * 2 + ch) * BM + srow] = l_sum;
+      __syncwarp();
+      mbar_arrive_if(&xbar[warp & 3], lane == 0);
+      if (!mbar_wait_bounded(&xbar[warp & 3], 0, abort_flag)) ok = false;
+      m_o = xch[(0 * 2 + (ch ^ 1)) * BM + srow];
+      l_o = xch[(1 * 2 + (ch ^ 1)) * BM + srow];
+    }
     if (!ok) {
       dev_error(p.status, SKV_DEV_TIMEOUT);
       *abort_flag = 1;
     }
     fence_after_sync();
+    // weights of O_0 and O_1 (this thread's half is O_ch, the other O_(ch^1))
+    const float M = fmaxf(m_used, m_o);
+    const float w_me = (l_sum > 0.f) ? exp2f(m_used - M) : 0.f;
+    const float w_ot = (l_o > 0.f) ? exp2f(m_o - M) : 0.f;
+    const float Lt = l_sum * w_me + l_o * w_ot;
+    const float w0 = ch == 0 ? w_me : w_ot, w1 = ch == 0 ? w_ot : w_me;
+    // this thread writes output dims ch*64 .. ch*64+63 from both accumulators
     float o[HC];
     if (n_tiles > 0) {
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + kColO + ch * HC + c * 32, v);
+        float v0[32], v1[32];
+        tmem_ld32(tmem + lane_base + kColO + ch * HC + c * 32, v0);
+        tmem_ld32(tmem + lane_base + kColO + BM + ch * HC + c * 32, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[c * 32 + i] = v[i];
+        for (int i = 0; i < 32; ++i) o[c * 32 + i] = v0[i] * w0 + v1[i] * w1;
       }
-      tmem_wait_ld();
     }
     if (row_valid) {
-      const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
+      const float inv = (Lt > 0.f) ? 1.f / Lt : 0.f;
       const size_t rows = (size_t)p.B * p.Tq * p.Hq;
       const size_t row = ((size_t)b * p.Tq + t_row) * p.Hq + (size_t)kvh * p.G + grow % p.G;
       float4* dst = reinterpret_cast<float4*>(p.out + ((size_t)shard * rows + row) * kHeadDim + ch * HC);
@@ -579,7 +578,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       }
       if (ch == 0)
         p.lse[(size_t)shard * rows + row] =
-            (l_sum > 0.f) ? (m_used + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+            (Lt > 0.f) ? (M + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
     }
   }
   // ---- teardown: every tcgen05 operation is complete; free TMEM
