@@ -233,6 +233,60 @@ def test_art_other_group_sizes(G):
                 check_art(wl, res, b, kvh, q=q, tau=tau, phi=phi, patience=p)
 
 
+@pytest.mark.parametrize("tau,phi,p", [(2e-2, 2e-3, 2), (1e-2, 5e-4, 3)])
+def test_art_stops_across_many_chunks(tau, phi, p):
+    # 130..256 blocks per sequence (5..8 chunks of 32 blocks): heads of one group
+    # stop in different chunks (blocks ~38..214), some never; later chunks of a
+    # group keep running for the heads still live and pass stopped heads on
+    lens = [64 * 256, 64 * 200 + 17, 64 * 130]
+    wl = skvgen.Workload("am", B=3, Hq=8, Hkv=2, L=max(lens), lens=lens, structured=True,
+                         paging="perm", seed=61)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev, art=(tau, phi, p))
+    assert res[3] == 0
+    q = skvgen.host_q(wl)
+    flagged = 0
+    for b in range(3):
+        for kvh in range(2):
+            f, _, _ = check_art(wl, res, b, kvh, q=q, tau=tau, phi=phi, patience=p)
+            flagged += f
+    assert flagged <= 2
+
+
+def test_art_early_stop_skips_later_chunks():
+    # every test passes: each head stops after 1 + p blocks, inside the first
+    # chunk of sequences of up to 400 blocks; the chunks taken later issue no
+    # loads (or, if already in flight, pass the stopped state on)
+    p = 3
+    lens = [64 * 400, 64 * 333 + 5, 64 * 40, 64 * 2 + 1] * 2
+    wl = skvgen.Workload("ae", B=8, Hq=8, Hkv=2, L=max(lens), lens=lens, structured=True,
+                         paging="perm", seed=62, softmax_scale=0.3)
+    dev = device_workload(wl)
+    res = run_decode(wl, dev, art=(10.0, 2.5, p))
+    assert res[3] == 0
+    for b in range(wl.B):
+        assert np.all(res[2][b] == min(1 + p, wl.nb(b)))
+    q = skvgen.host_q(wl)
+    for b in (0, 1, 3):
+        for kvh in range(2):
+            check_art(wl, res, b, kvh, q=q, tau=10.0, phi=2.5, patience=p)
+
+
+def test_art_caller_order_across_chunks():
+    # a caller order over 150 blocks (5 chunks) that also lists block 0 again
+    torch = _torch()
+    wl = skvgen.Workload("ac", B=1, Hq=8, Hkv=2, L=64 * 150, structured=True, seed=63)
+    dev = device_workload(wl)
+    rng = np.random.default_rng(2)
+    order = np.stack([rng.permutation(150) for _ in range(2)])[None].astype(np.int32)
+    tau, phi, p = 2e-2, 2e-3, 2
+    res = run_decode(wl, dev, art=(tau, phi, p), order=torch.tensor(order, device="cuda"))
+    assert res[3] == 0
+    q = skvgen.host_q(wl)
+    for kvh in range(2):
+        check_art(wl, res, 0, kvh, order=list(order[0, kvh]), q=q, tau=tau, phi=phi, patience=p)
+
+
 def test_art_with_caller_order_skips_block0_in_list():
     torch = _torch()
     wl = skvgen.Workload("ao", B=1, Hq=8, Hkv=2, L=64 * 50, structured=True, seed=47)
