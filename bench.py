@@ -227,17 +227,22 @@ def _paged_inputs(torch, skvgen, wl, layer=0):
     return q, k_pool, v_pool, block_table, seq_lens
 
 
-def build_decode(torch, skv, skvgen, wl, status, art=False):
-    """Full-traversal (or ART) decode of one paged workload."""
-    q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, wl)
-    skvgen.device_kv_paged(wl, q, k_pool, v_pool, bt, sl)
+def build_decode(torch, skv, skvgen, wl, status, art=None, inputs=None):
+    """Full-traversal (or ART: art = (tau, phi, patience)) decode of one paged
+    workload; `inputs` = (q, k_pool, v_pool, block_table, seq_lens) of another
+    step to share its cache."""
+    if inputs is None:
+        q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, wl)
+        skvgen.device_kv_paged(wl, q, k_pool, v_pool, bt, sl)
+    else:
+        q, k_pool, v_pool, bt, sl = inputs
     out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
     lse = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
     consumed = torch.zeros((wl.B, wl.Hq), dtype=torch.int32, device="cuda")
     common = (q, k_pool, v_pool, bt, sl, out, lse)
     kw = dict(max_seq_len=wl.Lmax, scale=wl.scale, status=status, blocks_consumed=consumed)
-    if art:
-        kw["art"] = (wl.tau, wl.phi, wl.patience)
+    if art is not None:
+        kw["art"] = tuple(art)
     n = skv.decode_workspace_size(*common, **kw)
     ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda") if n else None
     a = skv.make_decode_args(*common, workspace=ws, **kw)
@@ -425,7 +430,19 @@ def main():
         step = build_chunk(torch, skv, skvgen, wl, status)
     else:
         raise SystemExit(f"workload {args.workload}: no bench step")
-    art_step = build_decode(torch, skv, skvgen, wl, status, art=True) if (kind == "cfg2" and not args.no_art) else None
+    art_step, sweep_steps, dense_step = None, [], None
+    if kind == "cfg2" and not args.no_art:
+        T = step.tensors
+        shared = (T["q"], T["k_pool"], T["v_pool"], T["bt"], T["sl"])
+        art_step = build_decode(torch, skv, skvgen, wl, status, art=(wl.tau, wl.phi, wl.patience),
+                                inputs=shared)
+        # looser thresholds on the same cache, where heads do stop: savings vs blocks skipped
+        for thr in ((5e-2, 5e-3, 2), (2e-2, 2e-3, 2)):
+            sweep_steps.append((thr, build_decode(torch, skv, skvgen, wl, status, art=thr, inputs=shared)))
+    if kind == "cfg3":  # the same cache walked in full, for the savings of the selection
+        T = step.tensors
+        dense_step = build_decode(torch, skv, skvgen, wl, status,
+                                  inputs=(T["q"], T["k_pool"], T["v_pool"], T["bt"], T["sl"]))
     stream = torch.cuda.current_stream()
 
     def timed(st, steps, warmup):
@@ -468,6 +485,10 @@ def main():
         art_ms = None
         if art_step is not None:
             art_ms, _ = timed(art_step, args.steps, args.warmup)
+        sweep_ms = [timed(st, max(10, args.steps // 4), args.warmup)[0] / max(10, args.steps // 4)
+                    for _, st in sweep_steps]
+        dense_ms = (timed(dense_step, max(10, args.steps // 4), args.warmup)[0] / max(10, args.steps // 4)
+                    if dense_step is not None else None)
     clocks = clk.summary()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status word {int(status.item()):#x}")
@@ -560,6 +581,23 @@ def main():
                       "attended_tokens_per_s": float(cons.sum()) * wl.bs / (art_step_ms * 1e-3),
                       "tau": wl.tau, "phi": wl.phi, "patience": wl.patience}
         res["gpu_launches"] += args.steps * art_step.launches
+
+        def art_summary(st, ms):
+            cons = st.tensors["consumed"].cpu().numpy()
+            grp = cons.reshape(wl.B, wl.Hkv, wl.G).max(axis=2)
+            skipped = 1.0 - float(grp.sum()) / (wl.B * wl.Hkv * wl.nb(0))
+            saved = 1.0 - ms / ms_step
+            return {"ms_per_step": ms, "blocks_skipped_frac": skipped, "time_saved_frac": saved,
+                    "saved_per_skipped": saved / skipped if skipped > 0 else None,
+                    "blocks_consumed_mean": float(cons.mean())}
+        res["art_sweep"] = [dict(tau=thr[0], phi=thr[1], patience=thr[2], **art_summary(st, ms))
+                            for (thr, st), ms in zip(sweep_steps, sweep_ms)]
+        res["gpu_launches"] += sum(max(10, args.steps // 4) * st.launches for _, st in sweep_steps)
+    if dense_ms is not None:
+        res["selection"] = {"dense_ms_per_step": dense_ms, "time_vs_dense": ms_step / dense_ms,
+                            "bytes_vs_dense": step.nbytes / wl.kv_bytes(),
+                            "note": "same cache walked in full by the plain decode kernel"}
+        res["gpu_launches"] += max(10, args.steps // 4) * dense_step.launches
     if e2e is not None:
         res["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline and kind in ("cfg1", "cfg2"):

@@ -107,14 +107,15 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     probe.order_len = a->order_len;
     pl->sched = SCHED_ART;
     pl->nw = 1;
-    pl->art_chunk = art_chunk_blocks(G);
-    pl->art_maxc = (int)cdiv(art_positions(probe, a->max_seq_len), pl->art_chunk);
+    pl->n_ctas = num_sms() * art_ctas_per_sm(G);
+    const long long positions = art_positions(probe, a->max_seq_len);
+    pl->art_chunk = art_chunk_blocks(G, pl->n_ctas, groups, positions);
+    pl->art_maxc = (int)cdiv(positions, pl->art_chunk);
     const long long items = groups * pl->art_maxc;
     if (items >= (1ll << 30) || pl->art_maxc > 32768) return SKV_EUNSUPPORTED;
-    pl->n_ctas = num_sms() * art_ctas_per_sm(G);
     pl->hdr_bytes = (size_t)cdiv(art_ctl_words(groups, pl->art_maxc, G) * 4, 256) * 256;
     pl->lb_bytes = (size_t)cdiv(items * G * kLbFloats * 4, 256) * 256;
-    pl->scratch_bytes = (size_t)pl->n_ctas * art_scratch_bytes_per_cta(G);
+    pl->scratch_bytes = (size_t)pl->n_ctas * art_scratch_bytes_per_cta(G, pl->art_chunk);
     pl->ws_bytes = pl->hdr_bytes + pl->lb_bytes + pl->scratch_bytes +
                    (size_t)items * G * kRecFloats * sizeof(float);
     return SKV_OK;

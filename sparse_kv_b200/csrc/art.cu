@@ -35,10 +35,10 @@
 // (they stay in L2), which leaves the shared memory to a 3-stage ring at two
 // CTAs per SM.
 // A head that stops inside a chunk needs its state after the stop block, which
-// the consumers have already passed: the judge posts a request, and at a later
-// chunk boundary the consumers re-fold that chunk's blocks up to the stop for
-// the stopping heads straight from the pool in global memory (once per head;
-// the pages are usually still in L2); the judge overwrites the record.
+// the consumers have already passed: the judge queues a request, the producer
+// streams that chunk's blocks up to the stop once more through the ring (the
+// pages are usually still in L2) as tagged tiles, and the consumers fold them
+// for the stopping heads only; the judge overwrites the record.
 // Chunks taken after every head of a group has stopped issue no loads.
 // attn_decode's merge combines each head's records up to its stop chunk,
 // which is exact.
@@ -46,12 +46,9 @@
 #include "decode.cuh"
 #include "tile.cuh"
 
-// consumer warps per CTA, blocks per chunk, resident CTAs per SM (1 or 2)
+// consumer warps per CTA, resident CTAs per SM (1 or 2); SKV_ART_CHUNK forces the chunk length
 #ifndef SKV_ART_WARPS
 #define SKV_ART_WARPS 8
-#endif
-#ifndef SKV_ART_CHUNK
-#define SKV_ART_CHUNK 32
 #endif
 #ifndef SKV_ART_CTAS_PER_SM
 #define SKV_ART_CTAS_PER_SM 2
@@ -63,6 +60,9 @@ namespace {
 constexpr int kProbeFloats = 12;  // per (block, warp, head): m, l, pad, pad, O[0:8]
 constexpr int kReqs = 32;         // re-run requests in flight (a few chunks' worth)
 enum PostKind : int { POST_END = 1, POST_FIX = 2, POST_QUIT = 3, POST_DONE = 4 };
+// ring entry tags (meta.w): block in chunk (bits 0..7), request slot (8..15), re-fold flag
+constexpr int kFixTag = 1 << 30;
+constexpr int kDrainEntry = -2;  // meta.x of the entry that ends the items (before re-folds)
 
 constexpr size_t up16(size_t x) { return (x + 15) / 16 * 16; }
 
@@ -89,8 +89,7 @@ struct ArtCfg {  // shared-memory layout
   static constexpr size_t OFF_META = up16(OFF_BAR + NBAR * 8);        // int4 [ST]
   static constexpr size_t OFF_FLAGS = up16(OFF_META + ST * 16);       // int [4]
   static constexpr size_t OFF_TAG = OFF_FLAGS + 16;                   // int [2][4]
-  static constexpr size_t OFF_RTAG = OFF_TAG + 32;                    // int [2] (+ pad)
-  static constexpr size_t OFF_REQ = OFF_RTAG + 16;                    // int [kReqs][4] + int [kReqs][G]
+  static constexpr size_t OFF_REQ = OFF_TAG + 32;                     // int [kReqs][4] + int [kReqs][G]
   static constexpr size_t OFF_P = up16(OFF_REQ + kReqs * 16 + (size_t)kReqs * G * 4);  // float2 [NW][RPW][G]
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;   // float2 [NW][G]
   static constexpr size_t OFF_WCTL = up16(OFF_A + (size_t)NW * G * 8);  // int [NW][8]
@@ -158,10 +157,10 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   uint64_t* freed = posted + 2;     // [2] the judge is done with a post
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows | 0 = end of chunk, group, chunk, block in chunk | blocks}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
-  // flags[1]: abort (a bounded wait expired); flags[2]: consumers finished
-  // (entries consumed + 1)
+  // flags[0]: re-fold requests posted by the judge; flags[1]: abort (a bounded
+  // wait expired); flags[2]: consumers finished (entries consumed + 1);
+  // flags[3]: the judge has handled every chunk (no more requests)
   volatile int* tag = reinterpret_cast<volatile int*>(smem + C::OFF_TAG);    // [2][4]: kind, group, chunk, a
-  volatile int* rtag = reinterpret_cast<volatile int*>(smem + C::OFF_RTAG);  // [2] requests posted
   volatile int* req = reinterpret_cast<volatile int*>(smem + C::OFF_REQ);  // [kReqs][4]: group, chunk, vmask, stopmask
   volatile int* req_t = reinterpret_cast<volatile int*>(smem + C::OFF_REQ + kReqs * 16);  // [kReqs][G]
   float* probe = p.art_scratch + (size_t)blockIdx.x * scratch_floats<G, NW, CB>();  // [2][CB][NW][G][12]
@@ -226,9 +225,56 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       return true;
     };
     const long long items = (long long)groups * p.art_maxc;
+    // Re-fold request r: the chunk's blocks up to the last stop block, tagged,
+    // then a tagged end marker.  The request slot stays valid until the judge has
+    // taken the re-fold's post (it never has more than kReqs outstanding).
+    auto serve = [&](int r) {
+      const int slot = r % kReqs;
+      __threadfence_block();
+      const int g = req[slot * 4], c = req[slot * 4 + 1];
+      const uint32_t vm = (uint32_t)req[slot * 4 + 2], stop = (uint32_t)req[slot * 4 + 3];
+      int tmax = -1;
+      for (int h = 0; h < G; ++h)
+        if ((stop >> h) & 1u) tmax = max(tmax, req_t[slot * G + h]);
+      const int b = g / p.Hkv, kvh = g % p.Hkv;
+      int L = p.seq_lens[b];
+      if (L < 0 || L > p.max_seq_len) L = 0;
+      const int nb = (L + kBlock - 1) / kBlock;
+      const int* ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)g * p.order_len : nullptr;
+      const int* bt = p.block_table + (size_t)b * p.max_blocks;
+      int n = 0, page = 0;
+      if (lane <= tmax && ((vm >> lane) & 1u)) {
+        const int blk = art_block(p, ord, nb, c * CB + lane, nullptr);
+        page = bt[blk];  // validated when the block was first loaded
+        n = min(kBlock, L - blk * kBlock);
+      }
+      const uint16_t* qsrc = p.q + ((size_t)b * p.Hq + (size_t)kvh * G) * kHeadDim;
+      bool first = true;
+      for (int t = 0; t <= tmax && ok; ++t) {
+        if (!((vm >> t) & 1u)) continue;
+        const int nt = __shfl_sync(0xffffffffu, n, t), pgt = __shfl_sync(0xffffffffu, page, t);
+        int r1 = 1;
+        if (lane == 0) r1 = emit(nt, g, c, kFixTag | (slot << 8) | t, pgt, kvh, first ? qsrc : nullptr);
+        ok = __shfl_sync(0xffffffffu, r1, 0) != 0;
+        first = false;
+      }
+      if (ok) {
+        int r1 = 1;
+        if (lane == 0) r1 = emit(0, g, c, kFixTag | (slot << 8), 0, 0, nullptr);
+        ok = __shfl_sync(0xffffffffu, r1, 0) != 0;
+      }
+    };
+    int taken = 0;  // requests served
+    auto serve_pending = [&]() {
+      int posted = (lane == 0) ? flags[0] : 0;
+      posted = __shfl_sync(0xffffffffu, posted, 0);
+      while (ok && taken < posted) serve(taken++);
+    };
     long long w = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
     w = __shfl_sync(0xffffffffu, w, 0);
-    while (ok && w < items) {
+    while (ok) {
+      serve_pending();
+      if (w >= items) break;
       const long long w_next = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
       const int c = (int)(w / groups), g = (int)(w % groups);
       const int b = g / p.Hkv, kvh = g % p.Hkv;
@@ -266,6 +312,14 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         const uint16_t* qsrc = p.q + ((size_t)b * p.Hq + (size_t)kvh * G) * kHeadDim;
         for (int i = 0; i < npos && ok; ++i) {
           if (!((vm >> i) & 1u)) continue;
+          if ((i & 7) == 7) {  // the group may have stopped meanwhile: cut the chunk short
+            int stopped = 0;
+            if (lane == 0) {
+              const int sc = *reinterpret_cast<volatile int*>(ctl.stop_chunk + g);
+              stopped = sc != 0 && c >= sc;
+            }
+            if (__shfl_sync(0xffffffffu, stopped, 0)) break;
+          }
           const int ni = __shfl_sync(0xffffffffu, n, i), pgi = __shfl_sync(0xffffffffu, page, i);
           int r = 1;
           if (lane == 0) r = emit(ni, g, c, i, pgi, kvh, (vm & ((1u << i) - 1u)) ? nullptr : qsrc);
@@ -279,6 +333,28 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       }
       w = __shfl_sync(0xffffffffu, w_next, 0);
     }
+    // no more items: the consumers hand the judge a QUIT post; once the judge has
+    // handled every chunk, serve the last requests, then end the ring
+    if (ok) {
+      int r = 1;
+      if (lane == 0) r = emit(kDrainEntry, -1, 0, 0, 0, 0, nullptr);
+      ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+    }
+    if (ok) {
+      int done = 1;
+      if (lane == 0) {
+        const uint64_t t0 = globaltimer();
+        while (flags[3] == 0) {
+          if (flags[1] != 0 || globaltimer() - t0 > kWaitLimitNs) {
+            fail();
+            done = 0;
+            break;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, done, 0) != 0;
+    }
+    if (ok) serve_pending();
     if (lane != 0) return;
     if (ok) emit(-1, -1, 0, 0, 0, 0, nullptr);
     // Copies the consumers never waited for (abort) must land before the CTA
@@ -595,6 +671,8 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
               req[r * 4 + 3] = (int)stopmask;
 #pragma unroll
               for (int h = 0; h < G; ++h) req_t[r * G + h] = st[h];
+              __threadfence_block();
+              flags[0] = n_req + 1;  // the producer serves it between items
             }
             ++n_req;
           }
@@ -602,9 +680,10 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       } else if (kind == POST_FIX) {
         reduce_states(st_area, tg_g, tg_c, (uint32_t)tg_a);
         ++n_fix;
+      } else if (kind == POST_QUIT) {
+        __syncwarp();
+        if (lane == 0) flags[3] = 1;  // every chunk handled: no more requests
       }
-      __syncwarp();
-      if (lane == 0) rtag[par] = n_req;
       __syncwarp();
       mbar_arrive_if(&freed[par], lane == 0);
       ++kj;
@@ -621,28 +700,21 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
   // Warp-uniform counters used at chunk boundaries live in shared memory (one
   // block per warp): the fold loop is register-bound.
-  enum { W_KP = 0, W_RSEEN, W_RDONE, W_DRAIN, W_CURG, W_CURC };
+  enum { W_KP = 0, W_CURG, W_CURC, W_CURK };
   volatile int* wc = reinterpret_cast<volatile int*>(smem + C::OFF_WCTL) + warp * 8;
   wc[W_KP] = 0;      // posts made
-  wc[W_RSEEN] = 0;   // requests the judge had posted when it freed our buffer
-  wc[W_RDONE] = 0;   // requests served
-  wc[W_DRAIN] = 0;   // the producer's end entry has been seen
-  wc[W_CURG] = -1;   // chunk being folded
+  wc[W_CURG] = -1;   // item being folded: group, chunk, re-fold slot (-1: the chunk itself)
   wc[W_CURC] = -1;
-  int kpar = 0;  // parity of the next post (its buffers hold the current chunk)
+  wc[W_CURK] = -1;
+  int kpar = 0;  // parity of the next post (its buffers hold the current item)
   bool ok = true;
 
-  // Take the buffer of the next post (the judge is done with the post two
-  // back).  Every warp reads the judge's request count at the same handshake,
-  // so all take the same decisions.
+  // Take the buffers of the next post (the judge is done with the post two back).
   auto acquire = [&]() {
     const int kp = wc[W_KP];
-    if (kp >= 2) {
-      if (!mbar_wait_bounded(&freed[kp & 1], ((kp >> 1) - 1) & 1, &flags[1])) {
-        if (lane == 0) fail();
-        ok = false;
-      }
-      wc[W_RSEEN] = rtag[kp & 1];
+    if (kp >= 2 && !mbar_wait_bounded(&freed[kp & 1], ((kp >> 1) - 1) & 1, &flags[1])) {
+      if (lane == 0) fail();
+      ok = false;
     }
   };
   auto publish = [&](int kind, int g, int c, int a) {
@@ -677,130 +749,63 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
             make_float2(W.m_st[j], W.l_st[j]);
     }
   };
-  // Re-fold of a chunk for the heads that stop in it (a request of the judge):
-  // the chunk's blocks up to each head's stop block, from the pool.  Only the
-  // request index and the next block live in registers; the rest is re-read
-  // from the request slot (this path is rare, the fold loop is register-bound).
-  int rr = -1, rr_t = 0;
-  uint32_t done_mask = 0;
-  auto start_request = [&]() -> bool {
-    const int req_done = wc[W_RDONE];
-    if (req_done >= wc[W_RSEEN] || !ok) return false;
-    rr = req_done % kReqs;
-    rr_t = 0;
-    const int g = req[rr * 4];
-    const int b = g / p.Hkv, kvh = g % p.Hkv;
-    W.reset();
-    W.load_q(p.q, (size_t)b * p.Hq + (size_t)kvh * G, p.qscale, lane);
-    done_mask = ~(uint32_t)req[rr * 4 + 3];
-    return true;
-  };
 
   int s = 0, e = 0;  // ring stage, ring entries consumed
   uint32_t ph = 0;
-  uint32_t vmask = 0;
-  while (ok) {
-    const unsigned char* sK;
-    const unsigned char* sV;
-    int nv, pos = 0;
-    const bool from_ring = rr < 0;
-    if (!from_ring) {
-      const int rg = req[rr * 4], rc = req[rr * 4 + 1];
-      const uint32_t rvm = (uint32_t)req[rr * 4 + 2], rstop = (uint32_t)req[rr * 4 + 3];
-      int tmax = -1;
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        if ((rstop >> h) & 1u) tmax = max(tmax, req_t[rr * G + h]);
-      while (rr_t <= tmax && !((rvm >> rr_t) & 1u)) ++rr_t;
-      if (rr_t > tmax) {  // request complete: its states go to the judge
-        acquire();
-        write_state();
-        publish(POST_FIX, rg, rc, (int)rstop);
-        wc[W_RDONE] = wc[W_RDONE] + 1;
-        rr = -1;
-        wc[W_CURG] = -1;  // the registers were used: reload at the next block
-        if (!start_request() && wc[W_DRAIN]) {
-          acquire();
-          publish(POST_DONE, 0, 0, 0);
-          break;
-        }
-        continue;
-      }
-      const int b = rg / p.Hkv, kvh = rg % p.Hkv;
-      int L = p.seq_lens[b];
-      if (L < 0 || L > p.max_seq_len) L = 0;
-      const int* ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)rg * p.order_len : nullptr;
-      const int blk = art_block(p, ord, (L + kBlock - 1) / kBlock, rc * CB + rr_t, nullptr);
-      const int page = p.block_table[(size_t)b * p.max_blocks + blk];  // validated at load
-      const size_t off = ((size_t)page * p.Hkv + kvh) * kBlock * kHeadDim;
-      sK = reinterpret_cast<const unsigned char*>(p.k_pool + off);
-      sV = reinterpret_cast<const unsigned char*>(p.v_pool + off);
-      nv = min(kBlock, L - blk * kBlock) - rb;
-    } else {
-      if (!mbar_wait_bounded(&full[s], ph, &flags[1])) {
-        if (lane == 0) fail();
-        ok = false;
-        break;
-      }
-      const int4 mt = meta[s];
-      const int n = mt.x;
-      if (n < 0) {
-        // end of the traversal: once the judge has handled every chunk (the
-        // QUIT post's handshake), serve the last requests, then release it
-        wc[W_DRAIN] = 1;
-        acquire();
-        publish(POST_QUIT, 0, 0, 0);
-        const int kq = wc[W_KP] - 1;
-        if (!mbar_wait_bounded(&freed[kq & 1], (kq >> 1) & 1, &flags[1])) {
-          if (lane == 0) fail();
-          ok = false;
-          break;
-        }
-        wc[W_RSEEN] = rtag[kq & 1];
-        if (!start_request()) {
-          acquire();
-          publish(POST_DONE, 0, 0, 0);
-          break;
-        }
-        continue;
-      }
-      if (mt.y != wc[W_CURG] || mt.z != wc[W_CURC]) {  // a new chunk: take the next post's buffers
-        acquire();
-        wc[W_CURG] = mt.y;
-        wc[W_CURC] = mt.z;
-        W.reset();
-        if (n > 0)  // the chunk's first block carries the group's q rows
-          W.load_q(reinterpret_cast<const uint16_t*>(smem + s * C::STAGE_BYTES + 2 * kTileBytes), 0,
-                   p.qscale, lane);
-        vmask = 0;
-        done_mask = 0;
-      }
-      if (n == 0) {  // end of chunk
-        mbar_arrive_if(&empty[s], lane == 0);
-        ++e;
-        if (++s == ST) {
-          s = 0;
-          ph ^= 1u;
-        }
-        write_state();
-        publish(POST_END, mt.y, mt.z, (int)vmask);
-        start_request();
-        continue;
-      }
-      sK = smem + s * C::STAGE_BYTES;
-      sV = sK + kTileBytes;
-      nv = n - rb;
-      pos = mt.w;
+  uint32_t vmask = 0, done_mask = 0;
+  auto release = [&]() {
+    mbar_arrive_if(&empty[s], lane == 0);
+    ++e;
+    if (++s == ST) {
+      s = 0;
+      ph ^= 1u;
     }
+  };
+  while (ok) {
+    if (!mbar_wait_bounded(&full[s], ph, &flags[1])) {
+      if (lane == 0) fail();
+      ok = false;
+      break;
+    }
+    const int4 mt = meta[s];
+    const int n = mt.x;
+    if (n == -1) break;
+    if (n == kDrainEntry) {  // no more items: let the judge finish, re-folds may follow
+      release();
+      acquire();
+      publish(POST_QUIT, 0, 0, 0);
+      continue;
+    }
+    const bool fix = (mt.w & kFixTag) != 0;
+    const int slot = fix ? ((mt.w >> 8) & 0xFF) : -1;
+    if (mt.y != wc[W_CURG] || mt.z != wc[W_CURC] || slot != wc[W_CURK]) {
+      // a new item (a chunk, or the re-fold of one): take the next post's buffers
+      acquire();
+      wc[W_CURG] = mt.y;
+      wc[W_CURC] = mt.z;
+      wc[W_CURK] = slot;
+      W.reset();
+      if (n > 0)  // an item's first block carries the group's q rows
+        W.load_q(reinterpret_cast<const uint16_t*>(smem + s * C::STAGE_BYTES + 2 * kTileBytes), 0,
+                 p.qscale, lane);
+      vmask = 0;
+      __threadfence_block();
+      done_mask = fix ? ~(uint32_t)req[slot * 4 + 3] : 0u;  // a re-fold folds its stopping heads only
+    }
+    if (n == 0) {  // end of the item
+      release();
+      write_state();
+      publish(fix ? POST_FIX : POST_END, mt.y, mt.z, fix ? req[slot * 4 + 3] : (int)vmask);
+      continue;
+    }
+    const unsigned char* sK = smem + s * C::STAGE_BYTES;
+    const unsigned char* sV = sK + kTileBytes;
+    const int nv = n - rb;
     if (nv >= C::RPW) fold_tile<G, NW, false>(W, sK, sV, nv, done_mask, pbuf, abuf);
     else fold_tile<G, NW, true>(W, sK, sV, nv, done_mask, pbuf, abuf);
-    if (from_ring) {
-      mbar_arrive_if(&empty[s], lane == 0);
-      ++e;
-      if (++s == ST) {
-        s = 0;
-        ph ^= 1u;
-      }
+    release();
+    const int pos = mt.w & 0xFF;
+    if (!fix) {
       // this warp's running state after block `pos` of the chunk
       vmask |= 1u << pos;
       float* pw = probe + (size_t)kpar * probe_floats<G, NW, CB>() +
@@ -820,11 +825,15 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         }
       }
     } else {
+      // a stopping head takes no block after its stop block
 #pragma unroll
       for (int h = 0; h < G; ++h)
-        if (req_t[rr * G + h] == rr_t) done_mask |= 1u << h;
-      ++rr_t;
+        if (req_t[slot * G + h] == pos) done_mask |= 1u << h;
     }
+  }
+  if (ok) {  // release the judge
+    acquire();
+    publish(POST_DONE, 0, 0, 0);
   }
   __syncwarp();
   mbar_arrive_if(fin_bar, lane == 0);
@@ -834,22 +843,20 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   }
 }
 
-// Chunk length, resident CTAs per SM, and the deepest ring (up to 6 stages)
-// that fits in the shared memory of one CTA.
-template <int G> constexpr int art_cb() { return SKV_ART_CHUNK; }
+// Resident CTAs per SM, and the deepest ring (up to 6 stages) that fits in
+// the shared memory of one CTA.
 template <int G> constexpr int art_minb() { return G == 8 ? 1 : SKV_ART_CTAS_PER_SM; }
-template <int G, int NW>
+template <int G, int NW, int CB>
 constexpr int art_st() {
   const size_t budget = (art_minb<G>() == 2 ? 113 : 227) * 1024;
   int st = 6;
-  while (st > 2 && ArtCfg<G, NW, art_cb<G>(), 6>::TOTAL - (size_t)(6 - st) * 2 * kTileBytes > budget)
-    --st;
+  while (st > 2 && ArtCfg<G, NW, CB, 6>::TOTAL - (size_t)(6 - st) * 2 * kTileBytes > budget) --st;
   return st;
 }
 
-template <int G>
+template <int G, int CB>
 int launch_art_t(const DecodeParams& p, cudaStream_t st) {
-  constexpr int NW = SKV_ART_WARPS, CB = art_cb<G>(), ST = art_st<G, NW>(), MINB = art_minb<G>();
+  constexpr int NW = SKV_ART_WARPS, ST = art_st<G, NW, CB>(), MINB = art_minb<G>();
   using C = ArtCfg<G, NW, CB, ST>;
   static_assert(C::TOTAL <= (MINB == 2 ? 113 : 227) * 1024, "shared memory budget");
   static_assert(ST >= 3, "a ring of at least three stages");
@@ -867,36 +874,49 @@ int launch_art_t(const DecodeParams& p, cudaStream_t st) {
   return (int)cudaGetLastError();
 }
 
+template <int G>
+int launch_art_g(const DecodeParams& p, cudaStream_t st) {
+  return p.art_chunk == 16 ? launch_art_t<G, 16>(p, st) : launch_art_t<G, 32>(p, st);
+}
+
 }  // namespace
 
 int art_ctas_per_sm(int G) { return G == 8 ? art_minb<8>() : art_minb<4>(); }
 
-int art_chunk_blocks(int G) {
-  switch (G) {
-    case 1: return art_cb<1>();
-    case 2: return art_cb<2>();
-    case 4: return art_cb<4>();
-    default: return art_cb<8>();
-  }
+// Chunk length: 32 blocks, or 16 when the speculation window would be large.
+// About n_ctas / groups chunks of a group are in flight when one of its stops
+// is decided, and all of them are read in vain; keep that within 1/12 of the
+// traversal.  Shorter chunks cost more judging per block, so they are used
+// only where the window needs them.
+int art_chunk_blocks(int G, long long n_ctas, long long groups, long long positions) {
+  (void)G;
+#ifdef SKV_ART_CHUNK
+  return SKV_ART_CHUNK;
+#else
+  const double in_flight = (double)n_ctas / (double)(groups > 0 ? groups : 1);
+  return (in_flight * 32.0 <= (double)positions / 12.0) ? 32 : 16;
+#endif
 }
 
-size_t art_scratch_bytes_per_cta(int G) {
+size_t art_scratch_bytes_per_cta(int G, int CB) {
   constexpr int NW = SKV_ART_WARPS;
+  const bool s = CB == 16;
   switch (G) {
-    case 1: return scratch_floats<1, NW, art_cb<1>()>() * 4;
-    case 2: return scratch_floats<2, NW, art_cb<2>()>() * 4;
-    case 4: return scratch_floats<4, NW, art_cb<4>()>() * 4;
-    default: return scratch_floats<8, NW, art_cb<8>()>() * 4;
+    case 1: return (s ? scratch_floats<1, NW, 16>() : scratch_floats<1, NW, 32>()) * 4;
+    case 2: return (s ? scratch_floats<2, NW, 16>() : scratch_floats<2, NW, 32>()) * 4;
+    case 4: return (s ? scratch_floats<4, NW, 16>() : scratch_floats<4, NW, 32>()) * 4;
+    default: return (s ? scratch_floats<8, NW, 16>() : scratch_floats<8, NW, 32>()) * 4;
   }
 }
 
 int launch_art(const DecodeParams& p, int G, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p.art_chunk != 16 && p.art_chunk != 32) return (int)cudaErrorInvalidValue;
   switch (G) {
-    case 1: return launch_art_t<1>(p, st);
-    case 2: return launch_art_t<2>(p, st);
-    case 4: return launch_art_t<4>(p, st);
-    case 8: return launch_art_t<8>(p, st);
+    case 1: return launch_art_g<1>(p, st);
+    case 2: return launch_art_g<2>(p, st);
+    case 4: return launch_art_g<4>(p, st);
+    case 8: return launch_art_g<8>(p, st);
     default: return (int)cudaErrorInvalidValue;
   }
 }

@@ -108,9 +108,9 @@ int launch_decode(const DecodeParams& p, int G, void* stream);
 int decode_consumer_warps(int G);
 int decode_ctas_per_sm(int G);
 int launch_art(const DecodeParams& p, int G, void* stream);
-int art_chunk_blocks(int G);
+int art_chunk_blocks(int G, long long n_ctas, long long groups, long long positions);
 int art_ctas_per_sm(int G);
-size_t art_scratch_bytes_per_cta(int G);
+size_t art_scratch_bytes_per_cta(int G, int CB);
 int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int d, float* out,
                  float* lse, void* stream);
 int launch_merge_records(const DecodeParams& p, int G, void* stream);
