@@ -11,6 +11,10 @@
 #include "common.cuh"
 #include "decode.cuh"
 
+#ifndef SKV_ART_AHEAD
+#define SKV_ART_AHEAD 0
+#endif
+
 namespace skv {
 namespace {
 
@@ -27,7 +31,7 @@ struct Plan {
   size_t lb_bytes = 0;    // ART look-back records
   size_t scratch_bytes = 0;  // ART per-CTA scratch
   size_t ws_bytes = 0;
-  int art_chunk = 0, art_maxc = 0;
+  int art_chunk = 0, art_maxc = 0, art_ahead = 0;
 };
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -111,6 +115,11 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     const long long positions = art_positions(probe, a->max_seq_len);
     pl->art_chunk = art_chunk_blocks(G, pl->n_ctas, groups, positions);
     pl->art_maxc = (int)cdiv(positions, pl->art_chunk);
+    // speculation gate (SKV_ART_AHEAD > 0: that many times the chunks in flight
+    // per group at the start), off by default
+    pl->art_ahead = SKV_ART_AHEAD > 0
+                        ? (int)(SKV_ART_AHEAD * std::max<long long>(1, cdiv(pl->n_ctas, groups)))
+                        : (1 << 30);
     const long long items = groups * pl->art_maxc;
     if (items >= (1ll << 30) || pl->art_maxc > 32768) return SKV_EUNSUPPORTED;
     pl->hdr_bytes = (size_t)cdiv(art_ctl_words(groups, pl->art_maxc, G) * 4, 256) * 256;
@@ -211,6 +220,7 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
   if (pl.art) {
     p.art_chunk = pl.art_chunk;
     p.art_maxc = pl.art_maxc;
+    p.art_ahead = pl.art_ahead;
     p.art_ctl = reinterpret_cast<int*>(ws);
     p.art_lb = reinterpret_cast<float*>(ws + pl.hdr_bytes);
     p.art_scratch = reinterpret_cast<float*>(ws + pl.hdr_bytes + pl.lb_bytes);

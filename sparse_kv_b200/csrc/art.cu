@@ -16,20 +16,23 @@
 // order from an atomic counter.  Three roles per CTA:
 //   producer   one lane streams each chunk's blocks through a TMA ring
 //              (bulk copies, no multicast), exactly like the plain decode
-//              kernel, and ends each chunk with a marker entry;
+//              kernel; the chunk's last tile carries its end (a chunk that
+//              loads nothing, or is cut short, ends with a marker entry).  The
+//              next item is taken and its pages looked up while the current
+//              chunk's first tiles are in flight;
 //   consumers  NW warps fold every block into their online-softmax states
 //              (tile.cuh) and leave (m, l, O[0:8]) of their state after every
 //              block in a per-CTA scratch area; at the end of a chunk each
 //              warp writes its whole state and posts the chunk to the judge.
 //              They never meet and never wait for a decision;
 //   judge      one warp combines the warps' probes into the chunk-local prefix
-//              after every block (lane = (block, head)) and their states into
-//              the chunk's record, waits for the previous chunk's published
-//              prefix (m, l, O[0:8], run of passing tests, blocks consumed or
-//              the stop) -- a decoupled look-back, as in single-pass parallel
-//              prefix scans -- evaluates the test for all CB blocks at once
+//              after every block (lane = (block, head)), waits for the
+//              previous chunk's published prefix (m, l, O[0:8], run of passing
+//              tests, blocks consumed or the stop) -- a decoupled look-back,
+//              as in single-pass parallel prefix scans -- evaluates the test for all CB blocks at once
 //              (lane t: block t; the patience run by warp ballots) and
-//              publishes the inclusive prefix.
+//              publishes the inclusive prefix; only then does it reduce the
+//              warps' states into the chunk's record, which no decision needs.
 // Posts alternate between two buffers, so the consumers run a chunk ahead of
 // the judge.  The probes and states live in global memory rewritten in place
 // (they stay in L2), which leaves the shared memory to a 3-stage ring at two
@@ -39,7 +42,10 @@
 // streams that chunk's blocks up to the stop once more through the ring (the
 // pages are usually still in L2) as tagged tiles, and the consumers fold them
 // for the stopping heads only; the judge overwrites the record.
-// Chunks taken after every head of a group has stopped issue no loads.
+// Chunks taken after every head of a group has stopped issue no loads, and a
+// chunk in flight is cut short (checked every 8 tiles).  An optional gate
+// (DecodeParams::art_ahead) holds a group's chunk c until chunk c - ahead - 1
+// is judged, bounding the reads past a stop at the price of idle CTAs.
 // attn_decode's merge combines each head's records up to its stop chunk,
 // which is exact.
 #include "common.cuh"
@@ -60,7 +66,10 @@ namespace {
 constexpr int kProbeFloats = 12;  // per (block, warp, head): m, l, pad, pad, O[0:8]
 constexpr int kReqs = 32;         // re-run requests in flight (a few chunks' worth)
 enum PostKind : int { POST_END = 1, POST_FIX = 2, POST_QUIT = 3, POST_DONE = 4 };
-// ring entry tags (meta.w): block in chunk (bits 0..7), request slot (8..15), re-fold flag
+// ring entry tags (meta.w): block in chunk (bits 0..7), request slot (8..15), last
+// chunk of the group, last tile of the chunk, re-fold flag
+constexpr int kLastChunkTag = 1 << 28;
+constexpr int kLastTag = 1 << 29;
 constexpr int kFixTag = 1 << 30;
 constexpr int kDrainEntry = -2;  // meta.x of the entry that ends the items (before re-folds)
 
@@ -270,68 +279,140 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       posted = __shfl_sync(0xffffffffu, posted, 0);
       while (ok && taken < posted) serve(taken++);
     };
-    long long w = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
-    w = __shfl_sync(0xffffffffu, w, 0);
-    while (ok) {
-      serve_pending();
-      if (w >= items) break;
-      const long long w_next = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
-      const int c = (int)(w / groups), g = (int)(w % groups);
-      const int b = g / p.Hkv, kvh = g % p.Hkv;
+    // An item looked up ahead of its emission (lane i: block i of the chunk).
+    struct Item {
+      long long w;
+      int c, g, kvh, npos, n, page, lastc;
+      uint32_t vm;
+      bool skip;
+    };
+    auto resolve = [&](long long wi) -> Item {
+      Item it;
+      it.w = wi;
+      it.c = it.g = it.kvh = it.npos = it.n = it.page = it.lastc = 0;
+      it.vm = 0;
+      it.skip = true;
+      if (wi >= items) return it;
+      it.c = (int)(wi / groups);
+      it.g = (int)(wi % groups);
+      const int b = it.g / p.Hkv;
+      it.kvh = it.g % p.Hkv;
       int L = p.seq_lens[b];
       if (L < 0 || L > p.max_seq_len) {
-        if (c == 0 && kvh == 0 && lane == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
+        if (it.c == 0 && it.kvh == 0 && lane == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
         L = 0;
       }
       const int nb = (L + kBlock - 1) / kBlock;
       const int N = art_positions(p, L);
-      bool skip = c * CB >= N;
-      if (!skip) {
+      if (it.c * CB >= N) return it;
+      const int sc = *reinterpret_cast<volatile int*>(ctl.stop_chunk + it.g);
+      if (__shfl_sync(0xffffffffu, sc != 0 && it.c >= sc, 0)) return it;  // every head stopped earlier
+      it.skip = false;
+      const int* ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)it.g * p.order_len : nullptr;
+      const int* bt = p.block_table + (size_t)b * p.max_blocks;
+      const int pos0 = it.c * CB;
+      it.npos = min(CB, N - pos0);
+      it.lastc = pos0 + CB >= N ? kLastChunkTag : 0;
+      int blk = -1;
+      if (lane < it.npos) {
+        blk = art_block(p, ord, nb, pos0 + lane, p.status);
+        if (blk >= 0) {
+          it.page = bt[blk];
+          if (it.page < 0 || it.page >= p.num_pages) {
+            dev_error(p.status, SKV_DEV_BAD_PAGE);
+            blk = -1;
+          } else {
+            it.n = min(kBlock, L - blk * kBlock);
+          }
+        }
+      }
+      it.vm = __ballot_sync(0xffffffffu, blk >= 0);
+      return it;
+    };
+    // 1: the group stopped at or before chunk c
+    auto stopped_at = [&](int g, int c) -> bool {
+      int s = 0;
+      if (lane == 0) {
         const int sc = *reinterpret_cast<volatile int*>(ctl.stop_chunk + g);
-        skip = sc != 0 && c >= sc;  // every head stopped in an earlier chunk
-        skip = __shfl_sync(0xffffffffu, skip, 0);
+        s = sc != 0 && c >= sc;
       }
-      if (!skip) {
-        const int* ord = (p.mode == TRAV_ORDER) ? p.order + (size_t)g * p.order_len : nullptr;
-        const int* bt = p.block_table + (size_t)b * p.max_blocks;
-        const int pos0 = c * CB, npos = min(CB, N - pos0);
-        int blk = -1, n = 0, page = 0;
-        if (lane < npos) {
-          blk = art_block(p, ord, nb, pos0 + lane, p.status);
-          if (blk >= 0) {
-            page = bt[blk];
-            if (page < 0 || page >= p.num_pages) {
-              dev_error(p.status, SKV_DEV_BAD_PAGE);
-              blk = -1;
+      return __shfl_sync(0xffffffffu, s, 0) != 0;
+    };
+    long long w = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
+    Item cur = resolve(__shfl_sync(0xffffffffu, w, 0));
+    while (ok) {
+      serve_pending();
+      if (cur.w >= items) break;
+      // the next item is taken now and looked up while this chunk's first
+      // tiles are in the ring, so the ring does not drain between chunks
+      const long long w_next = (lane == 0) ? (long long)atomicAdd(ctl.counter, 1) : 0;
+      bool have_next = false;
+      Item nxt;
+      auto prefetch = [&]() {
+        if (!have_next) nxt = resolve(__shfl_sync(0xffffffffu, w_next, 0));
+        have_next = true;
+      };
+      if (!cur.skip && cur.c > p.art_ahead) {
+        // Speculation gate: start the chunk only once chunk c - ahead - 1 of the
+        // group has been judged.  The awaited chunk has a smaller item number,
+        // so the wait always ends.
+        const int* rdy = ctl.ready + (size_t)cur.g * p.art_maxc + (cur.c - p.art_ahead - 1);
+        const uint64_t t0 = globaltimer();
+        while (true) {
+          int st = 0;  // 0: wait, 1: go, 2: the group stopped, 3: abort
+          if (lane == 0) {
+            if (*reinterpret_cast<const volatile int*>(rdy) != 0) {
+              st = 1;
             } else {
-              n = min(kBlock, L - blk * kBlock);
+              const int sc = *reinterpret_cast<const volatile int*>(ctl.stop_chunk + cur.g);
+              if (sc != 0 && cur.c >= sc) st = 2;
+              else if (flags[1] != 0 || globaltimer() - t0 > kWaitLimitNs) st = 3;
             }
           }
+          st = __shfl_sync(0xffffffffu, st, 0);
+          if (st == 1) break;
+          if (st == 2) {
+            cur.skip = true;
+            break;
+          }
+          if (st == 3) {
+            if (lane == 0) fail();
+            ok = false;
+            break;
+          }
+          serve_pending();
+          __nanosleep(128);
         }
-        const uint32_t vm = __ballot_sync(0xffffffffu, blk >= 0);
-        const uint16_t* qsrc = p.q + ((size_t)b * p.Hq + (size_t)kvh * G) * kHeadDim;
-        for (int i = 0; i < npos && ok; ++i) {
-          if (!((vm >> i) & 1u)) continue;
-          if ((i & 7) == 7) {  // the group may have stopped meanwhile: cut the chunk short
-            int stopped = 0;
-            if (lane == 0) {
-              const int sc = *reinterpret_cast<volatile int*>(ctl.stop_chunk + g);
-              stopped = sc != 0 && c >= sc;
-            }
-            if (__shfl_sync(0xffffffffu, stopped, 0)) break;
+        if (!ok) break;
+      }
+      if (!cur.skip && stopped_at(cur.g, cur.c)) cur.skip = true;  // stopped since the look-up
+      if (!cur.skip) {
+        const int b = cur.g / p.Hkv;
+        const uint16_t* qsrc = p.q + ((size_t)b * p.Hq + (size_t)cur.kvh * G) * kHeadDim;
+        const int last = cur.vm ? 31 - __clz(cur.vm) : -1;
+        bool cut = false;
+        for (int i = 0; i < cur.npos && ok; ++i) {
+          if (!((cur.vm >> i) & 1u)) continue;
+          if ((i & 7) == 7 && stopped_at(cur.g, cur.c)) {  // cut the chunk short
+            cut = true;
+            break;
           }
-          const int ni = __shfl_sync(0xffffffffu, n, i), pgi = __shfl_sync(0xffffffffu, page, i);
+          const int ni = __shfl_sync(0xffffffffu, cur.n, i), pgi = __shfl_sync(0xffffffffu, cur.page, i);
           int r = 1;
-          if (lane == 0) r = emit(ni, g, c, i, pgi, kvh, (vm & ((1u << i) - 1u)) ? nullptr : qsrc);
+          if (lane == 0)
+            r = emit(ni, cur.g, cur.c, i | (i == last ? kLastTag | cur.lastc : 0), pgi, cur.kvh,
+                     (cur.vm & ((1u << i) - 1u)) ? nullptr : qsrc);
           ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+          prefetch();
         }
-        if (ok) {
+        if (ok && (cut || last < 0)) {  // no tile carried the end of the chunk
           int r = 1;
-          if (lane == 0) r = emit(0, g, c, npos, 0, 0, nullptr);  // end of chunk
+          if (lane == 0) r = emit(0, cur.g, cur.c, cur.npos | cur.lastc, 0, 0, nullptr);
           ok = __shfl_sync(0xffffffffu, r, 0) != 0;
         }
       }
-      w = __shfl_sync(0xffffffffu, w_next, 0);
+      prefetch();
+      cur = nxt;
     }
     // no more items: the consumers hand the judge a QUIT post; once the judge has
     // handled every chunk, serve the last requests, then end the ring
@@ -465,14 +546,11 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     // inclusive prefix; returns the heads that stop in the chunk, their stop
     // blocks in st_out (-1: none).  SEG lanes per head (lane t: block t), so
     // 32 / SEG heads per pass.
-    auto evaluate = [&](const float* loc, int g, int c, uint32_t vmask, int* st_out) -> uint32_t {
+    auto evaluate = [&](const float* loc, int g, int c, uint32_t vmask, bool last_chunk,
+                        int* st_out) -> uint32_t {
       constexpr int SEG = CB <= 8 ? 8 : (CB <= 16 ? 16 : 32);
       constexpr int HPP = 32 / SEG;
       const size_t item = (size_t)g * p.art_maxc + c;
-      const int b = g / p.Hkv;
-      int L = p.seq_lens[b];
-      if (L < 0 || L > p.max_seq_len) L = 0;
-      const int nch = (art_positions(p, L) + CB - 1) / CB;
 #pragma unroll
       for (int h = 0; h < G; ++h) st_out[h] = -1;
       // (1) the previous chunk's prefix: ready, or the group already stopped
@@ -608,7 +686,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
             } else {
               R2.w = __int_as_float(total);
             }
-            if (t == wl && c == nch - 1) ctl.consumed[(size_t)g * G + h] = total;
+            if (t == wl && last_chunk) ctl.consumed[(size_t)g * G + h] = total;
           }
         }
         if (hv && t == wl) {
@@ -650,15 +728,15 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         if (lane == 0) fail();
         break;
       }
-      const int kind = tag[par * 4], tg_g = tag[par * 4 + 1], tg_c = tag[par * 4 + 2],
+      const int kind = tag[par * 4] & 0xFF, tg_g = tag[par * 4 + 1], tg_c = tag[par * 4 + 2],
                 tg_a = tag[par * 4 + 3];
+      const bool last_chunk = (tag[par * 4] >> 16) & 1;
       const float* st_area = state + (size_t)par * NW * G * kRecFloats;
       if (kind == POST_END) {
         merge_probes(probe + (size_t)par * probe_floats<G, NW, CB>(), (uint32_t)tg_a);
-        reduce_states(st_area, tg_g, tg_c, (1u << G) - 1u);
         __syncwarp();  // the chunk-local prefixes are visible to every lane
         int st[G];
-        const uint32_t stopmask = evaluate(local, tg_g, tg_c, (uint32_t)tg_a, st);
+        const uint32_t stopmask = evaluate(local, tg_g, tg_c, (uint32_t)tg_a, last_chunk, st);
         if (stopmask) {
           if (n_req - n_fix >= kReqs) {
             if (lane == 0) fail();  // cannot happen: the consumers serve requests every chunk
@@ -677,6 +755,8 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
             ++n_req;
           }
         }
+        // the chunk's records (after the decision: they are not on its path)
+        reduce_states(st_area, tg_g, tg_c, (1u << G) - 1u);
       } else if (kind == POST_FIX) {
         reduce_states(st_area, tg_g, tg_c, (uint32_t)tg_a);
         ++n_fix;
@@ -795,7 +875,8 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     if (n == 0) {  // end of the item
       release();
       write_state();
-      publish(fix ? POST_FIX : POST_END, mt.y, mt.z, fix ? req[slot * 4 + 3] : (int)vmask);
+      publish(fix ? POST_FIX : (POST_END | ((mt.w & kLastChunkTag) ? 1 << 16 : 0)), mt.y, mt.z,
+              fix ? req[slot * 4 + 3] : (int)vmask);
       continue;
     }
     const unsigned char* sK = smem + s * C::STAGE_BYTES;
@@ -823,6 +904,10 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
           unpack2(W.acc[g2][1], x2, x3);
           *reinterpret_cast<float4*>(pw + g2 * kProbeFloats + 4 + lane * 4) = make_float4(x0, x1, x2, x3);
         }
+      }
+      if (mt.w & kLastTag) {  // the chunk's last tile: post the chunk
+        write_state();
+        publish(POST_END | ((mt.w & kLastChunkTag) ? 1 << 16 : 0), mt.y, mt.z, (int)vmask);
       }
     } else {
       // a stopping head takes no block after its stop block
