@@ -391,12 +391,15 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         const uint16_t* qsrc = p.q + ((size_t)b * p.Hq + (size_t)cur.kvh * G) * kHeadDim;
         const int last = cur.vm ? 31 - __clz(cur.vm) : -1;
         bool cut = false;
+        int sc_ahead = 0;  // lane 0: the group's stop chunk, loaded a tile before it is checked
         for (int i = 0; i < cur.npos && ok; ++i) {
           if (!((cur.vm >> i) & 1u)) continue;
-          if ((i & 7) == 7 && stopped_at(cur.g, cur.c)) {  // cut the chunk short
+          if ((i & 7) == 7 &&
+              __shfl_sync(0xffffffffu, sc_ahead != 0 && cur.c >= sc_ahead, 0)) {  // cut the chunk short
             cut = true;
             break;
           }
+          if ((i & 7) == 6 && lane == 0) sc_ahead = *reinterpret_cast<volatile int*>(ctl.stop_chunk + cur.g);
           const int ni = __shfl_sync(0xffffffffu, cur.n, i), pgi = __shfl_sync(0xffffffffu, cur.page, i);
           int r = 1;
           if (lane == 0)
