@@ -253,7 +253,7 @@ def build_decode(torch, skv, skvgen, wl, status, art=None, inputs=None):
         if st != 0:
             raise skv.SkvError(st, "attn_decode")
 
-    step = Step(run, wl.kv_bytes(), 2 if n else 1)  # decode or ART kernel, then the record merge
+    step = Step(run, wl.kv_bytes(), L.skv_decode_launches(ctypes.byref(a)))
     # keep every tensor the raw pointers in `a` refer to alive with the step
     step.tensors = dict(q=q, k_pool=k_pool, v_pool=v_pool, bt=bt, sl=sl, out=out, lse=lse,
                         consumed=consumed, ws=ws, kw=kw, common=common)
@@ -293,7 +293,7 @@ def build_select(torch, skv, skvgen, wl, status):
     torch.cuda.synchronize()
     sel_tokens = int((se - ss).sum().item())
     nbytes = sel_tokens * wl.d * 4 + cent.numel() * 2 + off.numel() * 4
-    step = Step(run, nbytes, 3, {"selected_tokens": sel_tokens,
+    step = Step(run, nbytes, 1 + L.skv_decode_launches(ctypes.byref(a)), {"selected_tokens": sel_tokens,
                                  "selected_frac": sel_tokens / (wl.B * wl.Hkv * wl.L),
                                  "centroid_bytes": cent.numel() * 2})
     # keep every tensor the raw pointers above refer to alive with the step
@@ -324,7 +324,7 @@ def build_routed(torch, skv, skvgen, wl, status):
         ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda") if n else None
         a = skv.make_decode_args(q, k_pool, v_pool, bt, sl, out, lse, workspace=ws, **kw)
         layers.append(dict(fa=fa, a=a, keep=(q, k_pool, v_pool, bt, sl, out, lse, consumed, ws),
-                           consumed=consumed, launches=2 if n else 1))
+                           consumed=consumed, launches=skv.lib().skv_decode_launches(ctypes.byref(a))))
     L = skv.lib()
 
     def run():

@@ -156,6 +156,13 @@ typedef struct {
  * partials); 0 if none.  Depends only on host-side fields. */
 SKV_API size_t skv_decode_workspace_size(const skv_decode_args* args);
 
+/* Kernels one attn_decode call launches for these arguments (1: the walk
+ * merges its own partials -- a query chunk, or the split schedule that small
+ * walks and segment lists take; 2: the walk, then the record merge), not
+ * counting the workspace zeroing (a device memset); 0 if the arguments are
+ * invalid.  Depends only on host-side fields; for profiling and accounting. */
+SKV_API int skv_decode_launches(const skv_decode_args* args);
+
 /* Decode attention, see above.  Option combinations: at most one of
  * {order, window, seg_start/seg_end, kv range}; ART only with natural or
  * `order` traversal. */

@@ -65,6 +65,8 @@ def lib():
         L = ctypes.CDLL(_build.SO)
         L.skv_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]
         L.skv_decode_workspace_size.restype = ctypes.c_size_t
+        L.skv_decode_launches.argtypes = [ctypes.POINTER(DecodeArgs)]
+        L.skv_decode_launches.restype = ctypes.c_int
         L.attn_decode.argtypes = [ctypes.POINTER(DecodeArgs), _p]
         L.attn_decode.restype = _i
         L.attn_decode_static_ws.argtypes = [ctypes.POINTER(DecodeArgs), _p]
@@ -140,6 +142,12 @@ def make_decode_args(q, k_pool, v_pool, block_table, seq_lens, out, lse, *, max_
 def decode_workspace_size(*args, **kw):
     """Bytes of workspace attn_decode needs (same arguments as attn_decode)."""
     return lib().skv_decode_workspace_size(ctypes.byref(make_decode_args(*args, **kw)))
+
+
+def decode_launches(*args, **kw):
+    """Kernels one attn_decode call launches for these arguments (see
+    skv_decode_launches in include/sparsekv.h)."""
+    return lib().skv_decode_launches(ctypes.byref(make_decode_args(*args, **kw)))
 
 
 def attn_decode(*args, stream=None, **kw):

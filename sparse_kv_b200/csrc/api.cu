@@ -39,10 +39,10 @@ inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 // Split count for traversals of up to n_tiles tiles per group: minimise
 // (waves x tiles per CTA) plus a per-wave fill cost, given the resident CTAs per SM.
-int choose_splits(long long groups, long long n_tiles, int ctas_per_sm) {
+int choose_splits(long long groups, long long n_tiles, int ctas_per_sm, int max_splits) {
   if (n_tiles <= 1 || groups <= 0) return 1;
   const int sms = num_sms() * ctas_per_sm;
-  const int s_max = (int)std::max<long long>(1, std::min<long long>(64, n_tiles / 4));
+  const int s_max = (int)std::max<long long>(1, std::min<long long>(max_splits, n_tiles / 4));
   int best = 1;
   long long best_cost = -1;
   for (int s = 1; s <= s_max; ++s) {
@@ -130,29 +130,34 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     return SKV_OK;
   }
   pl->nw = decode_consumer_warps(G);
-  long long slots = 0;
-  if (pl->mode != TRAV_SEGMENTS && a->batch <= kMaxPersistentBatch) {
-    DecodeParams probe{};
-    probe.mode = pl->mode;
-    probe.range_begin = a->kv_begin;
-    probe.range_end = a->kv_end;
-    probe.sink = a->window.sink_tokens;
-    probe.recent = a->window.recent_tokens;
-    probe.order_len = a->order_len;
-    const long long t_est = groups * group_tiles(probe, a->max_seq_len);
-    if (t_est >= (1ll << 31)) return SKV_EUNSUPPORTED;
+  DecodeParams probe{};
+  probe.mode = pl->mode;
+  probe.range_begin = a->kv_begin;
+  probe.range_end = a->kv_end;
+  probe.sink = a->window.sink_tokens;
+  probe.recent = a->window.recent_tokens;
+  probe.order_len = a->order_len;
+  const long long t_est =
+      pl->mode == TRAV_SEGMENTS ? 0 : groups * group_tiles(probe, a->max_seq_len);
+  if (t_est >= (1ll << 31)) return SKV_EUNSUPPORTED;
+  // Small walks (a few tiles per resident CTA) are latency-bound: there the
+  // split schedule, which merges inside the kernel, saves the second launch.
+  const long long small = (long long)num_sms() * decode_ctas_per_sm(G) * 8;
+  if (pl->mode != TRAV_SEGMENTS && a->batch <= kMaxPersistentBatch && t_est > small) {
     pl->sched = SCHED_PERSISTENT;
     const long long max_ctas = (long long)num_sms() * decode_ctas_per_sm(G);
     pl->n_ctas = (int)std::max<long long>(1, std::min<long long>(max_ctas, cdiv(t_est, 4)));
-    slots = pl->n_ctas + groups;
+    const long long slots = pl->n_ctas + groups;
     pl->hdr_bytes = (size_t)cdiv((a->batch + 2) * 4ll, 256) * 256;
+    pl->ws_bytes = pl->hdr_bytes + (size_t)slots * pl->nw * G * kRecFloats * sizeof(float);
   } else {
+    // one cluster of `splits` CTAs per group, merged in distributed shared
+    // memory: no workspace
     pl->sched = SCHED_SPLIT;
     pl->splits = choose_splits(groups, pl->mode == TRAV_SEGMENTS ? a->n_seg : cdiv(a->max_seq_len, kBlock),
-                               decode_ctas_per_sm(G));
-    slots = groups * pl->splits;
+                               decode_ctas_per_sm(G), kMaxClusterSplits);
+    pl->ws_bytes = 0;
   }
-  pl->ws_bytes = pl->hdr_bytes + (size_t)slots * pl->nw * G * kRecFloats * sizeof(float);
   return SKV_OK;
 }
 
@@ -167,6 +172,12 @@ size_t skv_decode_workspace_size(const skv_decode_args* args) {
   Plan pl;
   if (make_plan(args, &pl) != SKV_OK) return 0;
   return pl.ws_bytes;
+}
+
+int skv_decode_launches(const skv_decode_args* args) {
+  Plan pl;
+  if (make_plan(args, &pl) != SKV_OK) return 0;
+  return (pl.chunk || (!pl.art && pl.sched == SCHED_SPLIT)) ? 1 : 2;
 }
 
 skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
@@ -231,6 +242,7 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
     p.ws_hdr = reinterpret_cast<int*>(ws);
     p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes);
     if (launch_decode(p, pl.G, s) != 0) return SKV_ECUDA;
+    if (pl.sched == SCHED_SPLIT) return SKV_OK;  // merged inside the kernel
   }
   if (launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
   return SKV_OK;

@@ -193,6 +193,47 @@ struct Trav {
   }
 };
 
+// ---- thread-block cluster helpers (the split schedule: a cluster = the pieces of one group)
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier of another CTA of the cluster (release: this thread's
+// and, after the fence, its CTA's earlier shared-memory writes are visible).
+__device__ __forceinline__ void cluster_arrive_remote(uint32_t bar_cluster_addr) {
+  asm volatile("fence.acq_rel.cluster;\n\tmbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+               ::"r"(bar_cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (acquire at cluster scope): gives up after `limit_ns`.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 template <int G, int NW, int MINB>
 struct Cfg {
   using Ln = Lanes<G, NW>;
@@ -200,7 +241,7 @@ struct Cfg {
   static constexpr int STAGES = MINB == 2 ? 3 : 6;
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes;
-  static constexpr int NBAR = 2 * STAGES + 1;  // full, empty, fin
+  static constexpr int NBAR = 2 * STAGES + 6;  // full, empty, fin, fin2, fin3, fin4, gather, release
   static constexpr size_t OFF_BAR = STAGES * STAGE_BYTES;
   static constexpr size_t OFF_META = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;   // int4 [STAGES]
   static constexpr size_t OFF_FLAGS = (OFF_META + STAGES * 16 + 15) / 16 * 16;
@@ -224,7 +265,13 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + ST;
-  uint64_t* fin_bar = empty + ST;  // NW arrivals
+  uint64_t* fin_bar = empty + ST;  // NW arrivals: the consumers are done with the ring
+  // split schedule only:
+  uint64_t* fin2_bar = fin_bar + 1;     // NW arrivals: the warps' states are in the ring
+  uint64_t* fin3_bar = fin2_bar + 1;    // NW arrivals: the piece's records are written
+  uint64_t* fin4_bar = fin3_bar + 1;    // G arrivals: (rank 0) the merge is done
+  uint64_t* gather_bar = fin4_bar + 1;  // (rank 0) S arrivals, one per piece of the cluster
+  uint64_t* release_bar = gather_bar + 1;  // (ranks > 0) rank 0 has read this CTA's records
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows, group, slot, 0}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   // flags[1]: abort (a bounded wait expired)
@@ -237,10 +284,20 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       mbar_init(&empty[s], NW);
     }
     mbar_init(fin_bar, NW);
+    mbar_init(fin2_bar, NW);
+    mbar_init(fin3_bar, NW);
+    mbar_init(fin4_bar, G);
+    mbar_init(gather_bar, p.sched == SCHED_SPLIT ? p.n_splits : 1);
+    mbar_init(release_bar, 1);
     flags[0] = flags[1] = flags[2] = 0;
     fence_barrier_init();
   }
   __syncthreads();
+  // Split schedule: every thread marks the cluster barrier once its CTA's
+  // mbarriers are initialised (release); a wait on it before the first access
+  // to another CTA's shared memory then ends as soon as every CTA of the
+  // cluster is running with its barriers ready.
+  if (p.sched == SCHED_SPLIT) asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
   // ------------------------------------------------------------------ producer
   if (warp == NW) {
     int* pre = reinterpret_cast<int*>(smem + C::OFF_PRE);  // [B+1] tiles before batch b
@@ -482,6 +539,7 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
   uint32_t ph = 0;        // phase of the current ring round
   int k = 0;              // tiles folded for the current group piece
   int cur_g = -1, cur_slot = 0;
+  bool saw_end = false;  // the end entry was reached: every copy into the ring has landed
   W.reset();
   while (true) {
     if (!mbar_wait_bounded(&full[s], ph, &flags[1])) {
@@ -493,7 +551,10 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     }
     const int4 mt = meta[s];
     const int n = mt.x;
-    if (n < 0) break;  // end of traversal
+    if (n < 0) {  // end of traversal
+      saw_end = true;
+      break;
+    }
     if (mt.y != cur_g) {
       if (cur_g >= 0) flush(cur_slot, k);
       W.reset();
@@ -520,13 +581,172 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
   }
 
   // ------------------------------------------------------------------ epilogue
-  if (cur_g >= 0) flush(cur_slot, k);
-  // Every consumer warp ends here: let the producer know once all are done.
+  if (p.sched == SCHED_PERSISTENT) {
+    if (cur_g >= 0) flush(cur_slot, k);
+    // Every consumer warp ends here: let the producer know once all are done.
+    __syncwarp();
+    mbar_arrive_if(fin_bar, lane == 0);
+    if (warp == 0) {
+      if (!mbar_wait_bounded(fin_bar, 0, nullptr) && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+      if (lane == 0) flags[2] = (flags[1] != 0) ? 1 : e + 1;
+    }
+    return;
+  }
+  // Split schedule: the CTAs of a cluster are the S pieces of one group, and
+  // the merge happens here, over distributed shared memory.  Once every
+  // consumer warp is done with the ring (no copy is in flight after the end
+  // entry), the warps leave their states in it and warps 0..G-1 combine one
+  // head each into this piece's record (also in shared memory).  Every CTA then
+  // arrives on rank 0's gather barrier; rank 0 reads the S records of each head
+  // from the cluster's shared memory, writes the output row and releases the
+  // other CTAs, which stay resident until then.  Every wait is bounded; a CTA
+  // whose walk failed sends an empty record (the status word has the error).
   __syncwarp();
   mbar_arrive_if(fin_bar, lane == 0);
-  if (warp == 0) {
-    if (!mbar_wait_bounded(fin_bar, 0, nullptr) && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
-    if (lane == 0) flags[2] = (flags[1] != 0) ? 1 : e + 1;
+  const bool fin_ok = mbar_wait_bounded(fin_bar, 0, nullptr);
+  if (warp == 0 && lane == 0) {
+    if (!fin_ok) dev_error(p.status, SKV_DEV_TIMEOUT);
+    flags[2] = (flags[1] != 0) ? 1 : e + 1;
+  }
+  // after an abort a warp may have left the loop early (and copies may still land)
+  const bool good = fin_ok && flags[1] == 0 && saw_end;
+  float* st_sm = reinterpret_cast<float*>(smem);   // [NW][G][kRecFloats]: O, m, l, tiles
+  float* pc_sm = st_sm + NW * G * kRecFloats;       // [G][kRecFloats]: this piece's records
+  static_assert((size_t)(NW + 1) * G * kRecFloats * 4 <= ST * C::STAGE_BYTES, "states fit in the ring");
+  if (good) {
+#pragma unroll
+    for (int g2 = 0; g2 < G; ++g2) {
+      float x0, x1, x2, x3;
+      unpack2(W.acc[g2][0], x0, x1);
+      unpack2(W.acc[g2][1], x2, x3);
+      *reinterpret_cast<float4*>(st_sm + (warp * G + g2) * kRecFloats + lane * 4) =
+          make_float4(x0, x1, x2, x3);
+    }
+    if (W.owner) {
+#pragma unroll
+      for (int j = 0; j < Lanes<G, NW>::VPL; ++j)
+        *reinterpret_cast<float4*>(st_sm + (warp * G + W.hd[j]) * kRecFloats + 128) =
+            make_float4(W.m_st[j], W.l_st[j], (float)k, 0.f);
+    }
+  }
+  __syncwarp();
+  mbar_arrive_if(fin2_bar, lane == 0);
+  const bool ok2 = mbar_wait_bounded(fin2_bar, 0, nullptr);
+  if (warp < G) {  // this piece's record of head `warp`
+    const int h = warp;
+    float M = -INFINITY, L = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (good && ok2) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float2 ml = *reinterpret_cast<const float2*>(st_sm + (w * G + h) * kRecFloats + 128);
+        if (ml.y > 0.f) M = fmaxf(M, ml.x);
+      }
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const float* s = st_sm + (w * G + h) * kRecFloats;
+          const float2 ml = *reinterpret_cast<const float2*>(s + 128);
+          const float f = (ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
+          const float4 x = *reinterpret_cast<const float4*>(s + lane * 4);
+          L += ml.y * f;
+          o.x += x.x * f;
+          o.y += x.y * f;
+          o.z += x.z * f;
+          o.w += x.w * f;
+        }
+      }
+    }
+    *reinterpret_cast<float4*>(pc_sm + h * kRecFloats + lane * 4) = o;
+    if (lane == 0)
+      *reinterpret_cast<float4*>(pc_sm + h * kRecFloats + 128) =
+          make_float4(M, L, (good && ok2) ? (float)k : 0.f, 0.f);
+  }
+  __syncwarp();
+  mbar_arrive_if(fin3_bar, lane == 0);
+  const bool ok3 = mbar_wait_bounded(fin3_bar, 0, nullptr);
+  if (!ok2 || !ok3) {
+    if (lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+  }
+  const uint32_t rank = blockIdx.x;  // cluster (S, 1, 1) over grid.x = S
+  const int S = p.n_splits;
+  if (warp == 0) {  // this piece is ready: tell rank 0
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if (lane == 0) cluster_arrive_remote(cluster_addr(gather_bar, 0));
+  }
+  if (rank == 0) {
+    if (warp < G) {
+      if (warp != 0) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+      const int h = warp;
+      // (longer than any CTA's own bounded waits: a piece arrives once its walk ends)
+      const bool got = mbar_wait_cluster(gather_bar, 0, 4 * kWaitLimitNs);
+      if (!got && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+      if (got) {
+        // lane s holds piece s's scalars (S <= 32)
+        float ms = -INFINITY, ls = 0.f;
+        int ts = 0;
+        if (lane < S) {
+          const float4 v = ld_cluster_f4(cluster_addr(pc_sm + h * kRecFloats + 128, lane));
+          if (v.y > 0.f) {
+            ms = v.x;
+            ls = v.y;
+          }
+          ts = (int)v.z;
+        }
+        float M = ms;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+          ts += __shfl_xor_sync(0xffffffffu, ts, o);
+        }
+        const float fs = (ms != -INFINITY) ? exp2f(ms - M) : 0.f;
+        float Wl = fs * ls;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) Wl += __shfl_xor_sync(0xffffffffu, Wl, o);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const uint32_t own = smem_u32(pc_sm + h * kRecFloats + lane * 4);
+        for (int s0 = 0; s0 < S; s0 += 8) {
+          float4 x[8];
+          float f[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int s = s0 + q;
+            f[q] = __shfl_sync(0xffffffffu, fs, s & 31);
+            x[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s < S && f[q] > 0.f) {
+              uint32_t ra;
+              asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(own), "r"(s));
+              x[q] = ld_cluster_f4(ra);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            acc.x += f[q] * x[q].x;
+            acc.y += f[q] * x[q].y;
+            acc.z += f[q] * x[q].z;
+            acc.w += f[q] * x[q].w;
+          }
+        }
+        const size_t row = (size_t)blockIdx.z * p.Hq + (size_t)blockIdx.y * G + h;
+        const float inv = (Wl > 0.f) ? 1.f / Wl : 0.f;
+        *reinterpret_cast<float4*>(p.out + row * kHeadDim + lane * 4) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (lane == 0) {
+          p.lse[row] = (Wl > 0.f) ? (M + log2f(Wl)) * 0.6931471805599453f : -INFINITY;
+          if (p.blocks_consumed) p.blocks_consumed[row] = ts;
+        }
+      }
+      __syncwarp();
+      mbar_arrive_if(fin4_bar, lane == 0);
+      if (warp == 0) {  // every read of the other CTAs' records is done: release them
+        if (!mbar_wait_bounded(fin4_bar, 0, nullptr) && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+        __syncwarp();
+        if (lane >= 1 && lane < S) cluster_arrive_remote(cluster_addr(release_bar, lane));
+      }
+    }
+  } else if (warp == 0) {
+    // stay resident (shared memory valid) until rank 0 has read this piece
+    if (!mbar_wait_cluster(release_bar, 0, 8 * kWaitLimitNs) && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
   }
 }
 
@@ -555,11 +775,41 @@ int launch_t(const DecodeParams& p, cudaStream_t st) {
     if (err != cudaSuccess) return (int)err;
     attr_set[dev] = true;
   }
-  dim3 grid;
-  if (p.sched == SCHED_PERSISTENT) grid = dim3(p.n_ctas, 1, 1);
-  else grid = dim3(p.n_splits, p.Hkv, p.B);
-  kern<<<grid, C::THREADS, C::TOTAL, st>>>(p);
-  return (int)cudaGetLastError();
+  if (p.sched == SCHED_PERSISTENT) {
+    kern<<<dim3(p.n_ctas, 1, 1), C::THREADS, C::TOTAL, st>>>(p);
+    return (int)cudaGetLastError();
+  }
+  // split schedule: one cluster of n_splits CTAs per group (<= 16; above 8
+  // needs the non-portable size, allowed once per device)
+  if (p.n_splits < 1 || p.n_splits > kMaxClusterSplits) return (int)cudaErrorInvalidValue;
+  static bool np_set[64] = {};
+  if (!np_set[dev]) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return (int)err;
+    np_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_splits, p.Hkv, p.B);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::TOTAL;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.n_splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // refuse a cluster shape that cannot be resident at once (checked once per size)
+  static int fits[64][kMaxClusterSplits + 1] = {};
+  if (fits[dev][p.n_splits] == 0) {
+    int n = 0;
+    cudaError_t err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (err != cudaSuccess) return (int)err;
+    fits[dev][p.n_splits] = n > 0 ? 1 : -1;
+  }
+  if (fits[dev][p.n_splits] < 0) return (int)cudaErrorInvalidConfiguration;
+  return (int)cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 }  // namespace

@@ -15,11 +15,12 @@ enum TravMode : int {
 
 enum Schedule : int {
   SCHED_PERSISTENT = 0,  // one CTA per SM walks an even share of all tiles of all groups
-  SCHED_SPLIT = 1,       // grid (splits, kv_heads, batch), each CTA one piece of one group
+  SCHED_SPLIT = 1,       // grid (splits, kv_heads, batch), a cluster per group, merged in-kernel
   SCHED_ART = 2,         // persistent CTAs take (chunk, group) items (art.cu)
 };
 
 constexpr int kMaxPersistentBatch = 1024;  // batch prefix kept in shared memory
+constexpr int kMaxClusterSplits = 16;      // split schedule: CTAs per cluster (one group)
 constexpr int kRecFloats = 132;            // partial record: O[128], m (base 2), l, tiles, pad
 constexpr int kLbFloats = 12;              // ART look-back record per head: m, l, O[0:8], run, state
 

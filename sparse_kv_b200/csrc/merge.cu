@@ -76,8 +76,8 @@ int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int
 // Merge of the decode kernels' partial records.  Row (b, h) of group
 // g = b*Hkv + h/G collects the records of every piece of g: persistent
 // schedule -> slots c + g for the CTAs c whose tile share meets g's tiles
-// [T_g, T_g + n_g); split schedule -> slots g*S .. g*S + S-1; ART -> the
-// chunks of g up to the one where the row's head stopped.  Each record holds
+// [T_g, T_g + n_g); ART -> the chunks of g up to the one where the row's head
+// stopped.  (The split schedule merges inside decode_kernel.)  Each record holds
 // (O unnormalised, m in base 2, l, tiles); the merge is the same exact
 // online-softmax combination as above, in base 2.
 // ---------------------------------------------------------------------------
@@ -123,9 +123,6 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_records_kernel(const D
       s0 = (int)(((Tg + 1) * P - 1) / T) + g;
       s1 = (int)(((Tg + nt) * P - 1) / T) + g;
     }
-  } else {
-    s0 = g * p.n_splits;
-    s1 = s0 + p.n_splits - 1;
   }
   const int nrec = (s1 - s0 + 1) * NW;  // record r: slot s0 + r / NW, warp r % NW
   auto rec_ptr = [&](int r) {
@@ -232,9 +229,8 @@ int launch_merge_records(const DecodeParams& p, int G, void* stream) {
   const int N = p.B * p.Hq;
   if (N == 0) return 0;
   // records per row: pieces of one group (<= all persistent CTAs, or the splits) x warps
-  const int max_slots = (p.sched == SCHED_PERSISTENT) ? p.n_ctas
-                        : (p.sched == SCHED_ART)      ? p.art_maxc
-                                                      : p.n_splits;
+  if (p.sched != SCHED_PERSISTENT && p.sched != SCHED_ART) return (int)cudaErrorInvalidValue;
+  const int max_slots = (p.sched == SCHED_PERSISTENT) ? p.n_ctas : p.art_maxc;
   const size_t smem = (size_t)max_slots * p.rec_nw * sizeof(float);
   if (smem > 200 * 1024) return (int)cudaErrorInvalidConfiguration;
   static bool attr_set[64] = {};

@@ -96,18 +96,38 @@ def test_workspace_size_query():
     n = L.skv_decode_workspace_size(ctypes.byref(full))
     # header (batch prefix) + per-warp partial records of 132 floats per head
     assert n > 0 and (n % 256) == 0 and n >= 16 * 8 * 16 * 4 * 132 * 4
-    # ART: per (chunk of 32 blocks, KV group): a look-back record of 12 floats
-    # and a partial record of 132 floats per head, zeroed control words, and a
-    # scratch area of at most 192 KB per resident CTA (2 per SM)
+    # ART: per (chunk, KV group): a look-back record of 12 floats and a partial
+    # record of 132 floats per head, zeroed control words, and a scratch area of
+    # at most 192 KB per resident CTA (2 per SM).  This shape (128 groups of 512
+    # blocks, 296 CTAs: about 2.3 chunks of a group in flight) takes 16-block
+    # chunks, since 32-block ones would read 74 blocks past a stop, over 1/12
+    # of the walk.
     art = good_args(art=_Art(1, 1e-3, 1e-4, 4))
-    items = 16 * 8 * (512 // 32)
+    items = 16 * 8 * (512 // 16)
     na = L.skv_decode_workspace_size(ctypes.byref(art))
-    assert na >= items * 4 * (132 + 12) * 4 + (4 + 16 * 8 * (1 + 512 // 32 + 8)) * 4
+    assert na >= items * 4 * (132 + 12) * 4 + (4 + 16 * 8 * (1 + 512 // 16 + 8)) * 4
     assert na < items * 4 * (132 + 12) * 4 + 64 * 1024 + 2 * 148 * 192 * 1024
     assert status(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == skv.SKV_EWORKSPACE
     assert L.skv_decode_workspace_size(ctypes.byref(good_args(head_dim=64))) == 0
     small = good_args(workspace=FAKE, workspace_bytes=n - 16)
     assert status(small) == skv.SKV_EWORKSPACE
+
+
+def test_decode_launch_count():
+    # one kernel where the walk merges its own partials (small walks and
+    # segment lists take the split schedule; a query chunk writes its results
+    # directly), two where a record merge follows (large walks, ART)
+    L = skv.lib()
+    n = lambda a: L.skv_decode_launches(ctypes.byref(a))
+    assert n(good_args()) == 2                                    # 128 groups x 512 tiles
+    assert n(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == 2
+    small = good_args(batch=1, q_heads=8, kv_heads=2, max_seq_len=4096, max_blocks=64)
+    assert n(small) == 1                                          # 2 groups x 64 tiles
+    # the split schedule merges its pieces in the cluster's shared memory: no workspace
+    assert L.skv_decode_workspace_size(ctypes.byref(small)) == 0
+    assert n(good_args(seg_start=FAKE, seg_end=FAKE, n_seg=102)) == 1
+    assert n(good_args(q_tokens=128)) == 1
+    assert n(good_args(head_dim=64)) == 0
 
 
 def test_select_and_merge_reject_on_host():

@@ -77,6 +77,42 @@ def test_cfg1_full_traversal():
     assert np.all(res[2] == 64)
 
 
+def test_split_merge_repeats():
+    # The split schedule (small walks) merges inside the kernel: the pieces of a
+    # group form one cluster, and rank 0 combines them from the cluster's
+    # shared memory.  Three calls must give the oracle's result, bit-identical.
+    import sparse_kv_b200 as skv
+    torch = _torch()
+    lens = [4096, 64 * 7 + 3, 0]
+    wl = skvgen.Workload("w", B=3, Hq=8, Hkv=2, L=max(lens), lens=lens, paging="perm", seed=71)
+    dev = device_workload(wl)
+    out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
+    consumed = torch.full((wl.B, wl.Hq), -1, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    args = (dev["q"], dev["k_pool"], dev["v_pool"], dev["block_table"], dev["seq_lens"], out, lse)
+    kw = dict(max_seq_len=wl.Lmax, blocks_consumed=consumed, status=status, scale=wl.scale)
+    assert skv.decode_launches(*args, **kw) == 1
+    assert skv.decode_workspace_size(*args, **kw) == 0
+    first = None
+    for it in range(3):
+        out.fill_(float("nan"))
+        lse.fill_(float("nan"))
+        skv.attn_decode(*args, **kw)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        res = (out[:, 0].cpu().numpy().astype(np.float64), lse[:, 0].cpu().numpy().astype(np.float64),
+               consumed.cpu().numpy(), 0)
+        if first is None:
+            _check_all_groups(wl, res, lambda b: oracle.keys_full(wl.seq_len(b)))
+            first = res
+        else:
+            np.testing.assert_array_equal(res[0], first[0])
+            np.testing.assert_array_equal(res[1], first[1])
+        nb = np.array([wl.nb(b) for b in range(wl.B)])
+        np.testing.assert_array_equal(res[2], np.repeat(nb[:, None], wl.Hq, axis=1))
+
+
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_ragged_paged_full_traversal(G):
     lens = [1, 63, 64, 65, 200, 1000, 0, 4097]
