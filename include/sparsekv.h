@@ -95,8 +95,10 @@ typedef enum {
  * if ||x_t|| = 0 else +inf; a zero vector gives d_dir = 0 if both are zero,
  * else 1.  tau = phi = 0 never stops (full attention).  Block 0 is always
  * consumed first.  Key loads of a KV group stop once all of its query heads
- * have stopped; up to (pipeline depth - 1) further blocks may already be in
- * flight and are discarded. */
+ * have stopped.  The test is decided per chunk of 16 or 32 blocks, and
+ * chunks of the group that started before the stop was decided are read and
+ * discarded (cut short every 8 blocks); blocks_consumed counts only the
+ * blocks each head attended. */
 typedef struct {
   int enable;   /* 0 = off */
   float tau;    /* >= 0, scale-change threshold */
