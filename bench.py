@@ -395,6 +395,23 @@ def build_chunk(torch, skv, skvgen, wl, status):
 np = None
 
 
+def max_over_ranks(x, world, dist, device):
+    """The largest of every rank's `x` (a device time in ms): the job takes as
+    long as its slowest replica.  `x` itself on one rank."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(nbytes_per_rank, world, ms):
+    """Whole-job throughput in GB/s: every replica moves `nbytes_per_rank`
+    per step, and a step takes `ms` (the max over ranks)."""
+    return nbytes_per_rank * world / (ms * 1e-3) / 1e9
+
+
 def main():
     global np
     args = parse()
@@ -472,10 +489,7 @@ def main():
         torch.cuda.synchronize()
         total_ms = t0.elapsed_time(t1)
         per = [e0.elapsed_time(e1) for e0, e1 in evs]
-        if world > 1:
-            t = torch.tensor([total_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, world, dist, "cuda")
         del g
         return total_ms, per
 
@@ -494,7 +508,7 @@ def main():
         raise RuntimeError(f"device status word {int(status.item()):#x}")
 
     ms_step = total_ms / args.steps
-    value = step.nbytes * world / (ms_step * 1e-3) / 1e9
+    value = job_gbs(step.nbytes, world, ms_step)
     per_launch_ms = statistics.mean(per)
     achieved = step.nbytes / (per_launch_ms * 1e-3) / 1e9
 
@@ -527,13 +541,10 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, world, dist, "cuda")
         h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
         d2h = out_h.numel() * 4 + lse_h.numel() * 4
-        e2e = {"value": step.nbytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_gbs(step.nbytes, world, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "KV cache resident in HBM; per step q, block table and seq_lens copied in "
                        "from pinned host memory and O, LSE copied out"}
