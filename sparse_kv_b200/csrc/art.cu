@@ -23,29 +23,30 @@
 //   consumers  NW warps fold every block into their online-softmax states
 //              (tile.cuh) and leave (m, l, O[0:8]) of their state after every
 //              block in a per-CTA scratch area; at the end of a chunk each
-//              warp writes its whole state and posts the chunk to the judge.
+//              warp writes its whole state and posts the chunk to the arbiter.
 //              They never meet and never wait for a decision;
-//   judge      one warp combines the warps' probes into the chunk-local prefix
+//   arbiter    one warp combines the warps' probes into the chunk-local prefix
 //              after every block (lane = (block, head)), waits for the
 //              previous chunk's published prefix (m, l, O[0:8], run of passing
 //              tests, blocks consumed or the stop) -- a decoupled look-back,
-//              as in single-pass parallel prefix scans -- evaluates the test for all CB blocks at once
-//              (lane t: block t; the patience run by warp ballots) and
-//              publishes the inclusive prefix; only then does it reduce the
-//              warps' states into the chunk's record, which no decision needs.
+//              as in single-pass parallel prefix scans -- evaluates the test
+//              for all CB blocks at once (lane t: block t; the patience run by
+//              warp ballots) and publishes the inclusive prefix; only then does
+//              it reduce the warps' states into the chunk's record, which no
+//              decision needs.
 // Posts alternate between two buffers, so the consumers run a chunk ahead of
-// the judge.  The probes and states live in global memory rewritten in place
+// the arbiter.  The probes and states live in global memory rewritten in place
 // (they stay in L2), which leaves the shared memory to a 3-stage ring at two
 // CTAs per SM.
 // A head that stops inside a chunk needs its state after the stop block, which
-// the consumers have already passed: the judge queues a request, the producer
+// the consumers have already passed: the arbiter queues a request, the producer
 // streams that chunk's blocks up to the stop once more through the ring (the
 // pages are usually still in L2) as tagged tiles, and the consumers fold them
-// for the stopping heads only; the judge overwrites the record.
+// for the stopping heads only; the arbiter overwrites the record.
 // Chunks taken after every head of a group has stopped issue no loads, and a
 // chunk in flight is cut short (checked every 8 tiles).  An optional gate
 // (DecodeParams::art_ahead) holds a group's chunk c until chunk c - ahead - 1
-// is judged, bounding the reads past a stop at the price of idle CTAs.
+// is decided, bounding the reads past a stop at the price of idle CTAs.
 // attn_decode's merge combines each head's records up to its stop chunk,
 // which is exact.
 #include "common.cuh"
@@ -90,7 +91,7 @@ template <int G, int NW, int CB, int ST>
 struct ArtCfg {  // shared-memory layout
   using Ln = Lanes<G, NW>;
   static constexpr int RPW = Ln::RPW;
-  static constexpr int THREADS = (NW + 2) * 32;  // consumers, producer, judge
+  static constexpr int THREADS = (NW + 2) * 32;  // consumers, producer, arbiter
   // a stage: K rows, V rows, and the group's q rows (loaded with a chunk's first block)
   static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes + (size_t)G * kRowBytes;
   static constexpr int NBAR = 2 * ST + 5;  // full, empty, fin, posted[2], free[2]
@@ -102,13 +103,13 @@ struct ArtCfg {  // shared-memory layout
   static constexpr size_t OFF_P = up16(OFF_REQ + kReqs * 16 + (size_t)kReqs * G * 4);  // float2 [NW][RPW][G]
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;   // float2 [NW][G]
   static constexpr size_t OFF_WCTL = up16(OFF_A + (size_t)NW * G * 8);  // int [NW][8]
-  static constexpr size_t OFF_LOCAL = OFF_WCTL + (size_t)NW * 8 * 4;    // float [CB][G][12] (judge)
+  static constexpr size_t OFF_LOCAL = OFF_WCTL + (size_t)NW * 8 * 4;    // float [CB][G][12] (arbiter)
   static constexpr size_t TOTAL = OFF_LOCAL + (size_t)CB * G * kProbeFloats * 4;
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_P % 16 == 0, "alignment");
   static_assert(OFF_A % 16 == 0 && OFF_WCTL % 16 == 0 && OFF_LOCAL % 16 == 0, "alignment");
   static_assert(OFF_TAG % 16 == 0 && OFF_REQ % 16 == 0, "alignment");
   static_assert((RPW * G * 8) % 16 == 0 || G == 1, "pbuf rows");
-  static_assert(CB >= 1 && CB <= 32, "one judge lane per block of a chunk");
+  static_assert(CB >= 1 && CB <= 32, "one arbiter lane per block of a chunk");
   static_assert(G * kProbeFloats <= 96, "look-back records of a group in three loads per lane");
 };
 
@@ -163,12 +164,12 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   uint64_t* empty = full + ST;
   uint64_t* fin_bar = empty + ST;
   uint64_t* posted = fin_bar + 1;   // [2] a post is ready (one arrival per consumer warp)
-  uint64_t* freed = posted + 2;     // [2] the judge is done with a post
+  uint64_t* freed = posted + 2;     // [2] the arbiter is done with a post
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows | 0 = end of chunk, group, chunk, block in chunk | blocks}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
-  // flags[0]: re-fold requests posted by the judge; flags[1]: abort (a bounded
+  // flags[0]: re-fold requests posted by the arbiter; flags[1]: abort (a bounded
   // wait expired); flags[2]: consumers finished (entries consumed + 1);
-  // flags[3]: the judge has handled every chunk (no more requests)
+  // flags[3]: the arbiter has handled every chunk (no more requests)
   volatile int* tag = reinterpret_cast<volatile int*>(smem + C::OFF_TAG);    // [2][4]: kind, group, chunk, a
   volatile int* req = reinterpret_cast<volatile int*>(smem + C::OFF_REQ);  // [kReqs][4]: group, chunk, vmask, stopmask
   volatile int* req_t = reinterpret_cast<volatile int*>(smem + C::OFF_REQ + kReqs * 16);  // [kReqs][G]
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     };
     const long long items = (long long)groups * p.art_maxc;
     // Re-fold request r: the chunk's blocks up to the last stop block, tagged,
-    // then a tagged end marker.  The request slot stays valid until the judge has
+    // then a tagged end marker.  The request slot stays valid until the arbiter has
     // taken the re-fold's post (it never has more than kReqs outstanding).
     auto serve = [&](int r) {
       const int slot = r % kReqs;
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       };
       if (!cur.skip && cur.c > p.art_ahead) {
         // Speculation gate: start the chunk only once chunk c - ahead - 1 of the
-        // group has been judged.  The awaited chunk has a smaller item number,
+        // group has been decided.  The awaited chunk has a smaller item number,
         // so the wait always ends.
         const int* rdy = ctl.ready + (size_t)cur.g * p.art_maxc + (cur.c - p.art_ahead - 1);
         const uint64_t t0 = globaltimer();
@@ -417,7 +418,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       prefetch();
       cur = nxt;
     }
-    // no more items: the consumers hand the judge a QUIT post; once the judge has
+    // no more items: the consumers hand the arbiter a QUIT post; once the arbiter has
     // handled every chunk, serve the last requests, then end the ring
     if (ok) {
       int r = 1;
@@ -453,7 +454,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     return;
   }
 
-  // ------------------------------------------------------------------ judge
+  // ------------------------------------------------------------------ arbiter
   if (warp == NW + 1) {
     int kj = 0;     // posts consumed
     int n_req = 0;  // re-run requests posted
@@ -792,7 +793,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   int kpar = 0;  // parity of the next post (its buffers hold the current item)
   bool ok = true;
 
-  // Take the buffers of the next post (the judge is done with the post two back).
+  // Take the buffers of the next post (the arbiter is done with the post two back).
   auto acquire = [&]() {
     const int kp = wc[W_KP];
     if (kp >= 2 && !mbar_wait_bounded(&freed[kp & 1], ((kp >> 1) - 1) & 1, &flags[1])) {
@@ -853,7 +854,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     const int4 mt = meta[s];
     const int n = mt.x;
     if (n == -1) break;
-    if (n == kDrainEntry) {  // no more items: let the judge finish, re-folds may follow
+    if (n == kDrainEntry) {  // no more items: let the arbiter finish, re-folds may follow
       release();
       acquire();
       publish(POST_QUIT, 0, 0, 0);
@@ -919,7 +920,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         if (req_t[slot * G + h] == pos) done_mask |= 1u << h;
     }
   }
-  if (ok) {  // release the judge
+  if (ok) {  // release the arbiter
     acquire();
     publish(POST_DONE, 0, 0, 0);
   }
@@ -974,7 +975,7 @@ int art_ctas_per_sm(int G) { return G == 8 ? art_minb<8>() : art_minb<4>(); }
 // Chunk length: 32 blocks, or 16 when the speculation window would be large.
 // About n_ctas / groups chunks of a group are in flight when one of its stops
 // is decided, and all of them are read in vain; keep that within 1/12 of the
-// traversal.  Shorter chunks cost more judging per block, so they are used
+// traversal.  Shorter chunks cost more deciding per block, so they are used
 // only where the window needs them.
 int art_chunk_blocks(int G, long long n_ctas, long long groups, long long positions) {
   (void)G;

@@ -62,7 +62,7 @@ struct DecodeParams {
   // per (group, chunk, head) (rec_nw = 1).
   int art_chunk;
   int art_maxc;
-  int art_ahead;  // a group's chunk c starts once chunk c - art_ahead - 1 is judged
+  int art_ahead;  // a group's chunk c starts once chunk c - art_ahead - 1 is decided
   int* art_ctl;
   float* art_lb;
   float* art_scratch;  // per-CTA probe slots and state area (stays in L2)
