@@ -14,7 +14,7 @@ import os
 from . import _build
 
 __all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_merge_lse",
-           "decode_workspace_size",
+           "decode_workspace_size", "decode_launches",
            "strerror", "SkvError", "lib", "DEV_BITS"]
 
 SKV_OK, SKV_EINVAL, SKV_EUNSUPPORTED, SKV_ECUDA, SKV_ETIMEOUT, SKV_EWORKSPACE = range(6)
