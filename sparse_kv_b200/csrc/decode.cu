@@ -780,7 +780,9 @@ int launch_t(const DecodeParams& p, cudaStream_t st) {
     return (int)cudaGetLastError();
   }
   // split schedule: one cluster of n_splits CTAs per group (<= 16; above 8
-  // needs the non-portable size, allowed once per device)
+  // needs the non-portable size, allowed once per device).  The split count
+  // only divides each group's walk (no workspace depends on it), so a cluster
+  // shape that cannot be resident at once is halved until it can.
   if (p.n_splits < 1 || p.n_splits > kMaxClusterSplits) return (int)cudaErrorInvalidValue;
   static bool np_set[64] = {};
   if (!np_set[dev]) {
@@ -788,28 +790,32 @@ int launch_t(const DecodeParams& p, cudaStream_t st) {
     if (err != cudaSuccess) return (int)err;
     np_set[dev] = true;
   }
+  DecodeParams q = p;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_splits, p.Hkv, p.B);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::TOTAL;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.n_splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // refuse a cluster shape that cannot be resident at once (checked once per size)
-  static int fits[64][kMaxClusterSplits + 1] = {};
-  if (fits[dev][p.n_splits] == 0) {
-    int n = 0;
-    cudaError_t err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-    if (err != cudaSuccess) return (int)err;
-    fits[dev][p.n_splits] = n > 0 ? 1 : -1;
+  static int fits[64][kMaxClusterSplits + 1] = {};  // 1: resident at once, -1: not (per size)
+  while (true) {
+    cfg.gridDim = dim3(q.n_splits, q.Hkv, q.B);
+    attr[0].val.clusterDim.x = q.n_splits;
+    if (fits[dev][q.n_splits] == 0) {
+      int n = 0;
+      cudaError_t err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (err != cudaSuccess) return (int)err;
+      fits[dev][q.n_splits] = n > 0 ? 1 : -1;
+    }
+    if (fits[dev][q.n_splits] > 0) break;
+    if (q.n_splits == 1) return (int)cudaErrorInvalidConfiguration;
+    q.n_splits = (q.n_splits + 1) / 2;
   }
-  if (fits[dev][p.n_splits] < 0) return (int)cudaErrorInvalidConfiguration;
-  return (int)cudaLaunchKernelEx(&cfg, kern, p);
+  return (int)cudaLaunchKernelEx(&cfg, kern, q);
 }
 
 }  // namespace

@@ -6,7 +6,7 @@ import pytest
 import oracle
 import skvgen
 from helpers import (check_art, check_close, check_selection, device_workload, group_inputs,
-                     oracle_keys_attend, run_decode)
+                     oracle_keys_attend, outputs, run_decode)
 
 pytestmark = pytest.mark.gpu
 
@@ -75,6 +75,22 @@ def test_cfg1_full_traversal():
     assert res[3] == 0
     _check_all_groups(wl, res, lambda b: oracle.keys_full(wl.seq_len(b)))
     assert np.all(res[2] == 64)
+
+
+@pytest.mark.parametrize("G,Hkv,L", [(8, 1, 4096), (4, 1, 4096), (1, 2, 64 * 40 + 9), (2, 3, 64 * 5)])
+def test_split_cluster_sizes(G, Hkv, L):
+    # one KV group walked by clusters of up to 16 CTAs (G = 8 runs one CTA per
+    # SM, so 16 pieces need 16 SMs; a size that cannot be resident is halved)
+    import sparse_kv_b200 as skv
+    wl = skvgen.Workload("cs", B=1, Hq=G * Hkv, Hkv=Hkv, L=L, paging="perm", seed=80 + G)
+    dev = device_workload(wl)
+    out, lse = outputs(wl)
+    args = (dev["q"], dev["k_pool"], dev["v_pool"], dev["block_table"], dev["seq_lens"], out, lse)
+    assert skv.decode_launches(*args, max_seq_len=wl.Lmax) == 1
+    res = run_decode(wl, dev)
+    assert res[3] == 0
+    _check_all_groups(wl, res, lambda b: oracle.keys_full(wl.seq_len(b)))
+    np.testing.assert_array_equal(res[2], wl.nb(0))
 
 
 def test_split_merge_repeats():
