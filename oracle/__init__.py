@@ -16,6 +16,8 @@ each option attends, following the pages:
                               ("Squeezed Attention" Q2, steps 2-3)
 * causal query chunk       -- chunk token t sees the context and chunk keys 0..t
 * shard merge              -- "Pulsar Attention" Phase 2
+* layer routing            -- "Flux Attention" 2 (Layer Router: prefix and
+                              suffix pooling of the query tensor, hard routing)
 
 Parity pins for every function are in tests/test_oracle_pins.py.
 """
@@ -193,3 +195,26 @@ def topk_boundary_gap(scores, k):
         a, b = s[order[k - 1]], s[order[k]]
         out.append(abs(a - b) / max(abs(a), 1e-300))
     return np.array(out)
+
+
+def _bf16_values(bits):
+    """bf16 bit patterns -> float64 values (the upper half of an fp32)."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def route(q, w, bias, n_prefix, n_suffix):
+    """Flux-style layer routing ("Flux Attention" 2, Layer Router): the start
+    and end tokens of each layer's query tensor are pooled (mean over the
+    first n_prefix and the last n_suffix tokens), a linear map of the two
+    pooled vectors gives the layer's logit, and inference routes hard: full
+    attention where the logit is above zero.
+      q     bf16 bits [L][B][T][F] (F = q_heads * head_dim, a query row)
+      w     [L][2F] weights (prefix features first), bias [L]
+    Returns the logits z [L][B] (fp64) and the route bits [L][B] (1 = full)."""
+    x = _bf16_values(q)
+    T = x.shape[2]
+    prefix = x[:, :, :n_prefix, :].mean(axis=2)
+    suffix = x[:, :, T - n_suffix:, :].mean(axis=2)
+    f = np.concatenate([prefix, suffix], axis=-1)  # [L][B][2F]
+    z = np.einsum("lbf,lf->lb", f, np.asarray(w, dtype=np.float64)) + np.asarray(bias, dtype=np.float64)[:, None]
+    return z, (z > 0).astype(np.uint8)

@@ -390,3 +390,68 @@ def test_topk_boundary_gap():
     assert g[0] == 0.0
     g = oracle.topk_boundary_gap(np.array([[4.0, 1.0, 2.0]]), 1)
     assert abs(g[0] - 0.5) < 1e-15
+
+
+# ----------------------------------------------------------------------------- layer routing
+
+def test_route_constant_tokens_closed_form():
+    # every token of every layer equals c: both pooled vectors are c, so the
+    # logit is c * (sum of the layer's weights) + bias
+    L, B, T, F = 3, 2, 7, 16
+    c = 0.375
+    q = np.full((L, B, T, F), bf16_bits([c])[0], dtype=np.uint16)
+    w = RNG.standard_normal((L, 2 * F))
+    bias = RNG.standard_normal(L)
+    z, r = oracle.route(q, w, bias, 3, 2)
+    want = c * w.sum(axis=1) + bias
+    np.testing.assert_allclose(z, np.repeat(want[:, None], B, axis=1), rtol=1e-14, atol=1e-14)
+    np.testing.assert_array_equal(r, (z > 0).astype(np.uint8))
+
+
+def test_route_one_hot_weights_pick_one_pooled_feature():
+    # a weight vector with a single 1 reads one feature of one pooled vector:
+    # the mean of that feature over the prefix (or suffix) tokens, by a loop
+    L, B, T, F = 2, 3, 9, 8
+    q = bf16_bits(RNG.standard_normal((L, B, T, F)))
+    vals = bf16_vals(q)
+    n_p, n_s = 4, 3
+    for j, suffix in ((5, False), (2, True)):
+        w = np.zeros((L, 2 * F))
+        w[:, F * suffix + j] = 1.0
+        z, _ = oracle.route(q, w, np.zeros(L), n_p, n_s)
+        for l in range(L):
+            for b in range(B):
+                toks = range(T - n_s, T) if suffix else range(n_p)
+                s = 0.0
+                for t in toks:
+                    s += vals[l, b, t, j]
+                assert z[l, b] == pytest.approx(s / len(toks), rel=1e-15, abs=1e-15)
+
+
+def test_route_brute_force_tiny():
+    L, B, T, F = 2, 2, 5, 4
+    q = bf16_bits(RNG.standard_normal((L, B, T, F)))
+    vals = bf16_vals(q)
+    w = RNG.standard_normal((L, 2 * F))
+    bias = RNG.standard_normal(L)
+    n_p, n_s = 2, 4  # prefix and suffix overlap: each is pooled on its own
+    z, r = oracle.route(q, w, bias, n_p, n_s)
+    for l in range(L):
+        for b in range(B):
+            acc = bias[l]
+            for j in range(F):
+                pre = sum(vals[l, b, t, j] for t in range(n_p)) / n_p
+                suf = sum(vals[l, b, t, j] for t in range(T - n_s, T)) / n_s
+                acc += w[l, j] * pre + w[l, F + j] * suf
+            assert z[l, b] == pytest.approx(acc, rel=1e-12, abs=1e-12)
+            assert r[l, b] == (1 if acc > 0 else 0)
+
+
+def test_route_hard_decision_is_strict():
+    # zero queries and zero bias give a zero logit: not above zero, so sparse
+    L, B, T, F = 1, 2, 3, 8
+    q = np.zeros((L, B, T, F), dtype=np.uint16)
+    z, r = oracle.route(q, RNG.standard_normal((L, 2 * F)), np.zeros(L), 1, 1)
+    assert np.all(z == 0.0) and np.all(r == 0)
+    z, r = oracle.route(q, RNG.standard_normal((L, 2 * F)), np.full(L, 1e-30), 1, 1)
+    assert np.all(r == 1)
