@@ -355,6 +355,36 @@ def build_routed(torch, skv, skvgen, wl, status):
     return step
 
 
+def build_router(torch, skv, skvgen, wl, n_prefix=64, n_suffix=64):
+    """The routing decision of a routed stack ("Flux Attention" 2, Layer
+    Router): pooled prefix and suffix query rows of every layer -> one logit
+    and route bit per (layer, sequence).  Synthetic prefill queries (only the
+    pooled rows are held) and untrained router weights."""
+    L, B, T, F = wl.n_layers, wl.B, n_prefix + n_suffix, wl.Hq * wl.d
+    q = torch.empty((L, B, T, wl.Hq, wl.d), dtype=torch.bfloat16, device="cuda")
+    skvgen.device_normal_bf16(q, wl.seed, skvgen.S_Q, layer=1 << 20)
+    w = torch.empty((L, 2 * F), dtype=torch.bfloat16, device="cuda")
+    skvgen.device_normal_bf16(w, wl.seed, skvgen.S_ROUTER_W)
+    w = (w.float() / 32).contiguous()
+    bias = torch.zeros(L, dtype=torch.float32, device="cuda")
+    route = torch.empty((L, B), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((L, B), dtype=torch.float32, device="cuda")
+    L_ = skv.lib()
+    args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(w.data_ptr()), ctypes.c_void_p(bias.data_ptr()),
+            L, B, T, wl.Hq, wl.d, n_prefix, n_suffix, ctypes.c_void_p(logits.data_ptr()),
+            ctypes.c_void_p(route.data_ptr()))
+
+    def run():
+        st = L_.attn_route_layers(*args, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise skv.SkvError(st, "attn_route_layers")
+
+    step = Step(run, q.numel() * 2 + w.numel() * 4, 1, {"layers": L, "sequences": B,
+                                                          "pooled_rows": T, "features": F})
+    step.tensors = dict(q=q, w=w, bias=bias, route=route, logits=logits)
+    return step
+
+
 def build_chunk(torch, skv, skvgen, wl, status):
     """Query chunk of Tq tokens: 8 context shards (one launch, one partial per
     shard), the chunk's own keys under a causal mask, and the exact merge."""
@@ -456,6 +486,7 @@ def main():
         # looser thresholds on the same cache, where heads do stop: savings vs blocks skipped
         for thr in ((5e-2, 5e-3, 2), (2e-2, 2e-3, 2)):
             sweep_steps.append((thr, build_decode(torch, skv, skvgen, wl, status, art=thr, inputs=shared)))
+    router_step = build_router(torch, skv, skvgen, wl) if kind == "cfg5" else None
     if kind == "cfg3":  # the same cache walked in full, for the savings of the selection
         T = step.tensors
         dense_step = build_decode(torch, skv, skvgen, wl, status,
@@ -503,6 +534,8 @@ def main():
                     for _, st in sweep_steps]
         dense_ms = (timed(dense_step, max(10, args.steps // 4), args.warmup)[0] / max(10, args.steps // 4)
                     if dense_step is not None else None)
+        router_ms = (timed(router_step, args.steps, args.warmup)[0] / args.steps
+                     if router_step is not None else None)
     clocks = clk.summary()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status word {int(status.item()):#x}")
@@ -609,6 +642,15 @@ def main():
                             "bytes_vs_dense": step.nbytes / wl.kv_bytes(),
                             "note": "same cache walked in full by the plain decode kernel"}
         res["gpu_launches"] += max(10, args.steps // 4) * dense_step.launches
+    if router_ms is not None:
+        gbs = router_step.nbytes / (router_ms * 1e-3) / 1e9
+        res["router"] = {"ms_per_call": router_ms, "bytes_per_call": router_step.nbytes, "gbs": gbs,
+                         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                                      "frac": gbs / hbm_peak},
+                         **router_step.extra,
+                         "note": "per-layer route bits from pooled prefix/suffix query rows "
+                                 "(untrained weights); outside the timed decode step"}
+        res["gpu_launches"] += args.steps * router_step.launches
     if e2e is not None:
         res["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline and kind in ("cfg1", "cfg2"):

@@ -28,6 +28,11 @@
  *  attn_merge_lse   Exact merge of per-shard attention partials by their
  *                   log-sum-exp ("Pulsar Attention" Phase 2, online softmax
  *                   merge).
+ *  attn_route_layers
+ *                   Per-layer hard routing between full and sparse attention
+ *                   ("Flux Attention" section 2, Layer Router: pooling of the
+ *                   query tensor's first and last tokens), with caller-given
+ *                   router weights.
  *
  * Conventions (all calls):
  *  - The caller owns and allocates every buffer; the library never allocates
@@ -222,6 +227,29 @@ SKV_API skv_status attn_select_centroids(const void* q, const void* centroids, c
  * head_dim must be a multiple of 4 and <= 512; 16-byte aligned o_parts/out. */
 SKV_API skv_status attn_merge_lse(const float* o_parts, const float* lse_parts, int n_parts, int n_rows,
                           int head_dim, float* out, float* lse, skv_stream_t stream);
+
+/* Per-layer hard routing ("Flux Attention" section 2: a Layer Router pools
+ * the first and last tokens of the input query tensor and decides, per layer,
+ * full attention (FA) or sparse attention (SA); inference uses the hard
+ * decision, made once per prefill).  For layer l and sequence b, with
+ * F = q_heads * head_dim:
+ *   p = mean over t <  n_prefix          of q[l][b][t][:]
+ *   s = mean over t >= tokens - n_suffix of q[l][b][t][:]
+ *   z = w[l][0:F] . p + w[l][F:2F] . s + bias[l]
+ *   route[l][b] = z > 0 ? 1 (FA) : 0 (SA);   logits[l][b] = z
+ * The prefix and suffix may overlap.  The router's weights come from the
+ * caller (the pages train them; this call only applies them).
+ *  q       bf16 [n_layers][batch][tokens][q_heads][head_dim], 16-byte aligned
+ *  w       fp32 [n_layers][2 * F], 16-byte aligned
+ *  bias    fp32 [n_layers], or NULL for zero
+ *  logits  fp32 [n_layers][batch], or NULL
+ *  route   uint8 [n_layers][batch]
+ * Errors: SKV_EINVAL for a NULL q/w/route, a non-positive size, n_prefix or
+ * n_suffix outside [1, tokens], or misalignment; SKV_EUNSUPPORTED if F is not
+ * a multiple of 8 or n_layers > 65535; SKV_ECUDA if the launch fails. */
+SKV_API skv_status attn_route_layers(const void* q, const float* w, const float* bias, int n_layers,
+                             int batch, int tokens, int q_heads, int head_dim, int n_prefix,
+                             int n_suffix, float* logits, uint8_t* route, skv_stream_t stream);
 
 /* Static description of a status code. */
 SKV_API const char* skv_strerror(skv_status s);

@@ -18,7 +18,7 @@ from . import _build
 _HOST = None
 _DEV = None
 
-S_Q, S_K, S_V, S_CENTER, S_ASSIGN, S_PERM, S_HEAVY, S_ROUTE = 1, 2, 3, 4, 5, 6, 7, 8
+S_Q, S_K, S_V, S_CENTER, S_ASSIGN, S_PERM, S_HEAVY, S_ROUTE, S_ROUTER_W = 1, 2, 3, 4, 5, 6, 7, 8, 9
 
 _u64, _u32, _i32, _i64, _p = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
 

@@ -14,6 +14,7 @@ import os
 from . import _build
 
 __all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_merge_lse",
+           "attn_route_layers",
            "decode_workspace_size", "decode_launches",
            "strerror", "SkvError", "lib", "DEV_BITS"]
 
@@ -75,6 +76,8 @@ def lib():
         L.attn_select_centroids.restype = _i
         L.attn_merge_lse.argtypes = [_p, _p, _i, _i, _i, _p, _p, _p]
         L.attn_merge_lse.restype = _i
+        L.attn_route_layers.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p]
+        L.attn_route_layers.restype = _i
         L.skv_strerror.argtypes = [_i]
         L.skv_strerror.restype = ctypes.c_char_p
         _LIB = L
@@ -194,3 +197,13 @@ def attn_merge_lse(o_parts, lse_parts, out, lse, stream=None):
                               _stream(stream))
     if st != SKV_OK:
         raise SkvError(st, "attn_merge_lse")
+
+
+def attn_route_layers(q, w, bias, n_prefix, n_suffix, route, logits=None, stream=None):
+    """q bf16 [L, B, T, Hq, d]; w fp32 [L, 2 * Hq * d]; bias fp32 [L] or None ->
+    route uint8 [L, B] (1: full attention), logits fp32 [L, B] (optional)."""
+    L, B, T, Hq, d = q.shape
+    st = lib().attn_route_layers(_ptr(q), _ptr(w), _ptr(bias), L, B, T, Hq, d, int(n_prefix),
+                                 int(n_suffix), _ptr(logits), _ptr(route), _stream(stream))
+    if st != SKV_OK:
+        raise SkvError(st, "attn_route_layers")

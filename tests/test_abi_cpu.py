@@ -144,6 +144,23 @@ def test_select_and_merge_reject_on_host():
     assert mer(None, FAKE, 2, 10, 128, FAKE, FAKE, None) == skv.SKV_EINVAL
 
 
+def test_route_rejects_on_host():
+    L = skv.lib()
+    r = L.attn_route_layers
+    ok = (FAKE, FAKE, None, 32, 8, 128, 32, 128, 64, 64, None, FAKE, None)
+    args = lambda **kw: tuple(kw.get(n, v) for n, v in zip(
+        ["q", "w", "bias", "L", "B", "T", "Hq", "d", "np", "ns", "logits", "route", "s"], ok))
+    assert r(*args(q=None)) == skv.SKV_EINVAL
+    assert r(*args(route=None)) == skv.SKV_EINVAL
+    assert r(*args(L=0)) == skv.SKV_EINVAL
+    assert r(*args(np=0)) == skv.SKV_EINVAL
+    assert r(*args(ns=129)) == skv.SKV_EINVAL       # more suffix tokens than tokens
+    assert r(*args(q=FAKE + 8)) == skv.SKV_EINVAL   # misaligned
+    assert r(*args(w=FAKE + 4)) == skv.SKV_EINVAL
+    assert r(*args(Hq=3, d=5)) == skv.SKV_EUNSUPPORTED  # 15 features: not a multiple of 8
+    assert r(*args(L=70000)) == skv.SKV_EUNSUPPORTED
+
+
 def test_strerror():
     assert skv.strerror(skv.SKV_OK) == "ok"
     assert "workspace" in skv.strerror(skv.SKV_EWORKSPACE)
