@@ -620,6 +620,7 @@ def main():
         art_step_ms = art_ms / args.steps
         res["art"] = {"ms_per_step": art_step_ms, "kv_gbs": art_bytes / (art_step_ms * 1e-3) / 1e9,
                       "blocks_consumed_mean": float(cons.mean()), "blocks_total": wl.nb(0),
+                      "group_blocks_hist16": np.histogram(grp, bins=16, range=(0, wl.nb(0)))[0].tolist(),
                       "blocks_skipped_frac": 1.0 - float(grp.sum()) / (wl.B * wl.Hkv * wl.nb(0)),
                       "time_vs_full": art_step_ms / ms_step,
                       "attended_tokens_per_s": float(cons.sum()) * wl.bs / (art_step_ms * 1e-3),
@@ -633,7 +634,8 @@ def main():
             saved = 1.0 - ms / ms_step
             return {"ms_per_step": ms, "blocks_skipped_frac": skipped, "time_saved_frac": saved,
                     "saved_per_skipped": saved / skipped if skipped > 0 else None,
-                    "blocks_consumed_mean": float(cons.mean())}
+                    "blocks_consumed_mean": float(cons.mean()),
+                    "group_blocks_hist16": np.histogram(grp, bins=16, range=(0, wl.nb(0)))[0].tolist()}
         res["art_sweep"] = [dict(tau=thr[0], phi=thr[1], patience=thr[2], **art_summary(st, ms))
                             for (thr, st), ms in zip(sweep_steps, sweep_ms)]
         res["gpu_launches"] += sum(max(10, args.steps // 4) * st.launches for _, st in sweep_steps)
