@@ -18,6 +18,9 @@ each option attends, following the pages:
 * shard merge              -- "Pulsar Attention" Phase 2
 * layer routing            -- "Flux Attention" 2 (Layer Router: prefix and
                               suffix pooling of the query tensor, hard routing)
+* two-level selection      -- "Squeezed Attention" Q2 step 4 (hierarchical
+                              clustering: coarse clusters first, then the fine
+                              clusters inside the chosen coarse ones)
 
 Parity pins for every function are in tests/test_oracle_pins.py.
 """
@@ -169,6 +172,31 @@ def select(q, cent, k):
     sc = np.empty((U, C))
     lib().orc_select(U, G, d, _ptr(q), _ptr(cent), C, k, _ptr(ids), _ptr(sc))
     return ids, sc
+
+
+def select2(q, coarse, coarse_off, fine, k1, k2):
+    """Two-level centroid selection ("Squeezed Attention" Q2 step 4,
+    hierarchical clustering).  Per unit: pick the k1 best coarse clusters by
+    select(); their fine clusters (coarse cluster i owns the fine clusters
+    coarse_off[i] .. coarse_off[i+1] - 1) are the candidates; pick the
+    min(k2, #candidates) best candidates by select() over the candidates'
+    centroids.  Ties go to the lower index at both levels.
+      q [U][G][d], coarse [U][C1][d], fine [U][C][d] (bf16 bits);
+      coarse_off [U][C1 + 1] (int).
+    Returns fine ids [U][k2], ascending, then -1 for unused slots."""
+    q, coarse, fine = _u16(q), _u16(coarse), _u16(fine)
+    U = q.shape[0]
+    out = np.full((U, k2), -1, dtype=np.int32)
+    for u in range(U):
+        ids1, _ = select(q[u:u + 1], coarse[u:u + 1], k1)
+        cand = np.concatenate([np.arange(coarse_off[u][i], coarse_off[u][i + 1]) for i in ids1[0]]
+                              + [np.zeros(0, dtype=np.int64)]).astype(np.int64)
+        if cand.size == 0:
+            continue
+        kk = min(k2, cand.size)
+        local, _ = select(q[u:u + 1], fine[u:u + 1, cand], kk)
+        out[u, :kk] = cand[local[0]]
+    return out
 
 
 def merge(o_parts, lse_parts):

@@ -455,3 +455,73 @@ def test_route_hard_decision_is_strict():
     assert np.all(z == 0.0) and np.all(r == 0)
     z, r = oracle.route(q, RNG.standard_normal((L, 2 * F)), np.full(L, 1e-30), 1, 1)
     assert np.all(r == 1)
+
+
+# ----------------------------------------------------------------------------- two-level selection
+
+def _hier(U, G, d, C1, per, seed):
+    rng = np.random.default_rng(seed)
+    C = C1 * per
+    q = bf16_bits(rng.standard_normal((U, G, d)))
+    fine = bf16_bits(rng.standard_normal((U, C, d)))
+    coarse = bf16_bits(bf16_vals(fine).reshape(U, C1, per, d).mean(axis=2))
+    off = np.tile(np.arange(0, C + 1, per), (U, 1))
+    return q, coarse, off, fine
+
+
+def test_select2_all_coarse_is_flat_selection():
+    # keeping every coarse cluster leaves every fine cluster a candidate: the
+    # second level is then exactly the one-level top-k
+    q, coarse, off, fine = _hier(3, 4, 16, 8, 5, 11)
+    for k2 in (1, 7, 40):
+        got = oracle.select2(q, coarse, off, fine, 8, k2)
+        want, _ = oracle.select(q, fine, k2)
+        np.testing.assert_array_equal(got, want)
+
+
+def test_select2_picks_the_best_candidates_only():
+    # fine clusters outside the chosen coarse clusters never appear, and the
+    # chosen ones are the k2 best candidates by a plain sort (score desc, index asc)
+    q, coarse, off, fine = _hier(4, 2, 8, 10, 6, 12)
+    k1, k2 = 3, 5
+    got = oracle.select2(q, coarse, off, fine, k1, k2)
+    qs = bf16_vals(q).sum(axis=1)
+    for u in range(4):
+        sc1 = bf16_vals(coarse[u]) @ qs[u]
+        top1 = sorted(range(10), key=lambda i: (-sc1[i], i))[:k1]
+        cand = [c for i in sorted(top1) for c in range(off[u][i], off[u][i + 1])]
+        sc2 = bf16_vals(fine[u]) @ qs[u]
+        want = sorted(sorted(cand, key=lambda c: (-sc2[c], c))[:k2])
+        assert list(got[u]) == want
+
+
+def test_select2_fewer_candidates_than_k2():
+    # 2 coarse clusters of 3 fine ones each can offer only 6 candidates
+    q, coarse, off, fine = _hier(1, 1, 8, 4, 3, 13)
+    got = oracle.select2(q, coarse, off, fine, 2, 9)
+    assert (got[0, :6] >= 0).all() and (got[0, 6:] == -1).all()
+    assert list(got[0, :6]) == sorted(got[0, :6])
+
+
+def test_select2_squeezed_hierarchy_example():
+    rows, expect = {}, {}
+    for line in open(os.path.join(GOLDEN, "squeezed_hierarchy.txt")):
+        s = line.split()
+        if not s or s[0].startswith("#"):
+            continue
+        if s[0].startswith("expect_"):
+            expect[s[0]] = s[1:]
+        else:
+            rows[s[0]] = [float(x) for x in s[1:]]
+    names = ["apple", "banana", "carrot", "dog", "elephant", "fish"]
+    keys = np.array([rows[n] for n in names])
+    fine_members = [[0, 1], [2], [3, 4], [5]]           # A1, A2, B1, B2
+    coarse_members = [[0, 1, 2], [3, 4, 5]]             # A, B
+    fine = bf16_bits(np.array([keys[m].mean(axis=0) for m in fine_members]))[None]
+    coarse = bf16_bits(np.array([keys[m].mean(axis=0) for m in coarse_members]))[None]
+    off = np.array([[0, 2, 4]])
+    q = bf16_bits(np.array(rows["query"]))[None, None]
+    got = oracle.select2(q, coarse, off, fine, 1, 1)
+    fine_names = ["A1", "A2", "B1", "B2"]
+    assert [fine_names[i] for i in got[0]] == expect["expect_fine"]
+    assert [names[i] for i in fine_members[got[0][0]]] == expect["expect_keys"]
