@@ -28,6 +28,10 @@
  *  attn_merge_lse   Exact merge of per-shard attention partials by their
  *                   log-sum-exp ("Pulsar Attention" Phase 2, online softmax
  *                   merge).
+ *  attn_select_centroids2
+ *                   Two-level (hierarchical) centroid selection ("Squeezed
+ *                   Attention", Q2 step 4): coarse clusters first, then the
+ *                   fine clusters inside the chosen ones.
  *  attn_route_layers
  *                   Per-layer hard routing between full and sparse attention
  *                   ("Flux Attention" section 2, Layer Router: pooling of the
@@ -214,6 +218,35 @@ SKV_API skv_status attn_select_centroids(const void* q, const void* centroids, c
                                  int batch, int q_heads, int kv_heads, int head_dim,
                                  int n_clusters, int topk, int32_t* sel_ids, int32_t* seg_start,
                                  int32_t* seg_end, skv_stream_t stream);
+
+/* Two-level centroid selection ("Squeezed Attention" Q2 step 4, hierarchical
+ * clustering) for each KV group (b, kvh), with the group's query heads summed
+ * as in attn_select_centroids:
+ *   1. score the n_coarse coarse centroids, keep the k1 best (ties to the
+ *      lower id);
+ *   2. the candidates are the fine clusters of the kept coarse clusters
+ *      (coarse cluster i owns fine clusters coarse_off[i] .. coarse_off[i+1]-1);
+ *   3. score only the candidates' fine centroids and keep the
+ *      min(k2, #candidates) best (ties to the lower fine id).
+ * The kept fine ids are written ascending with their key ranges
+ *   seg_start[i] = cluster_off[id_i], seg_end[i] = cluster_off[id_i + 1];
+ * unused slots get id -1 and an empty range [0, 0) (which attn_decode's
+ * segment traversal attends as nothing).
+ *  q           bf16 [batch][q_heads][head_dim] (one query token)
+ *  coarse      bf16 [batch][kv_heads][n_coarse][head_dim], 16-byte aligned
+ *  coarse_off  int32 [batch][kv_heads][n_coarse + 1], within [0, n_fine]
+ *  fine        bf16 [batch][kv_heads][n_fine][head_dim], 16-byte aligned
+ *  cluster_off int32 [batch][kv_heads][n_fine + 1]: fine cluster f holds the
+ *              cache tokens [cluster_off[f], cluster_off[f+1])
+ *  sel_ids, seg_start, seg_end  int32 [batch][kv_heads][k2] (outputs)
+ * Supported: head_dim 128, n_coarse <= 1024, n_fine <= 4096; 1 <= k1 <=
+ * n_coarse, 1 <= k2 <= n_fine (else SKV_EINVAL).  coarse_off ranges are
+ * clamped to [0, n_fine). */
+SKV_API skv_status attn_select_centroids2(const void* q, const void* coarse, const int32_t* coarse_off,
+                                  const void* fine, const int32_t* cluster_off, int batch,
+                                  int q_heads, int kv_heads, int head_dim, int n_coarse,
+                                  int n_fine, int k1, int k2, int32_t* sel_ids,
+                                  int32_t* seg_start, int32_t* seg_end, skv_stream_t stream);
 
 /* Exact LSE merge ("Pulsar Attention" Phase 2) of n_parts partials of n_rows
  * rows each:

@@ -14,7 +14,7 @@ import os
 from . import _build
 
 __all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_merge_lse",
-           "attn_route_layers",
+           "attn_route_layers", "attn_select_centroids2",
            "decode_workspace_size", "decode_launches",
            "strerror", "SkvError", "lib", "DEV_BITS"]
 
@@ -78,6 +78,8 @@ def lib():
         L.attn_merge_lse.restype = _i
         L.attn_route_layers.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p]
         L.attn_route_layers.restype = _i
+        L.attn_select_centroids2.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p]
+        L.attn_select_centroids2.restype = _i
         L.skv_strerror.argtypes = [_i]
         L.skv_strerror.restype = ctypes.c_char_p
         _LIB = L
@@ -207,3 +209,18 @@ def attn_route_layers(q, w, bias, n_prefix, n_suffix, route, logits=None, stream
                                  int(n_suffix), _ptr(logits), _ptr(route), _stream(stream))
     if st != SKV_OK:
         raise SkvError(st, "attn_route_layers")
+
+
+def attn_select_centroids2(q, coarse, coarse_off, fine, cluster_off, k1, k2, ids, seg_start, seg_end,
+                           stream=None):
+    """q bf16 [B, Hq, d] (or [B, 1, Hq, d]); coarse bf16 [B, Hkv, C1, d]; coarse_off int32
+    [B, Hkv, C1 + 1]; fine bf16 [B, Hkv, C, d]; cluster_off int32 [B, Hkv, C + 1] ->
+    ids, seg_start, seg_end int32 [B, Hkv, k2] (unused slots: id -1, empty range)."""
+    B, Hkv, C1, d = coarse.shape
+    C = fine.shape[2]
+    Hq = q.shape[-2]
+    st = lib().attn_select_centroids2(_ptr(q), _ptr(coarse), _ptr(coarse_off), _ptr(fine), _ptr(cluster_off),
+                                      B, Hq, Hkv, d, C1, C, int(k1), int(k2), _ptr(ids), _ptr(seg_start),
+                                      _ptr(seg_end), _stream(stream))
+    if st != SKV_OK:
+        raise SkvError(st, "attn_select_centroids2")

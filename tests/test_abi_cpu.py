@@ -161,6 +161,28 @@ def test_route_rejects_on_host():
     assert r(*args(L=70000)) == skv.SKV_EUNSUPPORTED
 
 
+def test_select2_rejects_on_host():
+    s = skv.lib().attn_select_centroids2
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, 8, 32, 8, 128, 32, 1024, 4, 102, FAKE, FAKE, FAKE, None]
+    def call(**kw):
+        names = ["q", "coarse", "co", "fine", "clo", "B", "Hq", "Hkv", "d", "C1", "C", "k1", "k2",
+                 "ids", "ss", "se", "s"]
+        a = list(ok)
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return s(*a)
+    assert call(q=None) == skv.SKV_EINVAL
+    assert call(co=None) == skv.SKV_EINVAL
+    assert call(Hq=30) == skv.SKV_EINVAL
+    assert call(d=64) == skv.SKV_EUNSUPPORTED
+    assert call(k1=0) == skv.SKV_EINVAL
+    assert call(k1=33) == skv.SKV_EINVAL        # more coarse clusters kept than exist
+    assert call(k2=1025) == skv.SKV_EINVAL
+    assert call(C1=2048, k1=4) == skv.SKV_EUNSUPPORTED
+    assert call(C=8192) == skv.SKV_EUNSUPPORTED
+    assert call(fine=FAKE + 8) == skv.SKV_EINVAL
+
+
 def test_strerror():
     assert skv.strerror(skv.SKV_OK) == "ok"
     assert "workspace" in skv.strerror(skv.SKV_EWORKSPACE)
