@@ -355,6 +355,42 @@ def build_routed(torch, skv, skvgen, wl, status):
     return step
 
 
+def build_select_levels(torch, skv, skvgen, wl, sel_step, per=32, k1=8):
+    """Centroid selection alone, flat (all C fine centroids) and two-level
+    ("Squeezed Attention" Q2 step 4): coarse clusters = runs of `per`
+    consecutive fine clusters, centroid = mean of theirs (input preparation,
+    as offline clustering would be); keep k1 coarse, then the top-k of their
+    fine clusters.  Returns (flat step, two-level step)."""
+    T = sel_step.tensors
+    q, cent, off = T["q"], T["cent"], T["off"]
+    B, Hkv, C, k = wl.B, wl.Hkv, 1 << wl.c_log2, wl.topk
+    C1 = C // per
+    coarse = cent.view(B, Hkv, C1, per, wl.d).float().mean(dim=3).to(torch.bfloat16).contiguous()
+    coarse_off = torch.arange(0, C + 1, per, dtype=torch.int32, device="cuda").expand(B, Hkv, C1 + 1).contiguous()
+    outs = [torch.empty((B, Hkv, k), dtype=torch.int32, device="cuda") for _ in range(6)]
+    L = skv.lib()
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    cur = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def flat():
+        st = L.attn_select_centroids(p(q), p(cent), p(off), B, wl.Hq, Hkv, wl.d, C, k, p(outs[0]), p(outs[1]),
+                                     p(outs[2]), cur())
+        if st != 0:
+            raise skv.SkvError(st, "attn_select_centroids")
+
+    def two():
+        st = L.attn_select_centroids2(p(q), p(coarse), p(coarse_off), p(cent), p(off), B, wl.Hq, Hkv, wl.d,
+                                      C1, C, k1, k, p(outs[3]), p(outs[4]), p(outs[5]), cur())
+        if st != 0:
+            raise skv.SkvError(st, "attn_select_centroids2")
+
+    f = Step(flat, cent.numel() * 2, 1, {"centroids_read": C})
+    t = Step(two, coarse.numel() * 2 + B * Hkv * k1 * per * wl.d * 2, 1,
+             {"centroids_read": C1 + k1 * per, "coarse": C1, "k1": k1})
+    f.tensors = t.tensors = dict(q=q, cent=cent, off=off, coarse=coarse, coarse_off=coarse_off, outs=outs)
+    return f, t
+
+
 def build_router(torch, skv, skvgen, wl, n_prefix=64, n_suffix=64):
     """The routing decision of a routed stack ("Flux Attention" 2, Layer
     Router): pooled prefix and suffix query rows of every layer -> one logit
@@ -487,10 +523,12 @@ def main():
         for thr in ((5e-2, 5e-3, 2), (2e-2, 2e-3, 2)):
             sweep_steps.append((thr, build_decode(torch, skv, skvgen, wl, status, art=thr, inputs=shared)))
     router_step = build_router(torch, skv, skvgen, wl) if kind == "cfg5" else None
+    level_steps = None
     if kind == "cfg3":  # the same cache walked in full, for the savings of the selection
         T = step.tensors
         dense_step = build_decode(torch, skv, skvgen, wl, status,
                                   inputs=(T["q"], T["k_pool"], T["v_pool"], T["bt"], T["sl"]))
+        level_steps = build_select_levels(torch, skv, skvgen, wl, step)
     stream = torch.cuda.current_stream()
 
     def timed(st, steps, warmup):
@@ -536,6 +574,8 @@ def main():
                     if dense_step is not None else None)
         router_ms = (timed(router_step, args.steps, args.warmup)[0] / args.steps
                      if router_step is not None else None)
+        level_ms = ([timed(st, args.steps, args.warmup)[0] / args.steps for st in level_steps]
+                    if level_steps is not None else None)
     clocks = clk.summary()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status word {int(status.item()):#x}")
@@ -644,6 +684,14 @@ def main():
                             "bytes_vs_dense": step.nbytes / wl.kv_bytes(),
                             "note": "same cache walked in full by the plain decode kernel"}
         res["gpu_launches"] += max(10, args.steps // 4) * dense_step.launches
+    if level_ms is not None:
+        f, t = level_steps
+        res["selection_levels"] = {
+            "flat": {"ms_per_call": level_ms[0], "centroids_read": f.extra["centroids_read"]},
+            "two_level": {"ms_per_call": level_ms[1], **t.extra},
+            "note": "selection alone (no attention): flat top-k over all fine centroids vs coarse "
+                    "top-k1 then top-k among the kept coarse clusters' fine centroids"}
+        res["gpu_launches"] += 2 * args.steps
     if router_ms is not None:
         gbs = router_step.nbytes / (router_ms * 1e-3) / 1e9
         res["router"] = {"ms_per_call": router_ms, "bytes_per_call": router_step.nbytes, "gbs": gbs,
