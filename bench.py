@@ -153,10 +153,22 @@ def cpu_baseline(wl, budget_s=20.0, chunk=16):
         t_oracle += time.perf_counter() - t0
         done += n
     nbytes = done * wl.L * wl.d * 2 * 2
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = oracle.threads()
+    # the same oracle on one thread, over a few KV groups
+    n1 = min(8, total_groups)
+    qs, Ks, Vs, keys, _ = _oracle_sample_range(wl, 0, n1)
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.attend(qs, Ks, Vs, keys, wl.scale)
+        t1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(cores)
     return {"value": nbytes / t_oracle / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{done} of {total_groups} KV groups of {wl.name}, full traversal, fp64 "
-                      f"oracle time {t_oracle:.2f} s"}
+                      f"oracle time {t_oracle:.2f} s",
+            "one_core": {"value": n1 * wl.L * wl.d * 2 * 2 / t1 / 1e9, "unit": "GB/s",
+                         "sample": f"{n1} KV groups, oracle time {t1:.2f} s"}}
 
 
 def _oracle_sample_range(wl, g0, n):
@@ -195,7 +207,7 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / args.steps
     nbytes = n_groups * wl.L * wl.d * 4
     v = nbytes / dt / 1e9
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = oracle.threads()
     sample = f"{n_groups} of {wl.B * wl.Hkv} KV groups of {wl.name} per step, full traversal, fp64"
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,

@@ -54,6 +54,8 @@ def lib():
         L.orc_art.argtypes = [i64, i32, i32, _p, _p, _p, i64, _p, i32, _p, _p, i64, dbl, dbl, dbl,
                               i32, i32, _p, _p, _p, _p, _p]
         L.orc_select.argtypes = [i64, i32, i32, _p, _p, i32, i32, _p, _p]
+        L.orc_max_threads.restype = i32
+        L.orc_set_threads.argtypes = [i32]
         L.orc_merge.argtypes = [i32, i64, i32, _p, _p, _p, _p]
         _LIB = L
     return _LIB
@@ -246,3 +248,13 @@ def route(q, w, bias, n_prefix, n_suffix):
     f = np.concatenate([prefix, suffix], axis=-1)  # [L][B][2F]
     z = np.einsum("lbf,lf->lb", f, np.asarray(w, dtype=np.float64)) + np.asarray(bias, dtype=np.float64)[:, None]
     return z, (z > 0).astype(np.uint8)
+
+
+def threads():
+    """OpenMP threads the oracle's loops use."""
+    return int(lib().orc_max_threads())
+
+
+def set_threads(n):
+    """Use n threads from now on (for timing the oracle on one core)."""
+    lib().orc_set_threads(int(n))

@@ -23,6 +23,27 @@
 #include <stdlib.h>
 #include <string.h>
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads the OpenMP loops below use (1 without OpenMP), and a way to change
+ * them for timing the oracle on one core.  Not part of any definition. */
+int orc_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 static double bf(uint16_t h) {
   union { float f; uint32_t u; } c;
   c.u = (uint32_t)h << 16;

@@ -525,3 +525,23 @@ def test_select2_squeezed_hierarchy_example():
     fine_names = ["A1", "A2", "B1", "B2"]
     assert [fine_names[i] for i in got[0]] == expect["expect_fine"]
     assert [names[i] for i in fine_members[got[0][0]]] == expect["expect_keys"]
+
+
+def test_oracle_threads_do_not_change_results():
+    # the OpenMP loops run over independent units: one thread or many, the
+    # results are the same bits (the CPU baseline times both)
+    n0 = oracle.threads()
+    q = bf16_bits(RNG.standard_normal((6, 4, 16)))
+    K = bf16_bits(RNG.standard_normal((6, 70, 16)))
+    V = bf16_bits(RNG.standard_normal((6, 70, 16)))
+    keys = [[np.arange(70)] * 4 for _ in range(6)]  # per unit, per query row
+    a = oracle.attend(q, K, V, keys, 0.25)
+    oracle.set_threads(1)
+    try:
+        assert oracle.threads() == 1
+        b = oracle.attend(q, K, V, keys, 0.25)
+    finally:
+        oracle.set_threads(n0)
+    assert oracle.threads() == n0
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
