@@ -176,7 +176,18 @@ SKV_API int skv_decode_launches(const skv_decode_args* args);
 
 /* Decode attention, see above.  Option combinations: at most one of
  * {order, window, seg_start/seg_end, kv range}; ART only with natural or
- * `order` traversal. */
+ * `order` traversal.
+ * Launch shapes (they follow from host-side fields only):
+ *  - long walks: persistent CTAs (2 per SM) share all tiles, then a merge
+ *    kernel combines the partial records in the workspace;
+ *  - small walks (at most 8 tiles per resident CTA) and segment lists: one
+ *    thread-block cluster of up to 16 CTAs per KV group, merged inside the
+ *    kernel through distributed shared memory (no workspace); a cluster size
+ *    the device cannot hold at once is halved;
+ *  - ART: persistent CTAs over (chunk, group) items, then the merge kernel;
+ *  - query chunks (q_tokens > 1): one tensor-core kernel.
+ * skv_decode_launches and skv_decode_workspace_size report the kernels and
+ * the scratch a call needs. */
 SKV_API skv_status attn_decode(const skv_decode_args* args, skv_stream_t stream);
 
 /* attn_decode without any allocation -- for callers that cannot allocate.
