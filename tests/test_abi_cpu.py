@@ -187,3 +187,49 @@ def test_strerror():
     assert skv.strerror(skv.SKV_OK) == "ok"
     assert "workspace" in skv.strerror(skv.SKV_EWORKSPACE)
     assert skv.strerror(99) == "unknown status"
+
+
+def test_plan_small_walks_take_the_cluster_schedule():
+    # up to 8 tiles per resident CTA (148 SMs x 2 CTAs here) the walk runs as
+    # one cluster per KV group and merges in-kernel; one tile more, and the
+    # persistent schedule with its record merge takes over
+    L = skv.lib()
+    small = 148 * 2 * 8  # tiles
+    a = good_args(batch=1, q_heads=4, kv_heads=1, max_seq_len=small * 64, max_blocks=small)
+    assert L.skv_decode_launches(ctypes.byref(a)) == 1
+    assert L.skv_decode_workspace_size(ctypes.byref(a)) == 0
+    b = good_args(batch=1, q_heads=4, kv_heads=1, max_seq_len=(small + 1) * 64, max_blocks=small + 1)
+    assert L.skv_decode_launches(ctypes.byref(b)) == 2
+    assert L.skv_decode_workspace_size(ctypes.byref(b)) > 0
+
+
+@pytest.mark.parametrize("groups_b,hkv,blocks,want_cb", [
+    (16, 8, 512, 16),    # 128 groups of 512 blocks: ~2.3 chunks of a group in flight
+    (8, 8, 2048, 32),    # 64 groups of 2048 blocks (a routed stack's full layer)
+    (64, 8, 256, 32),    # 512 groups: under one chunk in flight per group
+])
+def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
+    # The ART chunk is 32 blocks when the chunks in flight per group (CTAs /
+    # groups) span at most 1/12 of the walk, else 16.  The workspace of a
+    # chunk length CB: zeroed control words (item counter, stop chunk per
+    # group, ready flag per (group, chunk), consumed and stop per head), per
+    # (group, chunk) a look-back record (12 floats) and a partial record (132
+    # floats) per head, and per resident CTA (148 SMs x 2) probes of CB blocks
+    # x 8 warps x G heads x 12 floats and 8 warps' states of G x 132 floats,
+    # both double-buffered; each of the first two parts rounded up to 256 B.
+    L = skv.lib()
+    G, NW, ctas = 4, 8, 148 * 2
+    a = good_args(batch=groups_b, q_heads=hkv * G, kv_heads=hkv, max_seq_len=blocks * 64, max_blocks=blocks,
+                  art=_Art(1, 1e-3, 1e-4, 4))
+    n = L.skv_decode_workspace_size(ctypes.byref(a))
+    groups = groups_b * hkv
+    up = lambda x: -(-x // 256) * 256
+    sizes = {}
+    for cb in (16, 32):
+        maxc = -(-blocks // cb)
+        items = groups * maxc
+        ctl = up((4 + groups + groups * maxc + 2 * groups * G) * 4)
+        lb = up(items * G * 12 * 4)
+        scratch = ctas * (2 * cb * NW * G * 12 + 2 * NW * G * 132) * 4
+        sizes[cb] = ctl + lb + scratch + items * G * 132 * 4
+    assert n == sizes[want_cb], (n, sizes)
