@@ -20,9 +20,30 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ["attn_decode", "attn_select_centroids", "attn_merge_lse", "skv_decode_workspace_size",
+    for n in ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_select_centroids2",
+              "attn_merge_lse", "attn_route_layers", "skv_decode_workspace_size", "skv_decode_launches",
               "skv_strerror"]:
         assert n in names
+
+
+def test_header_is_plain_c_and_cxx(tmp_path):
+    # the boundary is a C ABI: the header compiles as C99 and as C++, and a C
+    # program can name every entry point
+    import shutil
+    import subprocess
+    src = tmp_path / "use.c"
+    names = declared_functions()
+    src.write_text('#include "sparsekv.h"\n' + "void* table[] = {" +
+                   ", ".join(f"(void*){n}" for n in names) + "};\nint main(void) { return 0; }\n")
+    inc = os.path.join(ROOT, "include")
+    for cc, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not found")
+        args = [cc, std, "-Wall", "-Werror", "-fsyntax-only", "-I", inc]
+        if cc == "g++":
+            args += ["-x", "c++"]
+        r = subprocess.run(args + [str(src)], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
 
 
 def test_library_exports_every_declared_symbol():
