@@ -46,6 +46,28 @@ def test_header_is_plain_c_and_cxx(tmp_path):
         assert r.returncode == 0, r.stderr
 
 
+def test_binding_struct_matches_the_header(tmp_path):
+    # the ctypes mirror of skv_decode_args has the C layout: same size and the
+    # same offset for every field (checked with the C compiler's own offsetof)
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not found")
+    fields = [f[0] for f in DecodeArgs._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "sparsekv.h"\nint main(void) {\n'
+                   '  printf("size %zu\\n", sizeof(skv_decode_args));\n' +
+                   "".join(f'  printf("{n} %zu\\n", offsetof(skv_decode_args, {n}));\n' for n in fields) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                       check=True).stdout.splitlines())
+    assert int(got["size"]) == ctypes.sizeof(DecodeArgs)
+    for n in fields:
+        assert int(got[n]) == getattr(DecodeArgs, n).offset, n
+
+
 def test_library_exports_every_declared_symbol():
     L = skv.lib()
     for n in declared_functions():
