@@ -58,6 +58,10 @@
  *    optional causal mask over the chunk's own keys, optional equal shards;
  *    no ART, order, window or segments.  Other values return SKV_EUNSUPPORTED.
  *  - Alignment: q, out, k_pool and v_pool 16-byte aligned.
+ *  - The first call of each kernel shape on a device sets that kernel's
+ *    shared-memory (and cluster) attributes and queries whether a cluster
+ *    shape fits; make that first call outside CUDA stream capture.  Later
+ *    calls, inside a capture or not, only launch.
  */
 #ifndef SPARSEKV_H
 #define SPARSEKV_H
