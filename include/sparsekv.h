@@ -178,6 +178,30 @@ SKV_API size_t skv_decode_workspace_size(const skv_decode_args* args);
  * invalid.  Depends only on host-side fields; for profiling and accounting. */
 SKV_API int skv_decode_launches(const skv_decode_args* args);
 
+/* The launch plan attn_decode would follow for these arguments (host-side
+ * fields only; nothing is launched).  For profiling, capacity planning and
+ * tests. */
+typedef enum {
+  SKV_SCHED_PERSISTENT = 0, /* persistent CTAs over all tiles, then the record merge */
+  SKV_SCHED_CLUSTER = 1,    /* one cluster of `splits` CTAs per KV group, merged in-kernel */
+  SKV_SCHED_ART = 2,        /* ART: persistent CTAs over (chunk, group) items, then the merge */
+  SKV_SCHED_CHUNK = 3       /* query chunk (q_tokens > 1) on the tensor cores */
+} skv_schedule;
+
+typedef struct {
+  int schedule;           /* skv_schedule */
+  int ctas;               /* CTAs of the main kernel (cluster schedule: before any halving of
+                             a cluster size the device cannot hold; query chunks: 0) */
+  int splits;             /* cluster schedule: CTAs per cluster (pieces per KV group); else 0 */
+  int art_chunk_blocks;   /* ART: blocks per chunk (16 or 32); else 0 */
+  int art_chunks;         /* ART: chunks per KV group (the longest walk's); else 0 */
+  int launches;           /* kernels per call, as skv_decode_launches */
+  size_t workspace_bytes; /* as skv_decode_workspace_size */
+} skv_decode_plan;
+
+/* Fill *plan; SKV_EINVAL for a NULL plan, else attn_decode's validation status. */
+SKV_API skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* plan);
+
 /* Decode attention, see above.  Option combinations: at most one of
  * {order, window, seg_start/seg_end, kv range}; ART only with natural or
  * `order` traversal.

@@ -15,7 +15,7 @@ from . import _build
 
 __all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_merge_lse",
            "attn_route_layers", "attn_select_centroids2",
-           "decode_workspace_size", "decode_launches",
+           "decode_workspace_size", "decode_launches", "decode_plan",
            "strerror", "SkvError", "lib", "DEV_BITS"]
 
 SKV_OK, SKV_EINVAL, SKV_EUNSUPPORTED, SKV_ECUDA, SKV_ETIMEOUT, SKV_EWORKSPACE = range(6)
@@ -68,6 +68,8 @@ def lib():
         L.skv_decode_workspace_size.restype = ctypes.c_size_t
         L.skv_decode_launches.argtypes = [ctypes.POINTER(DecodeArgs)]
         L.skv_decode_launches.restype = ctypes.c_int
+        L.skv_decode_plan_info.argtypes = [ctypes.POINTER(DecodeArgs), ctypes.POINTER(DecodePlan)]
+        L.skv_decode_plan_info.restype = _i
         L.attn_decode.argtypes = [ctypes.POINTER(DecodeArgs), _p]
         L.attn_decode.restype = _i
         L.attn_decode_static_ws.argtypes = [ctypes.POINTER(DecodeArgs), _p]
@@ -147,6 +149,27 @@ def make_decode_args(q, k_pool, v_pool, block_table, seq_lens, out, lse, *, max_
 def decode_workspace_size(*args, **kw):
     """Bytes of workspace attn_decode needs (same arguments as attn_decode)."""
     return lib().skv_decode_workspace_size(ctypes.byref(make_decode_args(*args, **kw)))
+
+
+class DecodePlan(ctypes.Structure):
+    """Mirror of skv_decode_plan (include/sparsekv.h)."""
+    _fields_ = [("schedule", _i), ("ctas", _i), ("splits", _i), ("art_chunk_blocks", _i),
+                ("art_chunks", _i), ("launches", _i), ("workspace_bytes", ctypes.c_size_t)]
+
+
+SCHEDULES = {0: "persistent", 1: "cluster", 2: "art", 3: "chunk"}
+
+
+def decode_plan(*args, **kw):
+    """The launch plan attn_decode would follow (see skv_decode_plan_info in
+    include/sparsekv.h) as a dict; raises SkvError for invalid arguments."""
+    p = DecodePlan()
+    st = lib().skv_decode_plan_info(ctypes.byref(make_decode_args(*args, **kw)), ctypes.byref(p))
+    if st != SKV_OK:
+        raise SkvError(st, "skv_decode_plan_info")
+    d = {f: getattr(p, f) for f, _ in DecodePlan._fields_}
+    d["schedule"] = SCHEDULES[d["schedule"]]
+    return d
 
 
 def decode_launches(*args, **kw):

@@ -180,6 +180,32 @@ int skv_decode_launches(const skv_decode_args* args) {
   return (pl.chunk || (!pl.art && pl.sched == SCHED_SPLIT)) ? 1 : 2;
 }
 
+skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* plan) {
+  if (!plan) return SKV_EINVAL;
+  *plan = skv_decode_plan{};
+  Plan pl;
+  const skv_status st = make_plan(args, &pl);
+  if (st != SKV_OK) return st;
+  plan->launches = (pl.chunk || (!pl.art && pl.sched == SCHED_SPLIT)) ? 1 : 2;
+  plan->workspace_bytes = pl.ws_bytes;
+  if (pl.chunk) {
+    plan->schedule = SKV_SCHED_CHUNK;
+  } else if (pl.art) {
+    plan->schedule = SKV_SCHED_ART;
+    plan->ctas = pl.n_ctas;
+    plan->art_chunk_blocks = pl.art_chunk;
+    plan->art_chunks = pl.art_maxc;
+  } else if (pl.sched == SCHED_PERSISTENT) {
+    plan->schedule = SKV_SCHED_PERSISTENT;
+    plan->ctas = pl.n_ctas;
+  } else {
+    plan->schedule = SKV_SCHED_CLUSTER;
+    plan->splits = pl.splits;
+    plan->ctas = pl.splits * args->kv_heads * args->batch;
+  }
+  return SKV_OK;
+}
+
 skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
   Plan pl;
   const skv_status st = make_plan(a, &pl);

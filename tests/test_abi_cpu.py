@@ -22,7 +22,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_select_centroids2",
               "attn_merge_lse", "attn_route_layers", "skv_decode_workspace_size", "skv_decode_launches",
-              "skv_strerror"]:
+              "skv_decode_plan_info", "skv_strerror"]:
         assert n in names
 
 
@@ -66,6 +66,18 @@ def test_binding_struct_matches_the_header(tmp_path):
     assert int(got["size"]) == ctypes.sizeof(DecodeArgs)
     for n in fields:
         assert int(got[n]) == getattr(DecodeArgs, n).offset, n
+    # and the plan struct
+    pf = [f[0] for f in skv.DecodePlan._fields_]
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "sparsekv.h"\nint main(void) {\n'
+                   '  printf("size %zu\\n", sizeof(skv_decode_plan));\n' +
+                   "".join(f'  printf("{n} %zu\\n", offsetof(skv_decode_plan, {n}));\n' for n in pf) +
+                   "  return 0;\n}\n")
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                       check=True).stdout.splitlines())
+    assert int(got["size"]) == ctypes.sizeof(skv.DecodePlan)
+    for n in pf:
+        assert int(got[n]) == getattr(skv.DecodePlan, n).offset, n
 
 
 def test_library_exports_every_declared_symbol():
@@ -276,3 +288,48 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
         scratch = ctas * (2 * cb * NW * G * 12 + 2 * NW * G * 132) * 4
         sizes[cb] = ctl + lb + scratch + items * G * 132 * 4
     assert n == sizes[want_cb], (n, sizes)
+
+
+def test_decode_plan_info():
+    L = skv.lib()
+
+    def plan(a):
+        p = skv.DecodePlan()
+        assert L.skv_decode_plan_info(ctypes.byref(a), ctypes.byref(p)) == skv.SKV_OK
+        return p
+
+    full = plan(good_args())  # 16 x 8 groups of 512 tiles
+    assert (full.schedule, full.ctas, full.splits, full.launches) == (0, 296, 0, 2)
+    assert full.workspace_bytes == L.skv_decode_workspace_size(ctypes.byref(good_args()))
+    art = plan(good_args(art=_Art(1, 1e-3, 1e-4, 4)))
+    assert (art.schedule, art.ctas, art.art_chunk_blocks, art.art_chunks, art.launches) == (2, 296, 16, 32, 2)
+    art5 = plan(good_args(batch=8, max_seq_len=131072, max_blocks=2048, art=_Art(1, 1e-3, 1e-4, 4)))
+    assert (art5.art_chunk_blocks, art5.art_chunks) == (32, 64)
+    small = plan(good_args(batch=1, q_heads=8, kv_heads=2, max_seq_len=4096, max_blocks=64))
+    assert (small.schedule, small.splits, small.ctas, small.launches, small.workspace_bytes) == (1, 16, 32, 1, 0)
+    seg = plan(good_args(seg_start=FAKE, seg_end=FAKE, n_seg=102))
+    assert seg.schedule == 1 and 1 <= seg.splits <= 16 and seg.ctas == seg.splits * 16 * 8
+    chunk = plan(good_args(q_tokens=128))
+    assert (chunk.schedule, chunk.launches, chunk.workspace_bytes) == (3, 1, 0)
+    p = skv.DecodePlan()
+    assert L.skv_decode_plan_info(ctypes.byref(good_args(head_dim=64)), ctypes.byref(p)) == skv.SKV_EUNSUPPORTED
+    assert L.skv_decode_plan_info(ctypes.byref(good_args()), None) == skv.SKV_EINVAL
+
+
+def test_decode_plan_from_tensors():
+    # the Python binding's view of the plan (host tensors stand in: only their
+    # shapes, addresses and alignment are read)
+    import torch
+    B, Hq, Hkv, L = 1, 8, 2, 4096
+    q = torch.zeros((B, 1, Hq, 128), dtype=torch.bfloat16)
+    pool = torch.zeros((64, Hkv, 64, 128), dtype=torch.bfloat16)
+    bt = torch.zeros((B, 64), dtype=torch.int32)
+    sl = torch.full((B,), L, dtype=torch.int32)
+    out = torch.zeros((B, 1, Hq, 128), dtype=torch.float32)
+    lse = torch.zeros((B, 1, Hq), dtype=torch.float32)
+    p = skv.decode_plan(q, pool, pool, bt, sl, out, lse, max_seq_len=L)
+    assert p["schedule"] == "cluster" and p["launches"] == 1 and p["workspace_bytes"] == 0
+    p = skv.decode_plan(q, pool, pool, bt, sl, out, lse, max_seq_len=L, art=(1e-3, 1e-4, 4))
+    assert p["schedule"] == "art" and p["art_chunk_blocks"] in (16, 32)
+    with pytest.raises(skv.SkvError):
+        skv.decode_plan(q, pool, pool, bt, sl, out, lse, max_seq_len=L, art=(-1.0, 1e-4, 4))
