@@ -26,6 +26,8 @@ import statistics
 import sys
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -41,6 +43,8 @@ def parse():
     ap.add_argument("--workload", default="cfg2_b16_h32_l32k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-art", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time the headline workload only (skip the other workloads' lines)")
     return ap.parse_args()
 
 
@@ -314,12 +318,13 @@ def build_select(torch, skv, skvgen, wl, status):
     return step
 
 
-def build_routed(torch, skv, skvgen, wl, status):
-    """32 independent attention layers; layer l runs full attention with ART
-    when its seeded route bit is 1, else the sink + recent window only, whose
-    cache holds just those blocks."""
+def build_routed(torch, skv, skvgen, wl, status, layer_ids=None):
+    """Attention layers of a routed stack (all `wl.n_layers`, or `layer_ids`),
+    each independent; layer l runs full attention with ART when its seeded
+    route bit is 1, else the sink + recent window only, whose cache holds just
+    those blocks."""
     layers = []
-    for l in range(wl.n_layers):
+    for l in (range(wl.n_layers) if layer_ids is None else layer_ids):
         fa = skvgen.route_bit(wl.seed, l) == 1
         lw = wl.with_(paging="identity" if fa else "window")
         q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, lw, layer=l)
@@ -335,8 +340,9 @@ def build_routed(torch, skv, skvgen, wl, status):
         n = skv.decode_workspace_size(q, k_pool, v_pool, bt, sl, out, lse, **kw)
         ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda") if n else None
         a = skv.make_decode_args(q, k_pool, v_pool, bt, sl, out, lse, workspace=ws, **kw)
-        layers.append(dict(fa=fa, a=a, keep=(q, k_pool, v_pool, bt, sl, out, lse, consumed, ws),
-                           consumed=consumed, launches=skv.lib().skv_decode_launches(ctypes.byref(a))))
+        layers.append(dict(layer=l, fa=fa, a=a, keep=(q, k_pool, v_pool, bt, sl, out, lse, consumed, ws),
+                           out=out, lse=lse, consumed=consumed,
+                           launches=skv.lib().skv_decode_launches(ctypes.byref(a))))
     L = skv.lib()
 
     def run():
@@ -360,9 +366,9 @@ def build_routed(torch, skv, skvgen, wl, status):
         else:
             nbytes += wl.B * wl.Hkv * win_tokens * wl.d * 4
     step = Step(run, nbytes, sum(ly["launches"] for ly in layers),
-                {"fa_layers": fa_n, "sa_layers": wl.n_layers - fa_n,
+                {"fa_layers": fa_n, "sa_layers": len(layers) - fa_n,
                  "art_blocks_skipped_frac_mean": float(np.mean(skipped)) if skipped else 0.0,
-                 "dense_equivalent_bytes": fa_bytes_full + (wl.n_layers - fa_n) * wl.kv_bytes()})
+                 "dense_equivalent_bytes": fa_bytes_full + (len(layers) - fa_n) * wl.kv_bytes()})
     step.tensors = dict(layers=layers)
     return step
 
@@ -470,9 +476,6 @@ def build_chunk(torch, skv, skvgen, wl, status):
     return step
 
 
-np = None
-
-
 def max_over_ranks(x, world, dist, device):
     """The largest of every rank's `x` (a device time in ms): the job takes as
     long as its slowest replica.  `x` itself on one rank."""
@@ -490,31 +493,63 @@ def job_gbs(nbytes_per_rank, world, ms):
     return nbytes_per_rank * world / (ms * 1e-3) / 1e9
 
 
-def main():
-    global np
-    args = parse()
-    if args.impl == "reference":
-        run_reference(args)
-        return
-    import numpy
-    np = numpy
-    import torch
-    import torch.distributed as dist
+class Ctx:
+    """What every workload's measurement shares: torch, the process group, the
+    peaks and the device status word."""
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    def __init__(self, args, torch, dist, world, rank, local):
+        import skvgen
+        import sparse_kv_b200 as skv
+        self.args, self.torch, self.dist = args, torch, dist
+        self.world, self.rank, self.local = world, rank, local
+        self.skv, self.skvgen = skv, skvgen
+        self.hbm_peak, self.peak_kind = peaks()
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
 
-    import skvgen
-    import sparse_kv_b200 as skv
-    wl = skvgen.WORKLOADS[args.workload]
-    hbm_peak, peak_kind = peaks()
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    def timed(self, st, steps, warmup):
+        """CUDA-graph replay of `steps` steps, each bracketed by events on the
+        launching stream; returns (total ms, max over ranks; per-step ms)."""
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        for _ in range(warmup):
+            st.run()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            st.run()
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        if self.world > 1:
+            self.dist.barrier()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for e0, e1 in evs:
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        total_ms = t0.elapsed_time(t1)
+        per = [e0.elapsed_time(e1) for e0, e1 in evs]
+        total_ms = max_over_ranks(total_ms, self.world, self.dist, "cuda")
+        del g
+        return total_ms, per
 
-    kind = args.workload.split("_")[0]
+
+def measure_workload(c, name, headline):
+    """Build, time and summarise one workload's step; `headline` adds the
+    end-to-end leg.  Returns the result dict (the bench line for the
+    headline)."""
+    torch, skv, skvgen, args = c.torch, c.skv, c.skvgen, c.args
+    world, status = c.world, c.status
+    wl = skvgen.WORKLOADS[name]
+    kind = name.split("_")[0]
     if kind in ("cfg1", "cfg2"):
         step = build_decode(torch, skv, skvgen, wl, status)
     elif kind == "cfg3":
@@ -524,7 +559,7 @@ def main():
     elif kind == "cfg4":
         step = build_chunk(torch, skv, skvgen, wl, status)
     else:
-        raise SystemExit(f"workload {args.workload}: no bench step")
+        raise SystemExit(f"workload {name}: no bench step")
     art_step, sweep_steps, dense_step = None, [], None
     if kind == "cfg2" and not args.no_art:
         T = step.tensors
@@ -542,51 +577,18 @@ def main():
                                   inputs=(T["q"], T["k_pool"], T["v_pool"], T["bt"], T["sl"]))
         level_steps = build_select_levels(torch, skv, skvgen, wl, step)
     stream = torch.cuda.current_stream()
+    n_side = max(10, args.steps // 4)
 
-    def timed(st, steps, warmup):
-        """CUDA-graph replay of `steps` steps, each bracketed by events."""
-        for _ in range(warmup):
-            st.run()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            st.run()
-        for _ in range(2):
-            g.replay()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(steps)]
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for e0, e1 in evs:
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        total_ms = t0.elapsed_time(t1)
-        per = [e0.elapsed_time(e1) for e0, e1 in evs]
-        total_ms = max_over_ranks(total_ms, world, dist, "cuda")
-        del g
-        return total_ms, per
-
-    uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
-    with ClockSampler(uuid) as clk:
-        total_ms, per = timed(step, args.steps, args.warmup)
+    with ClockSampler(c.uuid) as clk:
+        total_ms, per = c.timed(step, args.steps, args.warmup)
         art_ms = None
         if art_step is not None:
-            art_ms, _ = timed(art_step, args.steps, args.warmup)
-        sweep_ms = [timed(st, max(10, args.steps // 4), args.warmup)[0] / max(10, args.steps // 4)
-                    for _, st in sweep_steps]
-        dense_ms = (timed(dense_step, max(10, args.steps // 4), args.warmup)[0] / max(10, args.steps // 4)
-                    if dense_step is not None else None)
-        router_ms = (timed(router_step, args.steps, args.warmup)[0] / args.steps
+            art_ms, _ = c.timed(art_step, args.steps, args.warmup)
+        sweep_ms = [c.timed(st, n_side, args.warmup)[0] / n_side for _, st in sweep_steps]
+        dense_ms = (c.timed(dense_step, n_side, args.warmup)[0] / n_side if dense_step is not None else None)
+        router_ms = (c.timed(router_step, args.steps, args.warmup)[0] / args.steps
                      if router_step is not None else None)
-        level_ms = ([timed(st, args.steps, args.warmup)[0] / args.steps for st in level_steps]
+        level_ms = ([c.timed(st, args.steps, args.warmup)[0] / args.steps for st in level_steps]
                     if level_steps is not None else None)
     clocks = clk.summary()
     if int(status.item()) != 0:
@@ -599,7 +601,7 @@ def main():
 
     # ---- end to end through the public API: q (and tables) in from pinned host, O/LSE out
     e2e = None
-    if kind in ("cfg1", "cfg2"):
+    if headline and kind in ("cfg1", "cfg2"):
         T = step.tensors
         q_h, bt_h, sl_h = (T[k].cpu().pin_memory() for k in ("q", "bt", "sl"))
         out_h = torch.empty(T["out"].shape, dtype=torch.float32).pin_memory()
@@ -617,7 +619,7 @@ def main():
             e2e_step()
         torch.cuda.synchronize()
         if world > 1:
-            dist.barrier()
+            c.dist.barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -626,7 +628,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.steps
-        e2e_ms = max_over_ranks(e2e_ms, world, dist, "cuda")
+        e2e_ms = max_over_ranks(e2e_ms, world, c.dist, "cuda")
         h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
         d2h = out_h.numel() * 4 + lse_h.numel() * 4
         e2e = {"value": job_gbs(step.nbytes, world, e2e_ms), "unit": "GB/s",
@@ -646,8 +648,8 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": step.nbytes / (wl.d * 4) * wl.G * world / (ms_step * 1e-3),
         "kv_tokens_per_s": step.nbytes / (wl.d * 4) * world / (ms_step * 1e-3),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": c.hbm_peak, "unit": "GB/s",
+                     "frac": achieved / c.hbm_peak, "peak_kind": c.peak_kind,
                      "frac_of_8000": achieved / 8000.0, "traffic": traffic_for(kind),
                      "kernel": "one step of our kernels (decode + merge; per-kernel shares in profiles/)"},
         "clocks": clocks,
@@ -690,12 +692,12 @@ def main():
                     "group_blocks_hist16": np.histogram(grp, bins=16, range=(0, wl.nb(0)))[0].tolist()}
         res["art_sweep"] = [dict(tau=thr[0], phi=thr[1], patience=thr[2], **art_summary(st, ms))
                             for (thr, st), ms in zip(sweep_steps, sweep_ms)]
-        res["gpu_launches"] += sum(max(10, args.steps // 4) * st.launches for _, st in sweep_steps)
+        res["gpu_launches"] += sum(n_side * st.launches for _, st in sweep_steps)
     if dense_ms is not None:
         res["selection"] = {"dense_ms_per_step": dense_ms, "time_vs_dense": ms_step / dense_ms,
                             "bytes_vs_dense": step.nbytes / wl.kv_bytes(),
                             "note": "same cache walked in full by the plain decode kernel"}
-        res["gpu_launches"] += max(10, args.steps // 4) * dense_step.launches
+        res["gpu_launches"] += n_side * dense_step.launches
     if level_ms is not None:
         f, t = level_steps
         res["selection_levels"] = {
@@ -707,16 +709,139 @@ def main():
     if router_ms is not None:
         gbs = router_step.nbytes / (router_ms * 1e-3) / 1e9
         res["router"] = {"ms_per_call": router_ms, "bytes_per_call": router_step.nbytes, "gbs": gbs,
-                         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                                      "frac": gbs / hbm_peak},
+                         "roofline": {"bound": "hbm", "achieved": gbs, "peak": c.hbm_peak, "unit": "GB/s",
+                                      "frac": gbs / c.hbm_peak},
                          **router_step.extra,
                          "note": "per-layer route bits from pooled prefix/suffix query rows "
                                  "(untrained weights); outside the timed decode step"}
         res["gpu_launches"] += args.steps * router_step.launches
     if e2e is not None:
         res["e2e"] = e2e
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and kind in ("cfg1", "cfg2"):
-        res["cpu_baseline"] = cpu_baseline(wl)
+    # ---- CPU-baseline leg (rank 0, one GPU): the oracle timed on the host cores, and
+    # the same oracle's check of sampled KV groups of what the GPU returned above
+    if c.rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if headline and kind in ("cfg1", "cfg2"):
+            res["cpu_baseline"] = cpu_baseline(wl)
+        checks = {}
+        if kind in ("cfg1", "cfg2"):
+            checks["full"] = oracle_check_full(wl, step)
+        if art_step is not None:
+            checks["art"] = oracle_check_art(wl, art_step, (wl.tau, wl.phi, wl.patience))
+            checks["art_sweep"] = [oracle_check_art(wl, st, thr) for thr, st in sweep_steps]
+        if kind == "cfg5":
+            fa = [ly for ly in step.tensors["layers"] if ly["fa"]]
+            if fa:
+                checks["art_layer"] = oracle_check_art(wl, fa[0], (wl.tau, wl.phi, wl.patience),
+                                                       layer=fa[0]["layer"], n_groups=2)
+        if checks:
+            res["oracle_check"] = checks
+    del step, art_step, sweep_steps, dense_step, router_step, level_steps
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def _sample_groups(wl, n):
+    """n KV groups spread over the batch and the KV heads."""
+    step = max(1, (wl.B * wl.Hkv) // n)
+    gs = list(range(0, wl.B * wl.Hkv, step))[:n]
+    return [(g // wl.Hkv, (g // wl.Hkv + g) % wl.Hkv) for g in gs]
+
+
+def oracle_check_full(wl, st, n_groups=4):
+    """Full traversal: max |dO| and relative |dlse| of sampled KV groups against
+    the oracle (CPU-baseline leg)."""
+    import oracle
+    import skvgen
+    T = st.tensors
+    out = T["out"][:, 0].cpu().numpy().astype(np.float64)
+    lse = T["lse"][:, 0].cpu().numpy().astype(np.float64)
+    q = skvgen.host_q(wl)
+    err, lerr = 0.0, 0.0
+    groups = _sample_groups(wl, n_groups)
+    for b, kvh in groups:
+        K, V = skvgen.host_kv_group(wl, b, kvh, q=q)
+        qg = q[b, 0, kvh * wl.G:(kvh + 1) * wl.G]
+        O, l = oracle.attend(qg[None], K[None], V[None], [[np.arange(wl.seq_len(b))] * wl.G], wl.scale)
+        hs = slice(kvh * wl.G, (kvh + 1) * wl.G)
+        err = max(err, float(np.abs(out[b, hs] - O[0]).max()))
+        lerr = max(lerr, float((np.abs(lse[b, hs] - l[0]) / np.maximum(1.0, np.abs(l[0]))).max()))
+    return {"groups": groups, "max_abs_dO": err, "max_rel_dlse": lerr, "tol_O": 2e-3, "tol_lse": 1e-4}
+
+
+def oracle_check_art(wl, st, thr, layer=0, n_groups=8, flag_margin=1e-3):
+    """ART decisions of sampled KV groups against the sequential fp64 oracle
+    (CPU-baseline leg).  A head whose blocks consumed differ from the oracle's is
+    "flagged" when the oracle's decision margin (relative distance of d_scale
+    or d_dir to its threshold) is within flag_margin, else "mismatched"; its
+    output is compared with the oracle forced to the GPU's stop."""
+    import oracle
+    import skvgen
+    tau, phi, pat = thr
+    T = st.tensors if hasattr(st, "tensors") else st
+    out = T["out"][:, 0].cpu().numpy().astype(np.float64)
+    lse = T["lse"][:, 0].cpu().numpy().astype(np.float64)
+    cons = T["consumed"].cpu().numpy()
+    q = skvgen.host_q(wl, layer)
+    flagged = mismatched = stop_diff = 0
+    err, lerr = 0.0, 0.0
+    groups = _sample_groups(wl, n_groups)
+    for b, kvh in groups:
+        K, V = skvgen.host_kv_group(wl, b, kvh, layer, q=q)
+        qg = q[b, 0, kvh * wl.G:(kvh + 1) * wl.G]
+        trav = [oracle.art_traversal(wl.nb(b))]
+        O, l, c_ref, mg = oracle.art(qg[None], K[None], V[None], [wl.seq_len(b)], wl.bs, trav, wl.scale,
+                                     tau, phi, pat)
+        hs = slice(kvh * wl.G, (kvh + 1) * wl.G)
+        cg = cons[b, hs]
+        diff = np.nonzero(cg != c_ref[0])[0]
+        for h in diff:
+            if mg[0, h] <= flag_margin:
+                flagged += 1
+            else:
+                mismatched += 1
+        if len(diff):
+            stop_diff = max(stop_diff, int(np.abs(cg - c_ref[0]).max()))
+            O, l, _, _ = oracle.art(qg[None], K[None], V[None], [wl.seq_len(b)], wl.bs, trav, wl.scale,
+                                    tau, phi, pat, forced=cg[None])
+        err = max(err, float(np.abs(out[b, hs] - O[0]).max()))
+        lerr = max(lerr, float((np.abs(lse[b, hs] - l[0]) / np.maximum(1.0, np.abs(l[0]))).max()))
+    return {"tau": tau, "phi": phi, "patience": pat, "layer": layer, "groups": len(groups),
+            "heads": len(groups) * wl.G, "flagged_near_threshold": flagged, "mismatched": mismatched,
+            "max_stop_diff_blocks": stop_diff, "max_abs_dO": err, "max_rel_dlse": lerr,
+            "flag_margin": flag_margin}
+
+
+# the other workloads measured in the default run, after the headline
+SIDE_WORKLOADS = ["cfg1_b1_h8_l4k", "cfg3_b8_h32_l64k_c1024_k102", "cfg4_b4_h32_l128k_chunk128",
+                  "cfg5_b8_h32_l128k_32layers"]
+SIDE_KEYS = ["value", "unit", "ms_per_step", "step_ms_p10_p50_p90", "roofline", "clocks", "config",
+             "gpu_launches", "step_detail", "metric_tflops", "selection", "selection_levels", "router",
+             "oracle_check", "attended_tokens_per_s"]
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    c = Ctx(args, torch, dist, world, rank, local)
+    res = measure_workload(c, args.workload, headline=True)
+    if args.workload == "cfg2_b16_h32_l32k" and not args.headline_only:
+        res["configs"] = {}
+        for name in SIDE_WORKLOADS:
+            r = measure_workload(c, name, headline=False)
+            res["configs"][name] = {k: r[k] for k in SIDE_KEYS if k in r}
+            res["gpu_launches_side"] = res.get("gpu_launches_side", 0) + r["gpu_launches"]
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -86,7 +86,7 @@ typedef enum {
   SKV_EINVAL = 1,       /* a bad argument (NULL pointer, size, alignment, threshold) */
   SKV_EUNSUPPORTED = 2, /* valid but not implemented (shape, option combination) */
   SKV_ECUDA = 3,        /* a CUDA runtime call failed (launch, attribute) */
-  SKV_ETIMEOUT = 4,     /* reserved for callers mapping SKV_DEV_TIMEOUT */
+  SKV_ETIMEOUT = 4,     /* a bounded wait inside a kernel expired (skv_status_of_word) */
   SKV_EWORKSPACE = 5    /* workspace NULL or smaller than *_workspace_size */
 } skv_status;
 
@@ -322,6 +322,25 @@ SKV_API skv_status attn_merge_lse(const float* o_parts, const float* lse_parts, 
 SKV_API skv_status attn_route_layers(const void* q, const float* w, const float* bias, int n_layers,
                              int batch, int tokens, int q_heads, int head_dim, int n_prefix,
                              int n_suffix, float* logits, uint8_t* route, skv_stream_t stream);
+
+/* The status a device status word stands for, once the caller has read it
+ * back after synchronising: SKV_ETIMEOUT if SKV_DEV_TIMEOUT is set (a bounded
+ * wait expired; the affected outputs are not valid), else SKV_EINVAL if any
+ * bad-input bit is set (SKV_DEV_BAD_*; the bad entries were skipped), else
+ * SKV_OK.  Host-only; no CUDA call. */
+SKV_API skv_status skv_status_of_word(uint32_t status_word);
+
+/* Test hook for failure detection, not for production use.  The NEXT
+ * attn_decode call that runs the plain decode kernel (no ART, q_tokens == 1)
+ * makes the producer warp of CTA `cta` (linear block index) stop before ring
+ * entry `entry` (0-based): that entry and everything after it in the CTA are
+ * never issued, so the CTA's consumers wait for it until their bounded wait
+ * (1 s) expires, set SKV_DEV_TIMEOUT in *status_word, drain the copies in
+ * flight and return; the call's outputs are then not valid.  Nothing faults
+ * and nothing hangs.  One-shot (the call that takes it clears it); a CTA or
+ * entry the launch does not reach leaves the launch unaffected.  cta < 0
+ * clears a pending hook; SKV_EINVAL for cta >= 0 and entry < 0. */
+SKV_API skv_status skv_test_withhold_tile(int cta, int entry);
 
 /* Static description of a status code. */
 SKV_API const char* skv_strerror(skv_status s);

@@ -16,7 +16,7 @@ from . import _build
 __all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_merge_lse",
            "attn_route_layers", "attn_select_centroids2",
            "decode_workspace_size", "decode_launches", "decode_plan",
-           "strerror", "SkvError", "lib", "DEV_BITS"]
+           "strerror", "status_of_word", "SkvError", "lib", "DEV_BITS"]
 
 SKV_OK, SKV_EINVAL, SKV_EUNSUPPORTED, SKV_ECUDA, SKV_ETIMEOUT, SKV_EWORKSPACE = range(6)
 DEV_BITS = {"timeout": 0x1, "bad_page": 0x2, "bad_seqlen": 0x4, "bad_order": 0x8, "bad_segment": 0x10}
@@ -82,6 +82,10 @@ def lib():
         L.attn_route_layers.restype = _i
         L.attn_select_centroids2.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p]
         L.attn_select_centroids2.restype = _i
+        L.skv_status_of_word.argtypes = [ctypes.c_uint32]
+        L.skv_status_of_word.restype = _i
+        L.skv_test_withhold_tile.argtypes = [_i, _i]
+        L.skv_test_withhold_tile.restype = _i
         L.skv_strerror.argtypes = [_i]
         L.skv_strerror.restype = ctypes.c_char_p
         _LIB = L
@@ -90,6 +94,19 @@ def lib():
 
 def strerror(status):
     return lib().skv_strerror(int(status)).decode()
+
+
+def status_of_word(word):
+    """The skv_status a device status word stands for (see skv_status_of_word)."""
+    return lib().skv_status_of_word(int(word) & 0xFFFFFFFF)
+
+
+def test_withhold_tile(cta, entry):
+    """Test hook: the next plain decode launch's CTA `cta` withholds ring entry
+    `entry`, so its bounded wait expires (see skv_test_withhold_tile)."""
+    st = lib().skv_test_withhold_tile(int(cta), int(entry))
+    if st != SKV_OK:
+        raise SkvError(st, "skv_test_withhold_tile")
 
 
 def _ptr(t):

@@ -3,6 +3,7 @@
 // exit crosses this boundary; every path returns an skv_status.
 #include <math.h>
 #include <algorithm>
+#include <atomic>
 #include <stdint.h>
 
 #include <cuda_runtime.h>
@@ -33,6 +34,9 @@ struct Plan {
   size_t ws_bytes = 0;
   int art_chunk = 0, art_maxc = 0, art_ahead = 0;
 };
+
+// Pending test hook of skv_test_withhold_tile: (cta << 32) | entry, 0 = none.
+std::atomic<unsigned long long> g_withhold{0};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -267,6 +271,11 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
   } else {
     p.ws_hdr = reinterpret_cast<int*>(ws);
     p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes);
+    const unsigned long long wh = g_withhold.exchange(0ull);
+    if (wh != 0ull) {
+      p.withhold_cta = (int)(wh >> 32);
+      p.withhold_entry = (int)(wh & 0xFFFFFFFFull);
+    }
     if (launch_decode(p, pl.G, s) != 0) return SKV_ECUDA;
     if (pl.sched == SCHED_SPLIT) return SKV_OK;  // merged inside the kernel
   }
@@ -299,6 +308,23 @@ skv_status attn_merge_lse(const float* o_parts, const float* lse_parts, int n_pa
   if (launch_merge(o_parts, lse_parts, n_parts, n_rows, head_dim, out, lse,
                    reinterpret_cast<cudaStream_t>(stream)) != 0)
     return SKV_ECUDA;
+  return SKV_OK;
+}
+
+skv_status skv_test_withhold_tile(int cta, int entry) {
+  if (cta < 0) {  // clear a pending hook
+    g_withhold.store(0ull);
+    return SKV_OK;
+  }
+  if (entry < 0 || entry > 0x7FFFFFFE) return SKV_EINVAL;
+  g_withhold.store(((unsigned long long)(unsigned)cta << 32) | (unsigned long long)(entry + 1));
+  return SKV_OK;
+}
+
+skv_status skv_status_of_word(uint32_t word) {
+  if (word & SKV_DEV_TIMEOUT) return SKV_ETIMEOUT;
+  if (word & (SKV_DEV_BAD_PAGE | SKV_DEV_BAD_SEQLEN | SKV_DEV_BAD_ORDER | SKV_DEV_BAD_SEGMENT))
+    return SKV_EINVAL;
   return SKV_OK;
 }
 

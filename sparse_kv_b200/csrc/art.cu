@@ -1,5 +1,5 @@
-// art.cu -- decode attention with run-time termination ("ART: Adaptive
-// Run-time Termination" 2.2-2.4) for sm_100a.
+// art.cu -- decode attention with run-time termination ("ART (Attention
+// Run-time Termination)" 2.2-2.4) for sm_100a.
 //
 // Traversal of a KV group: position 0 is block 0 (the attention sink, always
 // consumed), then the caller's block list without block 0, or every other
@@ -950,7 +950,7 @@ int launch_art_t(const DecodeParams& p, cudaStream_t st) {
   static_assert(C::TOTAL <= (MINB == 2 ? 113 : 227) * 1024, "shared memory budget");
   static_assert(ST >= 3, "a ring of at least three stages");
   auto kern = art_kernel<G, NW, CB, ST, MINB>;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // per device; racing first calls only repeat the set-up
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
   if (!attr_set[dev]) {

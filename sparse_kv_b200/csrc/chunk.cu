@@ -27,12 +27,14 @@
 //               S row with tcgen05.ld, masks, keeps its running max, rescales
 //               its accumulator O_h in TMEM only when the max grows by more than
 //               2^8 (the scale is applied consistently to O_h and l_h, so the
-//               result stays exact), and writes P_h as bf16 pairs with
-//               tcgen05.st.  The two halves meet once, at the end, to combine
-//               (m, l, O) of the row exactly.
+//               result stays exact), and writes P_h with tcgen05.st as two bf16
+//               terms (hi + lo, about 16 significant bits together), each over
+//               32 of the half's 64 S columns.  The two halves meet once, at the
+//               end, to combine (m, l, O) of the row exactly.
 // Operands: Q and K K-major, V MN-major, in the canonical 128B-swizzle layout
 // (8-row x 128-byte atoms, 1024-byte aligned) in shared memory; P in TMEM
-// (row = lane, two bf16 keys per 32-bit column); bf16 x bf16 -> fp32.
+// (row = lane, two bf16 keys per 32-bit column, hi and lo terms); bf16 x bf16
+// -> fp32.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -387,12 +389,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         const uint32_t pj = tmem + (uint32_t)(j & 1) * BN;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
-          // A = P_h rows x 16 keys (TMEM, 8 columns of the half's S columns);
-          // B = V 16 keys x 128 dims (MN-major); D = O_h
+          // A = P_h rows x 16 keys (TMEM, 8 columns of the half's S columns: the hi
+          // terms, then the lo terms 32 columns on); B = V 16 keys x 128 dims
+          // (MN-major); D = O_h
           const int h = ks >> 2, kk = ks & 3;
           const uint32_t b_off = ks * 16 * 128;
-          mma_bf16_ts(tmem + kColO + h * BM, pj + h * (BN / 2) + kk * 8,
-                      smem_desc(v_addr + b_off, kHalf, 1024), idesc_pv, j > 0 || kk > 0);
+          const uint64_t dv = smem_desc(v_addr + b_off, kHalf, 1024);
+          mma_bf16_ts(tmem + kColO + h * BM, pj + h * (BN / 2) + kk * 8, dv, idesc_pv, j > 0 || kk > 0);
+          mma_bf16_ts(tmem + kColO + h * BM, pj + h * (BN / 2) + BN / 4 + kk * 8, dv, idesc_pv, true);
         }
         mma_commit(&o_done[j & 1]);
         mma_commit(&v_empty[j & 1]);
@@ -472,14 +476,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         m_used = tmax;
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      // P_h = 2^(s * scale - m_h) as bf16 pairs over the first 32 of this half's S
-      // columns (already read); packed fp32x2 for the exponent argument and for
-      // l, which sums the unrounded values
+      // P_h = 2^(s * scale - m_h), split into two bf16 terms P_h = hi + lo
+      // (hi = bf16(p), lo = bf16(p - hi)): hi as bf16 pairs over the first 32 of
+      // this half's S columns, lo over the other 32 (all already read).  P.V runs
+      // on both, so the weights enter the product with a relative error of about
+      // 2^-16 instead of bf16's 2^-8.  Packed fp32x2 for the exponent argument
+      // and for l, which sums the unrounded values.
       const f2 sc2 = pack2(p.qscale, p.qscale), nm2 = pack2(-mu, -mu);
       f2 ls2[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) ls2[u] = pack2(0.f, 0.f);
-      uint32_t pw[HC / 2];
+      uint32_t pw[HC / 2], pl[HC / 2];
 #pragma unroll
       for (int c8 = 0; c8 < HC / 8; ++c8) {
 #pragma unroll
@@ -492,10 +499,18 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           const f2 pp = pack2(p0, p1);
           ls2[u] = fadd2(ls2[u], pp);
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);  // p0 in the low half
-          pw[c8 * 4 + u] = *reinterpret_cast<const uint32_t*>(&h2);
+          const uint32_t hw = *reinterpret_cast<const uint32_t*>(&h2);
+          pw[c8 * 4 + u] = hw;
+          f2 rem = pp;
+          ffma2(rem, bf2_to_f2(hw), pack2(-1.f, -1.f));  // p - hi, exact in fp32
+          float r0, r1;
+          unpack2(rem, r0, r1);
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(r0, r1);
+          pl[c8 * 4 + u] = *reinterpret_cast<const uint32_t*>(&l2);
         }
       }
       tmem_st32u(tmem + lane_base + col_s, pw);
+      tmem_st32u(tmem + lane_base + col_s + HC / 2, pl);
       tmem_wait_st();
       {
         const f2 t2 = fadd2(fadd2(ls2[0], ls2[1]), fadd2(ls2[2], ls2[3]));
@@ -651,7 +666,7 @@ int launch_chunk(const DecodeParams& dp, int Tq, int causal, int n_shards, void*
   p.n_shards = n_shards < 1 ? 1 : n_shards;
   p.m_tiles = (Tq * p.G + BM - 1) / BM;
   p.qscale = dp.qscale;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // per device; racing first calls only repeat the set-up
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
   if (!attr_set[dev]) {

@@ -338,9 +338,13 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     const size_t head_stride = (size_t)kBlock * kHeadDim;
     int e = 0, ps = 0, round = 0;  // entries issued, stage, ring round
     bool aborted = false;
+    // test hook: this CTA stops issuing before entry `withhold` (-1: never)
+    const int cta = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    const int withhold = (p.withhold_entry > 0 && cta == p.withhold_cta) ? p.withhold_entry - 1 : -1;
     // Issue one ring entry: `n` rows of group `g` (n = 0: a group marker with
     // no rows, n = -1: end of traversal).  Returns false to stop issuing.
     auto emit = [&](int n, int g, int slot, int kvh, int t0, int pg1, int pg2, int n1) -> bool {
+      if (e == withhold) return false;  // nothing issued: the consumers' wait expires
       if (round >= 1) {
         const uint32_t par = (round - 1) & 1;
         uint64_t t_start = 0;
@@ -386,6 +390,7 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     constexpr int kMaxPieces = 8;
     auto emit_packed = [&](int n, const int* pg, const int* r0, const int* cnt, int np, int g,
                            int slot, int kvh) -> bool {
+      if (e == withhold) return false;
       if (round >= 1) {
         const uint32_t par = (round - 1) & 1;
         uint64_t t_start = 0;
@@ -766,7 +771,7 @@ int launch_t(const DecodeParams& p, cudaStream_t st) {
   using C = Cfg<G, NW, MINB>;
   auto kern = decode_kernel<G, NW, MINB>;
   // Set the shared-memory attribute once per device (not inside a capture).
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // per device; racing first calls only repeat the set-up
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
@@ -784,7 +789,7 @@ int launch_t(const DecodeParams& p, cudaStream_t st) {
   // only divides each group's walk (no workspace depends on it), so a cluster
   // shape that cannot be resident at once is halved until it can.
   if (p.n_splits < 1 || p.n_splits > kMaxClusterSplits) return (int)cudaErrorInvalidValue;
-  static bool np_set[64] = {};
+  static std::atomic<bool> np_set[64];
   if (!np_set[dev]) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (err != cudaSuccess) return (int)err;
@@ -801,7 +806,7 @@ int launch_t(const DecodeParams& p, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  static int fits[64][kMaxClusterSplits + 1] = {};  // 1: resident at once, -1: not (per size)
+  static std::atomic<int> fits[64][kMaxClusterSplits + 1];  // 1: resident at once, -1: not (per size)
   while (true) {
     cfg.gridDim = dim3(q.n_splits, q.Hkv, q.B);
     attr[0].val.clusterDim.x = q.n_splits;
@@ -849,17 +854,18 @@ int launch_decode(const DecodeParams& p, int G, void* stream) {
   }
 }
 
+// SM count of the current device (cached per device index; 148, a B200's,
+// when no device can be queried, so that host-side planning works anywhere).
 int num_sms() {
-  static int cached = 0;
-  if (cached == 0) {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-      cached = n;
-    else
-      return 148;
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = cached[dev].load();
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    cached[dev].store(n);
   }
-  return cached;
+  return n;
 }
 
 }  // namespace skv

@@ -66,6 +66,10 @@ struct DecodeParams {
   int* art_ctl;
   float* art_lb;
   float* art_scratch;  // per-CTA probe slots and state area (stays in L2)
+  // Test hook (skv_test_withhold_tile): when withhold_entry > 0, the producer of
+  // CTA withhold_cta (linear block index) stops before ring entry
+  // withhold_entry - 1, so that the consumers' bounded wait for it expires.
+  int withhold_cta, withhold_entry;
 };
 
 // ART traversal positions of a sequence of L tokens: block 0, then the

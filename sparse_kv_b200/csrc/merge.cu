@@ -233,7 +233,7 @@ int launch_merge_records(const DecodeParams& p, int G, void* stream) {
   const int max_slots = (p.sched == SCHED_PERSISTENT) ? p.n_ctas : p.art_maxc;
   const size_t smem = (size_t)max_slots * p.rec_nw * sizeof(float);
   if (smem > 200 * 1024) return (int)cudaErrorInvalidConfiguration;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // per device; racing first calls only repeat the set-up
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
   if (!attr_set[dev]) {

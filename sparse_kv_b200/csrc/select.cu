@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int* ids, int* ss, int* se, void* stream) {
   const size_t smem = kSelSmem;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // per device; racing first calls only repeat the set-up
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
   if (!attr_set[dev]) {

@@ -253,7 +253,7 @@ SKV_API skv_status attn_select_centroids2(const void* q, const void* coarse, con
   if (n_coarse > kS2MaxCoarse || n_fine > kS2MaxFine) return SKV_EUNSUPPORTED;
   if (!aligned16(coarse) || !aligned16(fine)) return SKV_EINVAL;
   const size_t smem = sizeof(S2Smem);
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // per device; racing first calls only repeat the set-up
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SKV_ECUDA;
   if (!attr_set[dev]) {

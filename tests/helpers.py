@@ -131,8 +131,30 @@ def check_art(wl, dev_res, b, kvh, order=None, layer=0, q=None, tau=None, phi=No
     return flagged, cons[0], mg[0]
 
 
+def check_topk_valid(ids_gpu, scores, k, what=""):
+    """ids_gpu (k ids) is a valid top-k of `scores` (fp64, ranked by score desc,
+    index asc) up to near ties at the boundary: k distinct ids in ascending
+    order; every id whose score lies clearly above the k-th best score is kept;
+    every kept id scores at least the k-th best score, both within the flag
+    gap TOPK_FLAG_GAP (relative to the k-th score)."""
+    s = np.asarray(scores, dtype=np.float64)
+    ids = np.asarray(ids_gpu, dtype=np.int64)
+    assert ids.shape == (k,), f"{what}: {ids.shape} ids, expected {k}"
+    assert np.all(np.diff(ids) > 0), f"{what}: ids not strictly ascending"
+    assert ids.min() >= 0 and ids.max() < s.shape[0], f"{what}: id out of range"
+    order = sorted(range(s.shape[0]), key=lambda i: (-s[i], i))
+    kth = s[order[k - 1]]
+    band = TOPK_FLAG_GAP * max(abs(kth), 1e-300)
+    must = {i for i in range(s.shape[0]) if s[i] > kth + band}
+    kept = set(int(i) for i in ids)
+    assert must <= kept, f"{what}: ids {sorted(must - kept)[:4]} score above the boundary but were dropped"
+    low = [i for i in kept if s[i] < kth - band]
+    assert not low, f"{what}: ids {low[:4]} score below the k-th best but were kept"
+
+
 def check_selection(wl, ids_gpu, groups, q=None):
-    """ids must equal the oracle's except at flagged near-tie boundaries."""
+    """ids must equal the oracle's except at flagged near-tie boundaries, where
+    the GPU's choice must still be a valid top-k (check_topk_valid)."""
     q = skvgen.host_q(wl) if q is None else q
     flagged = 0
     for (b, kvh) in groups:
@@ -142,6 +164,6 @@ def check_selection(wl, ids_gpu, groups, q=None):
         if not np.array_equal(ids[0], ids_gpu[b, kvh]):
             gap = oracle.topk_boundary_gap(sc, wl.topk)[0]
             assert gap <= TOPK_FLAG_GAP, f"selection differs for ({b},{kvh}), gap {gap:.2e}"
-            # the GPU's choice must still be a valid top-k up to the near tie
+            check_topk_valid(ids_gpu[b, kvh], sc[0], wl.topk, f"selection ({b},{kvh})")
             flagged += 1
     return flagged

@@ -333,3 +333,23 @@ def test_decode_plan_from_tensors():
     assert p["schedule"] == "art" and p["art_chunk_blocks"] in (16, 32)
     with pytest.raises(skv.SkvError):
         skv.decode_plan(q, pool, pool, bt, sl, out, lse, max_seq_len=L, art=(-1.0, 1e-4, 4))
+
+
+def test_status_of_word_maps_device_bits():
+    import sparse_kv_b200 as skv
+    B = skv.DEV_BITS
+    assert skv.status_of_word(0) == skv.SKV_OK
+    assert skv.status_of_word(B["timeout"]) == skv.SKV_ETIMEOUT
+    for k in ("bad_page", "bad_seqlen", "bad_order", "bad_segment"):
+        assert skv.status_of_word(B[k]) == skv.SKV_EINVAL
+    # a timeout outranks bad-input bits: the outputs are not valid at all
+    assert skv.status_of_word(B["timeout"] | B["bad_page"]) == skv.SKV_ETIMEOUT
+    assert skv.strerror(skv.SKV_ETIMEOUT) == "device wait timed out"
+
+
+def test_withhold_hook_validates_and_clears():
+    import sparse_kv_b200 as skv
+    L = skv.lib()
+    assert L.skv_test_withhold_tile(0, -1) == skv.SKV_EINVAL
+    assert L.skv_test_withhold_tile(3, 2) == skv.SKV_OK
+    assert L.skv_test_withhold_tile(-1, 0) == skv.SKV_OK  # clears the pending hook

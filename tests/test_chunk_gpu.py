@@ -1,17 +1,18 @@
 """Query-chunk attention on the tensor cores (q_tokens > 1) against the oracle.
 
-Partials carry P in bf16 into the P.V product (fp32 accumulation), so a
-partial's output may differ from exact attention by at most 2^-9 max|v| (each
-weight's relative rounding error) on top of the usual 2e-3; the log-sum-exp
-uses the unrounded weights.  Merged results, which is what the method
-returns, are held to the usual 2e-3.
+Every partial (one shard, or the chunk's own keys under the causal mask) and
+every merged result is held to the same tolerances as decode: max |dO| <= 2e-3
+and |dlse| <= 1e-4 * max(1, |lse|).  The kernel carries P into the P.V product
+as two bf16 terms (hi + lo), so the weights keep about 16 significant bits; a
+single bf16 term would miss 2e-3 on partials dominated by a few keys (the first
+tokens of the causal chunk, peaky logits).
 """
 import numpy as np
 import pytest
 
 import oracle
 import skvgen
-from helpers import ATOL_O, RTOL_LSE, check_close, device_workload, outputs
+from helpers import check_close, device_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -47,15 +48,9 @@ def oracle_rows(wl, b, key_fn, q=None):
     return O, lse
 
 
-def check_partial(got_o, got_l, O, lse, vmax, what):
-    tol = ATOL_O + 2.0 ** -9 * vmax
-    both = np.isneginf(lse) & np.isneginf(got_l)
-    assert np.all(np.isfinite(got_o)), what
-    err = np.abs(got_o - O).max()
-    assert err <= tol, f"{what}: max |dO| {err:.3e} > {tol:.3e}"
-    with np.errstate(invalid="ignore"):
-        ok = both | (np.abs(got_l - lse) <= RTOL_LSE * np.maximum(1.0, np.abs(lse)))
-    assert np.all(ok), f"{what}: lse"
+def check_partial(got_o, got_l, O, lse, what):
+    """A partial against exact attention over its key set (decode tolerances)."""
+    return check_close(got_o, got_l, O, lse, what)
 
 
 @pytest.mark.parametrize("G,Tq", [(4, 32), (4, 40), (2, 64), (8, 16)])
@@ -68,7 +63,7 @@ def test_chunk_whole_sequence(G, Tq):
     q = skvgen.host_q(wl)
     for b in range(2):
         O, l = oracle_rows(wl, b, lambda t: oracle.keys_full(wl.seq_len(b)), q)
-        check_partial(out[0, b].cpu().numpy(), lse[0, b].cpu().numpy(), O, l, 6.0, f"seq {b}")
+        check_partial(out[0, b].cpu().numpy(), lse[0, b].cpu().numpy(), O, l, f"seq {b}")
 
 
 def test_chunk_causal_tail_and_shards_merge_exactly():
@@ -88,11 +83,11 @@ def test_chunk_causal_tail_and_shards_merge_exactly():
         a, e = s * ctx // S, (s + 1) * ctx // S
         for b in range(2):
             O, l = oracle_rows(wl, b, lambda t: np.arange(a, e), q)
-            check_partial(parts_o[s, b].cpu().numpy(), parts_l[s, b].cpu().numpy(), O, l, 6.0,
+            check_partial(parts_o[s, b].cpu().numpy(), parts_l[s, b].cpu().numpy(), O, l,
                           f"shard {s} seq {b}")
     for b in range(2):
         O, l = oracle_rows(wl, b, lambda t: np.arange(ctx, ctx + t + 1), q)
-        check_partial(parts_o[S, b].cpu().numpy(), parts_l[S, b].cpu().numpy(), O, l, 6.0,
+        check_partial(parts_o[S, b].cpu().numpy(), parts_l[S, b].cpu().numpy(), O, l,
                       f"causal chunk seq {b}")
     # merged = unsharded causal attention over context + chunk ("Pulsar Attention" Phase 2)
     N = wl.B * Tq * wl.Hq
@@ -135,3 +130,31 @@ def test_chunk_full_size_sampled():
             O, l = oracle.attend(qg, K[None], V[None], [[oracle.keys_chunk(ctx, t)] * wl.G], wl.scale)
             hs = slice(kvh * wl.G, (kvh + 1) * wl.G)
             check_close(mo[b, t, hs], ml[b, t, hs], O[0], l[0], f"cfg4 b{b} t{t} kvh{kvh}")
+
+
+@pytest.mark.parametrize("scale", [0.35, 1.0])
+def test_chunk_peaky_partials(scale):
+    """Sink + heavy-token keys and a large softmax scale: a few keys carry most of
+    every row's weight, the case where rounding the weights hurts most.  Each
+    shard's partial and the causal chunk partial are held to 2e-3."""
+    Tq, ctx, S = 48, 1500, 2
+    wl = skvgen.Workload("cpk", B=2, Hq=8, Hkv=2, L=ctx + Tq, Tq=Tq, paging="perm", structured=True,
+                         softmax_scale=scale, seed=340 + int(scale * 100))
+    dev = device_workload(wl)
+    q = skvgen.host_q(wl)
+    import torch
+    parts_o = torch.full((S + 1, wl.B, Tq, wl.Hq, wl.d), float("nan"), device="cuda")
+    parts_l = torch.full((S + 1, wl.B, Tq, wl.Hq), float("nan"), device="cuda")
+    chunk_call(wl, dev, S, kv_range=(0, ctx), shards=S, out=parts_o[:S], lse=parts_l[:S])
+    chunk_call(wl, dev, 1, kv_range=(ctx, ctx + Tq), causal=True, out=parts_o[S:], lse=parts_l[S:])
+    worst = 0.0
+    for b in range(2):
+        for s in range(S):
+            a, e = s * ctx // S, (s + 1) * ctx // S
+            O, l = oracle_rows(wl, b, lambda t: np.arange(a, e), q)
+            worst = max(worst, check_partial(parts_o[s, b].cpu().numpy(), parts_l[s, b].cpu().numpy(),
+                                             O, l, f"peaky shard {s} seq {b}"))
+        O, l = oracle_rows(wl, b, lambda t: np.arange(ctx, ctx + t + 1), q)
+        worst = max(worst, check_partial(parts_o[S, b].cpu().numpy(), parts_l[S, b].cpu().numpy(), O, l,
+                                         f"peaky causal chunk seq {b}"))
+    print(f"peaky chunk partials (scale {scale}): max |dO| = {worst:.3e}")
