@@ -243,13 +243,13 @@ def _paged_inputs(torch, skvgen, wl, layer=0):
     return q, k_pool, v_pool, block_table, seq_lens
 
 
-def build_decode(torch, skv, skvgen, wl, status, art=None, inputs=None):
+def build_decode(torch, skv, skvgen, wl, status, art=None, inputs=None, layer=0):
     """Full-traversal (or ART: art = (tau, phi, patience)) decode of one paged
-    workload; `inputs` = (q, k_pool, v_pool, block_table, seq_lens) of another
-    step to share its cache."""
+    workload (layer `layer` of its seeded inputs); `inputs` = (q, k_pool,
+    v_pool, block_table, seq_lens) of another step to share its cache."""
     if inputs is None:
-        q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, wl)
-        skvgen.device_kv_paged(wl, q, k_pool, v_pool, bt, sl)
+        q, k_pool, v_pool, bt, sl = _paged_inputs(torch, skvgen, wl, layer=layer)
+        skvgen.device_kv_paged(wl, q, k_pool, v_pool, bt, sl, layer=layer)
     else:
         q, k_pool, v_pool, bt, sl = inputs
     out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
@@ -316,6 +316,133 @@ def build_select(torch, skv, skvgen, wl, status):
     step.tensors = dict(q=q, k_pool=k_pool, v_pool=v_pool, bt=bt, sl=sl, off=off, cent=cent, ids=ids,
                         ss=ss, se=se, out=out, lse=lse, ws=ws)
     return step
+
+
+def build_select_shared(torch, skv, skvgen, wl, status):
+    """Centroid selection of B requests over one shared fixed context (its
+    centroids read once per cluster of up to 8 requests), then each request's
+    attention over its chosen clusters' keys in that one context."""
+    q, k_pool, v_pool, bt, sl, off, cent = skvgen.device_shared_context(wl)
+    shape = (wl.B, wl.Hkv, wl.topk)
+    ids = torch.empty(shape, dtype=torch.int32, device="cuda")
+    ss = torch.empty(shape, dtype=torch.int32, device="cuda")
+    se = torch.empty(shape, dtype=torch.int32, device="cuda")
+    out = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
+    kw = dict(max_seq_len=wl.Lmax, scale=wl.scale, status=status, segments=(ss, se))
+    n = skv.decode_workspace_size(q, k_pool, v_pool, bt, sl, out, lse, **kw)
+    ws = torch.empty(max(n, 16) // 4 + 4, dtype=torch.float32, device="cuda")
+    a = skv.make_decode_args(q, k_pool, v_pool, bt, sl, out, lse, workspace=ws, **kw)
+    L = skv.lib()
+    C, k = 1 << wl.c_log2, wl.topk
+    qp, cp, op = ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(cent.data_ptr()), ctypes.c_void_p(off.data_ptr())
+    ip, sp_, ep = (ctypes.c_void_p(t.data_ptr()) for t in (ids, ss, se))
+
+    def run():
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        st = L.attn_select_centroids_shared(qp, cp, op, wl.B, wl.Hq, wl.Hkv, wl.d, C, k, ip, sp_, ep, stream)
+        if st != 0:
+            raise skv.SkvError(st, "attn_select_centroids_shared")
+        st = L.attn_decode(ctypes.byref(a), stream)
+        if st != 0:
+            raise skv.SkvError(st, "attn_decode")
+
+    run()
+    torch.cuda.synchronize()
+    sel_tokens = int((se - ss).sum().item())
+    nbytes = sel_tokens * wl.d * 4 + cent.numel() * 2 + off.numel() * 4
+    step = Step(run, nbytes, 1 + L.skv_decode_launches(ctypes.byref(a)),
+                {"selected_tokens": sel_tokens, "selected_frac": sel_tokens / (wl.B * wl.Hkv * wl.L),
+                 "centroid_bytes": cent.numel() * 2,
+                 "centroid_bytes_per_request_copy": wl.B * cent.numel() * 2,
+                 "note": "one shared context: centroid bytes counted once for all requests"})
+    step.tensors = dict(q=q, k_pool=k_pool, v_pool=v_pool, bt=bt, sl=sl, off=off, cent=cent, ids=ids,
+                        ss=ss, se=se, out=out, lse=lse, ws=ws)
+    return step
+
+
+def build_lookahead(torch, skv, skvgen, wl, status, n_ctas=24):
+    """Lookahead prefetch ("SparDA" 2) on a pair of cfg5-shaped layers: layer
+    l is a full-attention layer whose cache is on the GPU (ART, as the routed
+    stack runs it); layer l+1 keeps its KV in page-locked host memory.  While
+    layer l attends (main stream), layer l's Forecast picks layer l+1's top-k
+    blocks from their summaries and the gather kernel pulls them into a device
+    cache (side stream, launched first so its CTAs are resident); then layer
+    l+1 attends the cache.  Returns (overlapped step, layer-l-alone step,
+    prefetch-alone step, layer-(l+1)-alone step)."""
+    layers = [l for l in range(wl.n_layers - 1) if skvgen.route_bit(wl.seed, l) == 1]
+    l0 = layers[0]
+    fa = wl.with_(paging="identity")
+    st_fa = build_decode(torch, skv, skvgen, fa, status, art=(wl.tau, wl.phi, wl.patience),
+                         inputs=None, layer=l0)
+    # layer l0 + 1: generated on the device, moved to page-locked host memory
+    q1, k1, v1, bt1, sl1 = _paged_inputs(torch, skvgen, fa, layer=l0 + 1)
+    skvgen.device_kv_paged(fa, q1, k1, v1, bt1, sl1, layer=l0 + 1)
+    summ = skvgen.device_block_means(fa, k1, bt1, sl1)
+    k_host = k1.cpu().pin_memory()
+    v_host = v1.cpu().pin_memory()
+    del k1, v1
+    torch.cuda.empty_cache()
+    kp, vp = skv.host_device_pointer(k_host), skv.host_device_pointer(v_host)
+    G, k, mb = wl.G, wl.extra["lookahead_blocks"], fa.max_blocks
+    q0 = st_fa.tensors["q"]
+    x = q0[:, 0, ::G].contiguous()
+    w = skvgen.device_forecast_weights(fa, layer=l0)
+    f = torch.empty_like(x)
+    off = torch.tensor([[[min(j * 64, fa.seq_len(b)) for j in range(mb + 1)]] * wl.Hkv for b in range(wl.B)],
+                       dtype=torch.int32, device="cuda")
+    ids = torch.empty((wl.B, wl.Hkv, k), dtype=torch.int32, device="cuda")
+    ss0, se0, ss, se = (torch.empty_like(ids) for _ in range(4))
+    k_cache = torch.empty((wl.B * k, wl.Hkv, 64, wl.d), dtype=torch.bfloat16, device="cuda")
+    v_cache = torch.empty_like(k_cache)
+    bt_c = torch.arange(wl.B * k, dtype=torch.int32, device="cuda").view(wl.B, k)
+    sl_c = torch.full((wl.B,), k * 64, dtype=torch.int32, device="cuda")
+    out1 = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.float32, device="cuda")
+    lse1 = torch.empty((wl.B, 1, wl.Hq), dtype=torch.float32, device="cuda")
+    a1 = skv.make_decode_args(q1, k_cache, v_cache, bt_c, sl_c, out1, lse1, max_seq_len=k * 64,
+                              scale=wl.scale, status=status, segments=(ss, se))
+    L = skv.lib()
+    side = torch.cuda.Stream()
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    cur = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def prefetch(stream_ptr):
+        for st in (L.attn_forecast(p(x), p(w), wl.B, wl.Hkv, wl.d, p(f), stream_ptr),
+                   L.attn_select_centroids(p(f), p(summ), p(off), wl.B, wl.Hkv, wl.Hkv, wl.d, mb, k, p(ids),
+                                           p(ss0), p(se0), stream_ptr),
+                   L.attn_prefetch_blocks(kp, vp, p(bt1), p(sl1), p(ids), wl.B, wl.Hkv, wl.d, k, mb,
+                                          k_host.shape[0], wl.Lmax, p(k_cache), p(v_cache), p(ss), p(se),
+                                          p(status), n_ctas, stream_ptr)):
+            if st != 0:
+                raise skv.SkvError(st, "lookahead prefetch")
+
+    def attend_next():
+        st = L.attn_decode(ctypes.byref(a1), cur())
+        if st != 0:
+            raise skv.SkvError(st, "attn_decode")
+
+    def overlapped():
+        main = torch.cuda.current_stream()
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            prefetch(ctypes.c_void_p(side.cuda_stream))  # its CTAs take their SM slots first
+        st_fa.run()                                      # layer l on the main stream meanwhile
+        main.wait_stream(side)
+        attend_next()                                    # layer l+1 over the fetched blocks
+
+    copy_bytes = wl.B * wl.Hkv * k * 64 * wl.d * 4       # chosen blocks' K + V (full blocks)
+    nb_fa = st_fa.nbytes
+    step = Step(overlapped, nb_fa + copy_bytes, st_fa.launches + 4,
+                {"layer_full": l0, "layer_offloaded": l0 + 1, "lookahead_blocks": k,
+                 "copy_bytes": copy_bytes, "gather_ctas": n_ctas})
+    step.tensors = dict(fa=st_fa, q1=q1, bt1=bt1, sl1=sl1, summ=summ, k_host=k_host, v_host=v_host, x=x, w=w,
+                        f=f, off=off, ids=ids, ss0=ss0, se0=se0, ss=ss, se=se, k_cache=k_cache,
+                        v_cache=v_cache, bt_c=bt_c, sl_c=sl_c, out=out1, lse=lse1, a1=a1, side=side,
+                        ptrs=(kp, vp))
+    alone_fa = Step(st_fa.run, nb_fa, st_fa.launches)
+    alone_pf = Step(lambda: prefetch(cur()), copy_bytes, 3)
+    alone_next = Step(attend_next, copy_bytes, L.skv_decode_launches(ctypes.byref(a1)))
+    return step, alone_fa, alone_pf, alone_next
 
 
 def build_routed(torch, skv, skvgen, wl, status, layer_ids=None):
@@ -554,13 +681,19 @@ def measure_workload(c, name, headline):
         step = build_decode(torch, skv, skvgen, wl, status)
     elif kind == "cfg3":
         step = build_select(torch, skv, skvgen, wl, status)
+    elif kind == "cfg3s":
+        step = build_select_shared(torch, skv, skvgen, wl, status)
     elif kind == "cfg5":
         step = build_routed(torch, skv, skvgen, wl, status)
+    elif kind == "cfg5p":
+        step, *look_steps = build_lookahead(torch, skv, skvgen, wl, status)
     elif kind == "cfg4":
         step = build_chunk(torch, skv, skvgen, wl, status)
     else:
         raise SystemExit(f"workload {name}: no bench step")
     art_step, sweep_steps, dense_step = None, [], None
+    if kind != "cfg5p":
+        look_steps = None
     if kind == "cfg2" and not args.no_art:
         T = step.tensors
         shared = (T["q"], T["k_pool"], T["v_pool"], T["bt"], T["sl"])
@@ -571,10 +704,11 @@ def measure_workload(c, name, headline):
             sweep_steps.append((thr, build_decode(torch, skv, skvgen, wl, status, art=thr, inputs=shared)))
     router_step = build_router(torch, skv, skvgen, wl) if kind == "cfg5" else None
     level_steps = None
-    if kind == "cfg3":  # the same cache walked in full, for the savings of the selection
+    if kind in ("cfg3", "cfg3s"):  # the same cache walked in full, for the savings of the selection
         T = step.tensors
         dense_step = build_decode(torch, skv, skvgen, wl, status,
                                   inputs=(T["q"], T["k_pool"], T["v_pool"], T["bt"], T["sl"]))
+    if kind == "cfg3":
         level_steps = build_select_levels(torch, skv, skvgen, wl, step)
     stream = torch.cuda.current_stream()
     n_side = max(10, args.steps // 4)
@@ -590,6 +724,8 @@ def measure_workload(c, name, headline):
                      if router_step is not None else None)
         level_ms = ([c.timed(st, args.steps, args.warmup)[0] / args.steps for st in level_steps]
                     if level_steps is not None else None)
+        look_ms = ([c.timed(st, args.steps, args.warmup)[0] / args.steps for st in look_steps]
+                   if look_steps is not None else None)
     clocks = clk.summary()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status word {int(status.item()):#x}")
@@ -715,6 +851,17 @@ def measure_workload(c, name, headline):
                          "note": "per-layer route bits from pooled prefix/suffix query rows "
                                  "(untrained weights); outside the timed decode step"}
         res["gpu_launches"] += args.steps * router_step.launches
+    if look_ms is not None:
+        fa_ms, pf_ms, nx_ms = look_ms
+        cb = step.extra["copy_bytes"]
+        res["lookahead"] = {
+            "ms_overlapped_pair": ms_step, "ms_full_layer_alone": fa_ms, "ms_prefetch_alone": pf_ms,
+            "ms_next_layer_alone": nx_ms, "ms_serial_pair": fa_ms + pf_ms + nx_ms,
+            "hidden_frac_of_prefetch": (fa_ms + pf_ms + nx_ms - ms_step) / pf_ms if pf_ms > 0 else None,
+            "host_to_device_gbs": cb / (pf_ms * 1e-3) / 1e9, "copy_bytes": cb,
+            "note": "prefetch = Forecast + block top-k + gather from page-locked host memory (side "
+                    "stream, launched first); hidden_frac = (serial - overlapped) / prefetch alone"}
+        res["gpu_launches"] += args.steps * sum(st.launches for st in look_steps)
     if e2e is not None:
         res["e2e"] = e2e
     # ---- CPU-baseline leg (rank 0, one GPU): the oracle timed on the host cores, and
@@ -728,6 +875,8 @@ def measure_workload(c, name, headline):
         if art_step is not None:
             checks["art"] = oracle_check_art(wl, art_step, (wl.tau, wl.phi, wl.patience))
             checks["art_sweep"] = [oracle_check_art(wl, st, thr) for thr, st in sweep_steps]
+        if kind == "cfg5p":
+            checks["lookahead"] = oracle_check_lookahead(wl, step)
         if kind == "cfg5":
             fa = [ly for ly in step.tensors["layers"] if ly["fa"]]
             if fa:
@@ -735,7 +884,7 @@ def measure_workload(c, name, headline):
                                                        layer=fa[0]["layer"], n_groups=2)
         if checks:
             res["oracle_check"] = checks
-    del step, art_step, sweep_steps, dense_step, router_step, level_steps
+    del step, art_step, sweep_steps, dense_step, router_step, level_steps, look_steps
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return res
@@ -812,12 +961,56 @@ def oracle_check_art(wl, st, thr, layer=0, n_groups=8, flag_margin=1e-3):
             "flag_margin": flag_margin}
 
 
+def oracle_check_lookahead(wl, st, n_groups=2):
+    """The offloaded layer of the lookahead pair on sampled KV groups (CPU-baseline
+    leg): Forecast bits, chosen blocks and attention over them against the oracle."""
+    import oracle
+    import skvgen
+    T = st.tensors
+    l0 = st.extra["layer_full"]
+    fa = wl.with_(paging="identity")
+    k, G, d = st.extra["lookahead_blocks"], wl.G, wl.d
+    f = T["f"].view(torch_int16()).cpu().numpy().view(np.uint16)
+    ids = T["ids"].cpu().numpy()
+    out = T["out"][:, 0].cpu().numpy().astype(np.float64)
+    lse = T["lse"][:, 0].cpu().numpy().astype(np.float64)
+    q0, q1 = skvgen.host_q(fa, l0), skvgen.host_q(fa, l0 + 1)
+    w = skvgen.host_forecast_weights(fa, l0)
+    res = {"groups": [], "forecast_bits_equal": True, "ids_equal": 0, "ids_flagged": 0, "max_abs_dO": 0.0,
+           "max_rel_dlse": 0.0}
+    for b, kvh in _sample_groups(wl, n_groups):
+        res["groups"].append((b, kvh))
+        fr = oracle.forecast(q0[b, 0, kvh * G][None], w[kvh][None])[0]
+        res["forecast_bits_equal"] &= bool(np.array_equal(fr, f[b, kvh]))
+        K, V = skvgen.host_kv_group(fa, b, kvh, l0 + 1, q=q1)
+        summ = skvgen.host_block_means(K)
+        ref, sc = oracle.select(fr[None, None], summ[None], k)
+        if np.array_equal(ref[0], ids[b, kvh]):
+            res["ids_equal"] += 1
+        elif oracle.topk_boundary_gap(sc, k)[0] <= 1e-5:
+            res["ids_flagged"] += 1
+        keys = oracle.keys_blocks(ids[b, kvh], wl.seq_len(b))
+        qg = q1[b, 0, kvh * G:(kvh + 1) * G]
+        O, l = oracle.attend(qg[None], K[None], V[None], [[keys] * G], wl.scale)
+        hs = slice(kvh * G, (kvh + 1) * G)
+        res["max_abs_dO"] = max(res["max_abs_dO"], float(np.abs(out[b, hs] - O[0]).max()))
+        res["max_rel_dlse"] = max(res["max_rel_dlse"],
+                                  float((np.abs(lse[b, hs] - l[0]) / np.maximum(1.0, np.abs(l[0]))).max()))
+    return res
+
+
+def torch_int16():
+    import torch
+    return torch.int16
+
+
 # the other workloads measured in the default run, after the headline
-SIDE_WORKLOADS = ["cfg1_b1_h8_l4k", "cfg3_b8_h32_l64k_c1024_k102", "cfg4_b4_h32_l128k_chunk128",
-                  "cfg5_b8_h32_l128k_32layers"]
+SIDE_WORKLOADS = ["cfg1_b1_h8_l4k", "cfg3_b8_h32_l64k_c1024_k102", "cfg3s_b8_h32_l64k_shared",
+                  "cfg4_b4_h32_l128k_chunk128", "cfg5_b8_h32_l128k_32layers",
+                  "cfg5p_b8_h32_l128k_lookahead16"]
 SIDE_KEYS = ["value", "unit", "ms_per_step", "step_ms_p10_p50_p90", "roofline", "clocks", "config",
              "gpu_launches", "step_detail", "metric_tflops", "selection", "selection_levels", "router",
-             "oracle_check", "attended_tokens_per_s"]
+             "lookahead", "oracle_check", "attended_tokens_per_s"]
 
 
 def main():
@@ -856,7 +1049,7 @@ KERNEL_SOURCES = {
     "chunk_kernel": ["chunk.cu", "common.cuh", "decode.cuh"],
     "select_kernel": ["select.cu", "common.cuh"],
 }
-DOMINANT = {"cfg1": "decode_kernel", "cfg2": "decode_kernel", "cfg3": "decode_kernel",
+DOMINANT = {"cfg1": "decode_kernel", "cfg2": "decode_kernel", "cfg3": "decode_kernel", "cfg3s": "decode_kernel",
             "cfg4": "chunk_kernel", "cfg5": "art_kernel"}
 
 

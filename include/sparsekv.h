@@ -28,10 +28,18 @@
  *  attn_merge_lse   Exact merge of per-shard attention partials by their
  *                   log-sum-exp ("Pulsar Attention" Phase 2, online softmax
  *                   merge).
+ *  attn_select_centroids_shared
+ *                   The same for a batch of requests over one shared fixed
+ *                   context ("Squeezed Attention" Q1: the fixed context is
+ *                   clustered once and reused across requests).
  *  attn_select_centroids2
  *                   Two-level (hierarchical) centroid selection ("Squeezed
  *                   Attention", Q2 step 4): coarse clusters first, then the
  *                   fine clusters inside the chosen ones.
+ *  attn_forecast, attn_prefetch_blocks
+ *                   Lookahead selection of the next layer's KV blocks by a
+ *                   Forecast projection, and their prefetch from host memory
+ *                   into a device cache ("SparDA", technical summary 2).
  *  attn_route_layers
  *                   Per-layer hard routing between full and sparse attention
  *                   ("Flux Attention" section 2, Layer Router: pooling of the
@@ -172,9 +180,9 @@ typedef struct {
 SKV_API size_t skv_decode_workspace_size(const skv_decode_args* args);
 
 /* Kernels one attn_decode call launches for these arguments (1: the walk
- * merges its own partials -- a query chunk, or the split schedule that small
- * walks and segment lists take; 2: the walk, then the record merge), not
- * counting the workspace zeroing (a device memset); 0 if the arguments are
+ * merges its own partials -- every schedule but ART; 2: the ART walk, then the
+ * record merge), not counting the zeroing of the workspace's control words (a
+ * device memset, persistent and ART schedules); 0 if the arguments are
  * invalid.  Depends only on host-side fields; for profiling and accounting. */
 SKV_API int skv_decode_launches(const skv_decode_args* args);
 
@@ -182,7 +190,7 @@ SKV_API int skv_decode_launches(const skv_decode_args* args);
  * fields only; nothing is launched).  For profiling, capacity planning and
  * tests. */
 typedef enum {
-  SKV_SCHED_PERSISTENT = 0, /* persistent CTAs over all tiles, then the record merge */
+  SKV_SCHED_PERSISTENT = 0, /* persistent CTAs over all tiles; a group's last arrival merges it */
   SKV_SCHED_CLUSTER = 1,    /* one cluster of `splits` CTAs per KV group, merged in-kernel */
   SKV_SCHED_ART = 2,        /* ART: persistent CTAs over (chunk, group) items, then the merge */
   SKV_SCHED_CHUNK = 3       /* query chunk (q_tokens > 1) on the tensor cores */
@@ -206,8 +214,10 @@ SKV_API skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_
  * {order, window, seg_start/seg_end, kv range}; ART only with natural or
  * `order` traversal.
  * Launch shapes (they follow from host-side fields only):
- *  - long walks: persistent CTAs (2 per SM) share all tiles, then a merge
- *    kernel combines the partial records in the workspace;
+ *  - long walks: persistent CTAs (2 per SM) share all tiles; each warp
+ *    writes a partial record per KV group it touched to the workspace and
+ *    arrives on the group's counter (zeroed by a memset before the launch),
+ *    and the warp whose arrival is the group's last merges its records;
  *  - small walks (at most 8 tiles per resident CTA) and segment lists: one
  *    thread-block cluster of up to 16 CTAs per KV group, merged inside the
  *    kernel through distributed shared memory (no workspace); a cluster size
@@ -238,8 +248,18 @@ SKV_API skv_status attn_decode(const skv_decode_args* args, skv_stream_t stream)
  *    Nothing in it needs to start at zero (every byte read is written earlier
  *    in the same call), but calls that can overlap on the GPU (other streams,
  *    other host threads) race on it: serialise them.
- * Errors: as attn_decode, plus SKV_ECUDA if the address lookup fails. */
-#define SKV_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)
+ * Errors: as attn_decode, plus SKV_ECUDA if the address lookup fails.
+ * What fits in the array (skv_decode_workspace_size on a 148-SM B200): every
+ * walk without ART of up to about 3,600 KV groups at 4 query heads per KV
+ * head, 1,800 at 8 (the persistent schedule needs about 17 KiB, or 34 KiB,
+ * per resident CTA and per KV group; small walks and segment lists need
+ * none), and ART at the Llama-3.1-8B shape (32 query / 8 KV heads) for up to
+ * 64 sequences of 32K tokens or 16 of 128K (ART needs 24 to 39 MiB of
+ * per-CTA scratch plus about 0.6 KiB per (KV group, chunk, query head)).
+ * The device address is
+ * looked up once per device and kept for the whole process: it assumes the
+ * device's primary context is not reset (cudaDeviceReset) in between. */
+#define SKV_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 SKV_API skv_status attn_decode_static_ws(const skv_decode_args* args, skv_stream_t stream);
 
 /* Centroid selection ("Squeezed Attention" Q2 step 2) for each KV group
@@ -257,6 +277,28 @@ SKV_API skv_status attn_select_centroids(const void* q, const void* centroids, c
                                  int batch, int q_heads, int kv_heads, int head_dim,
                                  int n_clusters, int topk, int32_t* sel_ids, int32_t* seg_start,
                                  int32_t* seg_end, skv_stream_t stream);
+
+/* Centroid selection over ONE shared fixed context ("Squeezed Attention" Q1:
+ * the fixed part of the prompt is clustered offline once and reused by every
+ * request; Q2 step 2 per request).  Every request b of the batch has its own
+ * query, all requests share one centroid set and one key layout per KV head:
+ *   score_c(b, kvh) = (sum of request b's query heads of KV head kvh) . centroid[kvh][c]
+ * and the kept clusters follow the same rule as attn_select_centroids (top
+ * `topk`, ties to the lower index, ids ascending, key ranges from
+ * cluster_off[kvh]).  Up to 8 requests are served together: each centroid row
+ * is read once for all of them.
+ *  q           bf16 [batch][q_heads][head_dim] (one query token per request)
+ *  centroids   bf16 [kv_heads][n_clusters][head_dim] (shared)
+ *  cluster_off int32 [kv_heads][n_clusters + 1] (shared)
+ *  sel_ids, seg_start, seg_end  int32 [batch][kv_heads][topk] (outputs)
+ * The selected ranges index the shared context: attend them with attn_decode
+ * (segments) over a block_table whose rows map every request to the same
+ * pages.  Supported: head_dim 128, 1 <= topk <= n_clusters <= 4096. */
+SKV_API skv_status attn_select_centroids_shared(const void* q, const void* centroids,
+                                        const int32_t* cluster_off, int batch, int q_heads,
+                                        int kv_heads, int head_dim, int n_clusters, int topk,
+                                        int32_t* sel_ids, int32_t* seg_start, int32_t* seg_end,
+                                        skv_stream_t stream);
 
 /* Two-level centroid selection ("Squeezed Attention" Q2 step 4, hierarchical
  * clustering) for each KV group (b, kvh), with the group's query heads summed
@@ -322,6 +364,68 @@ SKV_API skv_status attn_merge_lse(const float* o_parts, const float* lse_parts, 
 SKV_API skv_status attn_route_layers(const void* q, const float* w, const float* bias, int n_layers,
                              int batch, int tokens, int q_heads, int head_dim, int n_prefix,
                              int n_suffix, float* logits, uint8_t* route, skv_stream_t stream);
+
+/* Lookahead block selection and prefetch from host memory ("SparDA",
+ * technical summary section 2: "Trainable Lookahead Sparse Selection" and
+ * "Asynchronous Prefetch with Persistent UVA Kernel").  Layer l's Forecast
+ * projection F_l (one head per GQA group) predicts the top-k KV blocks that
+ * layer l+1 needs; while layer l runs, those blocks are pulled from CPU
+ * memory into a small device cache, and layer l+1 attends them there.
+ *
+ * attn_forecast: f[b][kvh] = bf16( W[kvh]^T x[b][kvh] ) for every request b
+ * and KV head kvh: output dim j accumulates w[kvh][i][j] * x[b][kvh][i] in
+ * fp32 with fused multiply-adds in order i = 0 .. head_dim-1, then rounds to
+ * bf16 (nearest even).  Untrained weights make this a random projection.
+ *  x  bf16 [batch][kv_heads][head_dim]   the layer-l activation per GQA group
+ *  w  bf16 [kv_heads][head_dim][head_dim] (input dim major)
+ *  f  bf16 [batch][kv_heads][head_dim]   (output)
+ * The block choice is then attn_select_centroids with q = f (q_heads =
+ * kv_heads), the block summaries of layer l+1 as the centroids and the block
+ * boundaries (j * 64, clipped to the sequence) as cluster_off.
+ * Supported: head_dim 128; batch, kv_heads <= 65535. */
+SKV_API skv_status attn_forecast(const void* x, const void* w, int batch, int kv_heads, int head_dim,
+                                 void* f, skv_stream_t stream);
+
+/* Device-accessible address of page-locked host memory (allocated with
+ * cudaHostAlloc, or registered with cudaHostRegister and mapped); under
+ * unified addressing it is the host address itself.  SKV_EINVAL if the memory
+ * is not page-locked and mapped.  Not stream-ordered: call it at set-up, not
+ * during stream capture. */
+SKV_API skv_status skv_host_device_pointer(const void* host, void** dev);
+
+/* attn_prefetch_blocks: copy the chosen blocks from a host KV pool into a
+ * device cache.  n_ctas CTAs walk the (b, kvh, i) items; item (b, kvh, i)
+ * copies logical block j = block_ids[b][kvh][i] of sequence b (its page
+ * block_table[b][j] of the host pools, K and V rows of KV head kvh) into page
+ * b * topk + i of the cache pools (slot kvh), read from host memory with
+ * 16-byte loads through the pools' device-accessible addresses, and writes
+ * the slot's token range in the cache
+ *     seg_start[b][kvh][i] = i * 64,  seg_end = i * 64 + (tokens of block j)
+ * (an empty range for block_ids = -1 or a block at or past the sequence's
+ * end, as an empty cluster contributes no keys).  attn_decode with these segments, the
+ * cache pools and a block table with row b = b*topk .. b*topk + topk - 1 then
+ * attends exactly the chosen blocks.  Rows of the cache past a block's last
+ * token are left untouched.
+ *  k_host, v_host  device-accessible addresses (skv_host_device_pointer) of
+ *                  page-locked bf16 pools [num_pages][kv_heads][64][head_dim]
+ *  block_table     int32 [batch][max_blocks] (device), pages of the host pools
+ *  seq_lens        int32 [batch] (device)
+ *  block_ids       int32 [batch][kv_heads][topk] (device), e.g. from
+ *                  attn_select_centroids
+ *  k_cache, v_cache bf16 [batch * topk][kv_heads][64][head_dim] (device)
+ *  seg_start, seg_end int32 [batch][kv_heads][topk] (device, outputs)
+ *  status_word     NULL or a device uint32: SKV_DEV_BAD_PAGE and _BAD_SEQLEN
+ *                  are OR-ed in and the item copies nothing
+ * Launch it on its own stream, before the kernels it should overlap, with a
+ * few CTAs (16-32 saturate a PCIe link) so that it stays resident beside
+ * them.  Supported: head_dim 128; 16-byte aligned pools and caches. */
+SKV_API skv_status attn_prefetch_blocks(const void* k_host, const void* v_host,
+                                        const int32_t* block_table, const int32_t* seq_lens,
+                                        const int32_t* block_ids, int batch, int kv_heads,
+                                        int head_dim, int topk, int max_blocks, int num_pages,
+                                        int max_seq_len, void* k_cache, void* v_cache,
+                                        int32_t* seg_start, int32_t* seg_end,
+                                        uint32_t* status_word, int n_ctas, skv_stream_t stream);
 
 /* The status a device status word stands for, once the caller has read it
  * back after synchronising: SKV_ETIMEOUT if SKV_DEV_TIMEOUT is set (a bounded

@@ -18,6 +18,11 @@ each option attends, following the pages:
 * shard merge              -- "Pulsar Attention" Phase 2
 * layer routing            -- "Flux Attention" 2 (Layer Router: prefix and
                               suffix pooling of the query tensor, hard routing)
+* shared-context selection -- "Squeezed Attention" Q1 (one fixed context,
+                              clustered once, shared by every request)
+* lookahead block choice   -- "SparDA" 2 (Forecast projection, then the top-k
+                              blocks by the projection's dot product with each
+                              block's summary)
 * two-level selection      -- "Squeezed Attention" Q2 step 4 (hierarchical
                               clustering: coarse clusters first, then the fine
                               clusters inside the chosen coarse ones)
@@ -57,6 +62,7 @@ def lib():
         L.orc_max_threads.restype = i32
         L.orc_set_threads.argtypes = [i32]
         L.orc_merge.argtypes = [i32, i64, i32, _p, _p, _p, _p]
+        L.orc_forecast.argtypes = [i64, i32, _p, _p, _p]
         _LIB = L
     return _LIB
 
@@ -174,6 +180,42 @@ def select(q, cent, k):
     sc = np.empty((U, C))
     lib().orc_select(U, G, d, _ptr(q), _ptr(cent), C, k, _ptr(ids), _ptr(sc))
     return ids, sc
+
+
+def select_shared(q, cent, k):
+    """Centroid top-k for a batch of requests over ONE shared fixed context
+    ("Squeezed Attention" Q1: the fixed context is clustered offline once and
+    reused by every request; Q2 step 2 per request): request u's selection is
+    the per-sequence selection of select() with its own query against the
+    shared centroids.  q [U][G][d]; cent [C][d] (bf16 bits).  Returns ids
+    [U][k] (ascending) and scores [U][C] (fp64)."""
+    q = _u16(q)
+    cent = _u16(cent)
+    U = q.shape[0]
+    return select(q, np.broadcast_to(cent, (U,) + cent.shape), k)
+
+
+def forecast(x, w):
+    """Forecast projection ("SparDA" 2: one Forecast head per GQA group maps
+    layer l's activation to the query that ranks layer l+1's KV blocks):
+    f[u][j] = bf16(sum_i w[u][i][j] x[u][i]) with the sum in fp32, one fused
+    multiply-add per term in ascending i, rounded to nearest even.
+    x [U][d], w [U][d][d] (input dim major), bf16 bits.  Returns f [U][d] bits."""
+    x, w = _u16(x), _u16(w)
+    U, d = x.shape
+    f = np.empty((U, d), dtype=np.uint16)
+    lib().orc_forecast(U, d, _ptr(x), _ptr(w), _ptr(f))
+    return f
+
+
+def keys_blocks(ids, L, bs=64):
+    """Token set of logical blocks `ids` of a sequence of L tokens (the keys a
+    layer attends once its chosen blocks are fetched)."""
+    s = set()
+    for j in ids:
+        if int(j) >= 0:
+            s.update(range(int(j) * bs, min((int(j) + 1) * bs, L)))
+    return np.array(sorted(s), dtype=np.int64)
 
 
 def select2(q, coarse, coarse_off, fine, k1, k2):

@@ -14,8 +14,15 @@
  *              layers keep only a minimal KV set)
  *   [PULSAR]   "Pulsar Attention", Phase 1 (64-token sink) and Phase 2
  *              (exact online-softmax merge of per-shard partials)
+ *   [SPARDA]   "SparDA", technical summary section 2 (a per-layer Forecast
+ *              projection, one head per GQA group, picks the next layer's
+ *              KV blocks ahead of time)
  *
- * Precision: fp64 throughout; inputs are bf16 (exact in fp64).
+ * Precision: fp64 throughout; inputs are bf16 (exact in fp64).  One
+ * exception, orc_forecast: its output is a bf16 query that then decides
+ * integer block ids, so it is computed in the precision the method's kernel
+ * fixes (fp32 fused multiply-adds in input order, one rounding to bf16), and
+ * both sides take the decision from the same bits.
  * Build: gcc -O2 -fPIC -shared -fopenmp -ffp-contract=off oracle.c -lm
  */
 #include <math.h>
@@ -331,5 +338,39 @@ void orc_merge(int S, int64_t N, int d, const double* o_parts /*[S][N][d]*/,
     }
     for (int j = 0; j < d; ++j) out[n * d + j] /= W;
     lse[n] = M + log(W);
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Forecast projection.  [SPARDA] 2: layer l's Forecast head (one per GQA   */
+/* group) maps the layer's activation x to a vector whose dot products with */
+/* the next layer's block summaries rank the blocks to fetch:               */
+/*   f[j] = bf16( sum_i w[i][j] x[i] ),                                     */
+/* the sum taken in fp32 with one fused multiply-add per term, i ascending, */
+/* and rounded to bf16 to nearest, ties to even.                            */
+/* ------------------------------------------------------------------------ */
+static uint16_t f32_to_bf16_rne(float f) {
+  union { float f; uint32_t u; } c;
+  c.f = f;
+  if ((c.u & 0x7F800000u) == 0x7F800000u && (c.u & 0x007FFFFFu)) return (uint16_t)((c.u >> 16) | 0x40u);
+  uint32_t lsb = (c.u >> 16) & 1u;
+  return (uint16_t)((c.u + 0x7FFFu + lsb) >> 16);
+}
+
+void orc_forecast(int64_t n_units, int d, const uint16_t* x /*[u][d]*/, const uint16_t* w /*[u][d][d]*/,
+                  uint16_t* f /*[u][d]*/) {
+#pragma omp parallel for schedule(static)
+  for (int64_t u = 0; u < n_units; ++u) {
+    const uint16_t* wu = w + u * d * d;
+    for (int j = 0; j < d; ++j) {
+      float acc = 0.0f;
+      for (int i = 0; i < d; ++i) {
+        union { float f; uint32_t u; } a, b;
+        a.u = (uint32_t)wu[(int64_t)i * d + j] << 16;
+        b.u = (uint32_t)x[u * d + i] << 16;
+        acc = fmaf(a.f, b.f, acc);
+      }
+      f[u * d + j] = f32_to_bf16_rne(acc);
+    }
   }
 }

@@ -19,6 +19,7 @@ _HOST = None
 _DEV = None
 
 S_Q, S_K, S_V, S_CENTER, S_ASSIGN, S_PERM, S_HEAVY, S_ROUTE, S_ROUTER_W = 1, 2, 3, 4, 5, 6, 7, 8, 9
+S_FORECAST_W = 12  # Forecast projection weights (lookahead block selection)
 
 _u64, _u32, _i32, _i64, _p = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
 
@@ -47,6 +48,7 @@ def host_lib():
         lib.skvg_host_f64_to_bf16.restype = ctypes.c_uint16
         lib.skvg_host_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.skvg_host_f32_to_bf16.restype = ctypes.c_uint16
+        lib.skvg_host_block_means.argtypes = [_p, _u64, ctypes.c_int, ctypes.c_int, _p]
         lib.skvg_host_key.argtypes = [_u64, _u32, _u32]
         lib.skvg_host_key.restype = _u64
         _HOST = lib
@@ -65,7 +67,9 @@ def dev_lib():
                                           _p, _p, ctypes.c_int, ctypes.c_int, _p, _p, _p, _p]
         lib.skvg_dev_mixture.argtypes = [_u64, _u32, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u64, _u64,
                                          _u32, _p, ctypes.c_int, ctypes.c_int, _p, _p, _p, _p]
-        for f in (lib.skvg_dev_normal_bf16, lib.skvg_dev_qhat, lib.skvg_dev_kv_paged, lib.skvg_dev_mixture):
+        lib.skvg_dev_block_means.argtypes = [_p, _p, _p] + [ctypes.c_int] * 5 + [_p, _p]
+        for f in (lib.skvg_dev_normal_bf16, lib.skvg_dev_qhat, lib.skvg_dev_kv_paged, lib.skvg_dev_mixture,
+                  lib.skvg_dev_block_means):
             f.restype = ctypes.c_int
         _DEV = lib
     return _DEV
@@ -125,6 +129,24 @@ def host_mixture_group(wl, b, kvh, layer=0, want_keys=True):
     host_lib().skvg_host_mixture_group(wl.seed, layer, g, wl.Lmax, L, wl.d, wl.c_log2, _ptr(off),
                                        _ptr(K) if K is not None else None, _ptr(cent))
     return K, off, cent
+
+
+def host_block_means(K, bs=64):
+    """Block summaries of one KV group's keys K [L][d] (bf16 bits): [nb][d],
+    bf16 of the fp64 mean of each block's keys (the last block may be short)."""
+    K = np.ascontiguousarray(K, dtype=np.uint16)
+    L, d = K.shape
+    out = np.empty(((L + bs - 1) // bs, d), dtype=np.uint16)
+    host_lib().skvg_host_block_means(_ptr(K), L, d, bs, _ptr(out))
+    return out
+
+
+def host_forecast_weights(wl, layer=0):
+    """Forecast projection weights of a layer, bf16 bits [Hkv][d][d]: seeded
+    normals times 2^-4 (exact in bf16), untrained."""
+    w = host_normal_bf16(wl.seed, S_FORECAST_W, wl.Hkv * wl.d * wl.d, layer=layer)
+    v = bf16_to_f64(w) * 0.0625
+    return (v.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16).reshape(wl.Hkv, wl.d, wl.d)
 
 
 def host_perm(seed, n, stream=S_PERM, layer=0):
@@ -209,6 +231,60 @@ def device_mixture(wl, k_pool, block_table, layer=0):
                                       ctypes.c_void_p(cent.data_ptr()), _stream_ptr(torch)),
            "skvg_dev_mixture")
     return off, cent
+
+
+def device_block_means(wl, k_pool, block_table, seq_lens):
+    """Block summaries of every (sequence, KV head) of a paged cache:
+    bf16 [B][Hkv][max_blocks][d] (0 past a sequence's end)."""
+    import torch
+    mb = block_table.shape[1]
+    out = torch.empty((wl.B, wl.Hkv, mb, wl.d), dtype=torch.bfloat16, device=k_pool.device)
+    _check(dev_lib().skvg_dev_block_means(ctypes.c_void_p(k_pool.data_ptr()),
+                                          ctypes.c_void_p(block_table.data_ptr()),
+                                          ctypes.c_void_p(seq_lens.data_ptr()), wl.B, wl.Hkv, wl.d, mb,
+                                          wl.bs, ctypes.c_void_p(out.data_ptr()), _stream_ptr(torch)),
+           "skvg_dev_block_means")
+    return out
+
+
+def device_forecast_weights(wl, layer=0):
+    """The same weights as host_forecast_weights, on the device."""
+    import torch
+    w = torch.empty((wl.Hkv, wl.d, wl.d), dtype=torch.bfloat16, device="cuda")
+    device_normal_bf16(w, wl.seed, S_FORECAST_W, layer)
+    return w * 0.0625  # a power of two: exact in bf16
+
+
+def device_shared_context(wl):
+    """Inputs of a shared-context workload: one context (that of request 0 of
+    `wl`, a mixture) in a pool of its own pages, a block table whose B rows all
+    map to those pages, and every request's own query.  Returns q [B][1][Hq][d],
+    k_pool, v_pool, block_table [B][max_blocks], seq_lens [B], cluster_off
+    [Hkv][C+1] and centroids [Hkv][C][d]."""
+    import torch
+    one = wl.with_(B=1, shared_context=False)
+    bt1, num_pages = block_table_host(one)
+    q = device_q(wl)
+    q1 = device_q(one)
+    shape = (max(num_pages, 1), wl.Hkv, wl.bs, wl.d)
+    k_pool = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    v_pool = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    bt = torch.tensor(bt1, dtype=torch.int32, device="cuda")
+    sl1 = torch.tensor([one.seq_len(0)], dtype=torch.int32, device="cuda")
+    off, cent = device_mixture(one, k_pool, bt)
+    device_kv_paged(one, q1, k_pool, v_pool, bt, sl1, keys=False)
+    block_table = bt.expand(wl.B, bt.shape[1]).contiguous()
+    seq_lens = sl1.expand(wl.B).contiguous()
+    return q, k_pool, v_pool, block_table, seq_lens, off[0].contiguous(), cent[0].contiguous()
+
+
+def host_shared_context(wl, kvh):
+    """Logical keys [L][d], values [L][d], cluster offsets [C+1] and centroids
+    [C][d] of KV head kvh of a shared-context workload's one context."""
+    one = wl.with_(B=1, shared_context=False)
+    K, off, cent = host_mixture_group(one, 0, kvh)
+    _, V = host_kv_group(one.with_(mixture=False, structured=False), 0, kvh)
+    return K, V, off, cent
 
 
 from .workloads import Workload, WORKLOADS, block_table_host  # noqa: E402,F401

@@ -129,6 +129,31 @@ __global__ void k_mix_centroids(uint64_t kc, uint64_t kk, int d, uint64_t Lmax, 
   }
 }
 
+// Block summaries: element (b, kvh, j, dim) = bf16( fp64 mean of the keys of
+// logical block j of sequence b, KV head kvh ); blocks past the sequence are 0.
+__global__ void k_block_means(const uint16_t* k_pool, const int* block_table, const int* seq_lens,
+                              int B, int Hkv, int d, int max_blocks, int bs, uint16_t* out) {
+  uint64_t n = (uint64_t)B * Hkv * max_blocks * d;
+  for (uint64_t e = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; e < n;
+       e += (uint64_t)gridDim.x * blockDim.x) {
+    uint64_t j = e % d;
+    uint64_t blk = (e / d) % max_blocks;
+    uint64_t kvh = (e / ((uint64_t)d * max_blocks)) % Hkv;
+    uint64_t b = e / ((uint64_t)d * max_blocks * Hkv);
+    int L = seq_lens[b];
+    int t0 = (int)blk * bs, t1 = t0 + bs < L ? t0 + bs : L;
+    int page = block_table[b * max_blocks + blk];
+    if (t1 <= t0 || page < 0) {
+      out[e] = 0;
+      continue;
+    }
+    double sum = 0.0;
+    for (int t = t0; t < t1; ++t)
+      sum = SKVG_DADD(sum, skvg_bf16_to_f64(k_pool[(((uint64_t)page * Hkv + kvh) * bs + (t - t0)) * d + j]));
+    out[e] = skvg_f64_to_bf16(SKVG_DDIV(sum, (double)(t1 - t0)));
+  }
+}
+
 inline int grid_for(uint64_t n) {
   uint64_t g = (n + 255) / 256;
   return (int)(g > 148ull * 64 ? 148ull * 64 : (g == 0 ? 1 : g));
@@ -185,6 +210,14 @@ int skvg_dev_mixture(uint64_t seed, uint32_t layer, int B, int Hkv, int d, uint6
   if (centroids)
     k_mix_centroids<<<grid_for((uint64_t)G * C * d), 256, 0, st>>>(kc, kk, d, Lmax, c_log2, off,
                                                                    G, centroids);
+  return (int)cudaGetLastError();
+}
+
+int skvg_dev_block_means(const uint16_t* k_pool, const int* block_table, const int* seq_lens, int B,
+                         int Hkv, int d, int max_blocks, int bs, uint16_t* out, cudaStream_t st) {
+  uint64_t n = (uint64_t)B * Hkv * max_blocks * d;
+  if (n == 0) return 0;
+  k_block_means<<<grid_for(n), 256, 0, st>>>(k_pool, block_table, seq_lens, B, Hkv, d, max_blocks, bs, out);
   return (int)cudaGetLastError();
 }
 

@@ -124,3 +124,17 @@ int skvg_host_is_heavy(uint64_t seed, uint32_t layer, uint64_t g, uint64_t Lmax,
 
 uint16_t skvg_host_f64_to_bf16(double x) { return skvg_f64_to_bf16(x); }
 uint16_t skvg_host_f32_to_bf16(float x) { return skvg_f32_to_bf16(x); }
+
+/* Block summaries of one KV group: out[j][:] = bf16( fp64 mean of the keys
+ * K[t][:] of block j, t in [j*bs, min((j+1)*bs, L)) ), ascending t. */
+void skvg_host_block_means(const uint16_t* K, uint64_t L, int d, int bs, uint16_t* out) {
+  uint64_t nb = (L + (uint64_t)bs - 1) / (uint64_t)bs;
+  for (uint64_t blk = 0; blk < nb; ++blk) {
+    uint64_t t0 = blk * (uint64_t)bs, t1 = t0 + (uint64_t)bs < L ? t0 + (uint64_t)bs : L;
+    for (int j = 0; j < d; ++j) {
+      double sum = 0.0;
+      for (uint64_t t = t0; t < t1; ++t) sum = SKVG_DADD(sum, skvg_bf16_to_f64(K[t * (uint64_t)d + j]));
+      out[blk * (uint64_t)d + j] = skvg_f64_to_bf16(SKVG_DDIV(sum, (double)(t1 - t0)));
+    }
+  }
+}

@@ -26,6 +26,7 @@ class Workload:
     structured: bool = False    # token-0 sink (+6 qhat) and 1% heavy tokens (+4 qhat)
     paging: str = "identity"    # "identity" | "perm" | "window"
     mixture: bool = False       # Gaussian-mixture keys, cluster-contiguous
+    shared_context: bool = False  # every request reads one context (that of request 0)
     c_log2: int = 10            # 1024 clusters
     topk: int = 102
     # ART (recency-first traversal)
@@ -126,9 +127,19 @@ WORKLOADS = {
     # centroid-selected decode over a 1024-component Gaussian mixture per KV head
     "cfg3_b8_h32_l64k_c1024_k102": Workload("cfg3_b8_h32_l64k_c1024_k102", B=8, Hq=32, Hkv=8, L=65536,
                                             seed=0x5EED0003, mixture=True, c_log2=10, topk=102),
+    # centroid-selected decode of 8 requests over ONE shared fixed context
+    # (clustered once, per KV head, reused by every request)
+    "cfg3s_b8_h32_l64k_shared": Workload("cfg3s_b8_h32_l64k_shared", B=8, Hq=32, Hkv=8, L=65536,
+                                         seed=0x5EED0006, mixture=True, c_log2=10, topk=102,
+                                         shared_context=True),
     # 8 shards of 16384 context keys + a causal 128-token query chunk
     "cfg4_b4_h32_l128k_chunk128": Workload("cfg4_b4_h32_l128k_chunk128", B=4, Hq=32, Hkv=8,
                                            L=131072 + 128, Tq=128, seed=0x5EED0004, shards=8, chunk=128),
+    # lookahead prefetch on cfg5's layers: a full layer on the GPU, the next layer's KV in
+    # host memory, its top-16 blocks (of 2048) chosen by the Forecast and fetched meanwhile
+    "cfg5p_b8_h32_l128k_lookahead16": Workload("cfg5p_b8_h32_l128k_lookahead16", B=8, Hq=32, Hkv=8,
+                                               L=131072, seed=0x5EED0005, structured=True, n_layers=32,
+                                               extra={"lookahead_blocks": 16}),
     # 32-layer routed attention-only decode stack
     "cfg5_b8_h32_l128k_32layers": Workload("cfg5_b8_h32_l128k_32layers", B=8, Hq=32, Hkv=8, L=131072,
                                            seed=0x5EED0005, structured=True, n_layers=32),

@@ -13,7 +13,9 @@ import os
 
 from . import _build
 
-__all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids", "attn_merge_lse",
+__all__ = ["attn_decode", "attn_decode_static_ws", "attn_select_centroids",
+           "attn_select_centroids_shared", "attn_merge_lse", "attn_forecast", "attn_prefetch_blocks",
+           "host_device_pointer",
            "attn_route_layers", "attn_select_centroids2",
            "decode_workspace_size", "decode_launches", "decode_plan",
            "strerror", "status_of_word", "SkvError", "lib", "DEV_BITS"]
@@ -76,12 +78,20 @@ def lib():
         L.attn_decode_static_ws.restype = _i
         L.attn_select_centroids.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p]
         L.attn_select_centroids.restype = _i
+        L.attn_select_centroids_shared.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p]
+        L.attn_select_centroids_shared.restype = _i
         L.attn_merge_lse.argtypes = [_p, _p, _i, _i, _i, _p, _p, _p]
         L.attn_merge_lse.restype = _i
         L.attn_route_layers.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p]
         L.attn_route_layers.restype = _i
         L.attn_select_centroids2.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p]
         L.attn_select_centroids2.restype = _i
+        L.attn_forecast.argtypes = [_p, _p, _i, _i, _i, _p, _p]
+        L.attn_forecast.restype = _i
+        L.skv_host_device_pointer.argtypes = [_p, ctypes.POINTER(_p)]
+        L.skv_host_device_pointer.restype = _i
+        L.attn_prefetch_blocks.argtypes = [_p, _p, _p, _p, _p] + [_i] * 8 + [_p, _p, _p, _p, _p, _i, _p]
+        L.attn_prefetch_blocks.restype = _i
         L.skv_status_of_word.argtypes = [ctypes.c_uint32]
         L.skv_status_of_word.restype = _i
         L.skv_test_withhold_tile.argtypes = [_i, _i]
@@ -94,6 +104,41 @@ def lib():
 
 def strerror(status):
     return lib().skv_strerror(int(status)).decode()
+
+
+def attn_forecast(x, w, f, stream=None):
+    """Forecast projection: x bf16 [B, Hkv, d], w bf16 [Hkv, d, d] (input dim
+    major) -> f bf16 [B, Hkv, d] (see attn_forecast in include/sparsekv.h)."""
+    B, Hkv, d = x.shape
+    st = lib().attn_forecast(_ptr(x), _ptr(w), B, Hkv, d, _ptr(f), _stream(stream))
+    if st != SKV_OK:
+        raise SkvError(st, "attn_forecast")
+
+
+def host_device_pointer(t):
+    """Device-accessible address of a page-locked (pinned) host tensor."""
+    p = ctypes.c_void_p()
+    st = lib().skv_host_device_pointer(ctypes.c_void_p(t.data_ptr()), ctypes.byref(p))
+    if st != SKV_OK:
+        raise SkvError(st, "skv_host_device_pointer")
+    return p
+
+
+def attn_prefetch_blocks(k_host, v_host, block_table, seq_lens, block_ids, k_cache, v_cache, seg_start,
+                         seg_end, *, max_seq_len, status=None, n_ctas=16, stream=None, host_ptrs=None):
+    """Copy the chosen blocks from pinned host pools [P, Hkv, 64, 128] into the
+    device caches [B * k, Hkv, 64, 128]; block_ids int32 [B, Hkv, k]; writes the
+    cache token ranges seg_start / seg_end [B, Hkv, k] (see attn_prefetch_blocks
+    in include/sparsekv.h).  host_ptrs: (k, v) from host_device_pointer, to skip
+    the look-up."""
+    B, Hkv, k = block_ids.shape
+    P, _, _, d = k_host.shape
+    kp, vp = host_ptrs if host_ptrs is not None else (host_device_pointer(k_host), host_device_pointer(v_host))
+    st = lib().attn_prefetch_blocks(kp, vp, _ptr(block_table), _ptr(seq_lens), _ptr(block_ids), B, Hkv, d, k,
+                                    block_table.shape[1], P, int(max_seq_len), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(seg_start), _ptr(seg_end), _ptr(status), int(n_ctas), _stream(stream))
+    if st != SKV_OK:
+        raise SkvError(st, "attn_prefetch_blocks")
 
 
 def status_of_word(word):
@@ -230,6 +275,20 @@ def attn_select_centroids(q, centroids, cluster_off, topk, sel_ids, seg_start, s
                                      _stream(stream))
     if st != SKV_OK:
         raise SkvError(st, "attn_select_centroids")
+
+
+def attn_select_centroids_shared(q, centroids, cluster_off, topk, sel_ids, seg_start, seg_end,
+                                 stream=None):
+    """q [B, Hq, 128] bf16 (or [B, 1, Hq, 128]), one query per request; centroids
+    [Hkv, C, 128] bf16 and cluster_off [Hkv, C+1] int32 shared by every request;
+    outputs int32 [B, Hkv, topk]."""
+    Hkv, C, d = centroids.shape
+    B, Hq = q.shape[0], q.shape[-2]
+    st = lib().attn_select_centroids_shared(_ptr(q), _ptr(centroids), _ptr(cluster_off), B, Hq, Hkv, d,
+                                            C, int(topk), _ptr(sel_ids), _ptr(seg_start), _ptr(seg_end),
+                                            _stream(stream))
+    if st != SKV_OK:
+        raise SkvError(st, "attn_select_centroids_shared")
 
 
 def attn_merge_lse(o_parts, lse_parts, out, lse, stream=None):

@@ -8,7 +8,7 @@ CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libsparsekv.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 SOURCES = ["api.cu", "decode.cu", "art.cu", "merge.cu", "select.cu", "chunk.cu", "static_ws.cu",
-           "route.cu", "select2.cu"]
+           "route.cu", "select2.cu", "prefetch.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared"]
 

@@ -152,7 +152,7 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     const long long max_ctas = (long long)num_sms() * decode_ctas_per_sm(G);
     pl->n_ctas = (int)std::max<long long>(1, std::min<long long>(max_ctas, cdiv(t_est, 4)));
     const long long slots = pl->n_ctas + groups;
-    pl->hdr_bytes = (size_t)cdiv((a->batch + 2) * 4ll, 256) * 256;
+    pl->hdr_bytes = (size_t)cdiv(groups * 4ll, 256) * 256;  // one arrival counter per KV group
     pl->ws_bytes = pl->hdr_bytes + (size_t)slots * pl->nw * G * kRecFloats * sizeof(float);
   } else {
     // one cluster of `splits` CTAs per group, merged in distributed shared
@@ -181,7 +181,7 @@ size_t skv_decode_workspace_size(const skv_decode_args* args) {
 int skv_decode_launches(const skv_decode_args* args) {
   Plan pl;
   if (make_plan(args, &pl) != SKV_OK) return 0;
-  return (pl.chunk || (!pl.art && pl.sched == SCHED_SPLIT)) ? 1 : 2;
+  return pl.art ? 2 : 1;
 }
 
 skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* plan) {
@@ -190,7 +190,7 @@ skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* pl
   Plan pl;
   const skv_status st = make_plan(args, &pl);
   if (st != SKV_OK) return st;
-  plan->launches = (pl.chunk || (!pl.art && pl.sched == SCHED_SPLIT)) ? 1 : 2;
+  plan->launches = pl.art ? 2 : 1;
   plan->workspace_bytes = pl.ws_bytes;
   if (pl.chunk) {
     plan->schedule = SKV_SCHED_CHUNK;
@@ -271,13 +271,16 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
   } else {
     p.ws_hdr = reinterpret_cast<int*>(ws);
     p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes);
+    if (pl.sched == SCHED_PERSISTENT &&
+        cudaMemsetAsync(ws, 0, (size_t)a->batch * a->kv_heads * sizeof(int), s) != cudaSuccess)
+      return SKV_ECUDA;
     const unsigned long long wh = g_withhold.exchange(0ull);
     if (wh != 0ull) {
       p.withhold_cta = (int)(wh >> 32);
       p.withhold_entry = (int)(wh & 0xFFFFFFFFull);
     }
     if (launch_decode(p, pl.G, s) != 0) return SKV_ECUDA;
-    if (pl.sched == SCHED_SPLIT) return SKV_OK;  // merged inside the kernel
+    return SKV_OK;  // merged inside the kernel
   }
   if (launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
   return SKV_OK;
@@ -293,7 +296,25 @@ skv_status attn_select_centroids(const void* q, const void* centroids, const int
   if (head_dim != kHeadDim || n_clusters > 4096) return SKV_EUNSUPPORTED;
   if (!aligned16(q) || !aligned16(centroids)) return SKV_EINVAL;
   if (launch_select(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(centroids),
-                    cluster_off, batch, q_heads, kv_heads, n_clusters, topk, sel_ids, seg_start,
+                    cluster_off, batch, q_heads, kv_heads, n_clusters, topk, 0, sel_ids, seg_start,
+                    seg_end, reinterpret_cast<cudaStream_t>(stream)) != 0)
+    return SKV_ECUDA;
+  return SKV_OK;
+}
+
+skv_status attn_select_centroids_shared(const void* q, const void* centroids,
+                                        const int32_t* cluster_off, int batch, int q_heads,
+                                        int kv_heads, int head_dim, int n_clusters, int topk,
+                                        int32_t* sel_ids, int32_t* seg_start, int32_t* seg_end,
+                                        skv_stream_t stream) {
+  if (!q || !centroids || !cluster_off || !sel_ids || !seg_start || !seg_end) return SKV_EINVAL;
+  if (batch < 1 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads != 0) return SKV_EINVAL;
+  if (n_clusters < 1 || topk < 1 || topk > n_clusters) return SKV_EINVAL;
+  if (head_dim != kHeadDim || n_clusters > 4096) return SKV_EUNSUPPORTED;
+  if (batch > 65535 * 8) return SKV_EUNSUPPORTED;
+  if (!aligned16(q) || !aligned16(centroids)) return SKV_EINVAL;
+  if (launch_select(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(centroids),
+                    cluster_off, batch, q_heads, kv_heads, n_clusters, topk, 1, sel_ids, seg_start,
                     seg_end, reinterpret_cast<cudaStream_t>(stream)) != 0)
     return SKV_ECUDA;
   return SKV_OK;
@@ -307,6 +328,51 @@ skv_status attn_merge_lse(const float* o_parts, const float* lse_parts, int n_pa
   if (!aligned16(o_parts) || !aligned16(out)) return SKV_EINVAL;
   if (launch_merge(o_parts, lse_parts, n_parts, n_rows, head_dim, out, lse,
                    reinterpret_cast<cudaStream_t>(stream)) != 0)
+    return SKV_ECUDA;
+  return SKV_OK;
+}
+
+skv_status attn_forecast(const void* x, const void* w, int batch, int kv_heads, int head_dim, void* f,
+                         skv_stream_t stream) {
+  if (!x || !w || !f) return SKV_EINVAL;
+  if (batch < 1 || kv_heads < 1 || batch > 65535 || kv_heads > 65535) return SKV_EINVAL;
+  if (head_dim != kHeadDim) return SKV_EUNSUPPORTED;
+  if (launch_forecast(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w), batch, kv_heads,
+                      static_cast<uint16_t*>(f), reinterpret_cast<cudaStream_t>(stream)) != 0)
+    return SKV_ECUDA;
+  return SKV_OK;
+}
+
+skv_status skv_host_device_pointer(const void* host, void** dev) {
+  if (!host || !dev) return SKV_EINVAL;
+  void* p = nullptr;
+  if (cudaHostGetDevicePointer(&p, const_cast<void*>(host), 0) != cudaSuccess || !p) {
+    cudaGetLastError();  // the failed query's error is not sticky: clear it
+    return SKV_EINVAL;
+  }
+  *dev = p;
+  return SKV_OK;
+}
+
+skv_status attn_prefetch_blocks(const void* k_host, const void* v_host, const int32_t* block_table,
+                                const int32_t* seq_lens, const int32_t* block_ids, int batch,
+                                int kv_heads, int head_dim, int topk, int max_blocks, int num_pages,
+                                int max_seq_len, void* k_cache, void* v_cache, int32_t* seg_start,
+                                int32_t* seg_end, uint32_t* status_word, int n_ctas,
+                                skv_stream_t stream) {
+  if (!k_host || !v_host || !block_table || !seq_lens || !block_ids || !k_cache || !v_cache ||
+      !seg_start || !seg_end)
+    return SKV_EINVAL;
+  if (batch < 1 || kv_heads < 1 || topk < 1 || max_blocks < 0 || num_pages < 1 || max_seq_len < 0 ||
+      n_ctas < 1 || n_ctas > 65535)
+    return SKV_EINVAL;
+  if (head_dim != kHeadDim) return SKV_EUNSUPPORTED;
+  if ((long long)max_blocks * kBlock < (long long)max_seq_len) return SKV_EINVAL;
+  if (!aligned16(k_host) || !aligned16(v_host) || !aligned16(k_cache) || !aligned16(v_cache))
+    return SKV_EINVAL;
+  if (launch_gather(k_host, v_host, block_table, seq_lens, block_ids, batch, kv_heads, topk, max_blocks,
+                    num_pages, max_seq_len, k_cache, v_cache, seg_start, seg_end, status_word, n_ctas,
+                    reinterpret_cast<cudaStream_t>(stream)) != 0)
     return SKV_ECUDA;
   return SKV_OK;
 }

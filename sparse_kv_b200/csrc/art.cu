@@ -886,8 +886,12 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     const unsigned char* sK = smem + s * C::STAGE_BYTES;
     const unsigned char* sV = sK + kTileBytes;
     const int nv = n - rb;
-    if (nv >= C::RPW) fold_tile<G, NW, false>(W, sK, sV, nv, done_mask, pbuf, abuf);
-    else fold_tile<G, NW, true>(W, sK, sV, nv, done_mask, pbuf, abuf);
+    if (!fix) {  // the common path: every head folds the tile (a constant mask)
+      if (nv >= C::RPW) fold_tile<G, NW, false>(W, sK, sV, nv, 0u, pbuf, abuf);
+      else fold_tile<G, NW, true>(W, sK, sV, nv, 0u, pbuf, abuf);
+    } else {     // a re-fold: only the stopping heads fold
+      fold_tile<G, NW, true>(W, sK, sV, nv, done_mask, pbuf, abuf);
+    }
     release();
     const int pos = mt.w & 0xFF;
     if (!fix) {

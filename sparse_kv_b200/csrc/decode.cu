@@ -12,12 +12,14 @@
 // online-softmax state (m, l, O) for the G query heads of the group (the warp
 // arithmetic is in tile.cuh).
 //
-// Schedules.  Index-based traversals run persistently: one CTA per SM takes
-// an even share of the concatenated tile lists of all KV groups (a share may
+// Schedules.  Long index-based walks run persistently: two CTAs per SM take
+// even shares of the concatenated tile lists of all KV groups (a share may
 // span group boundaries; consumers then write a partial record per warp and
-// start the next group without any CTA-wide synchronisation).  Segment lists
-// split each group across a fixed number of CTAs.  Both end with an exact
-// merge of the per-warp records (launch_merge_records).
+// start the next group without any CTA-wide synchronisation).  Each warp
+// arrives on its group's counter after writing its record, and the last
+// arrival merges the group's records into the output, so one launch does the
+// whole walk.  Small walks and segment lists split each group across a
+// thread-block cluster and merge in distributed shared memory.
 #include "common.cuh"
 #include "decode.cuh"
 #include "tile.cuh"
@@ -49,13 +51,9 @@ struct Trav {
   int ra, re;      // natural / range token interval
   int A, Rs, nt1;  // window: [0, A) then [Rs, L)
   const int* ord;
-  // segments
-  const int* ss;
-  const int* se;
-  int seg_i, seg_end_i, seg_pos, seg_stop;
 
-  // Whole traversal of group (b, kvh), then narrowed with set_range
-  // (index-based modes: tile indices; segments: segment indices).
+  // Whole traversal of group (b, kvh), then narrowed with set_range (tile
+  // indices).  Segment lists are walked by the producer warp directly.
   __device__ void init(const DecodeParams& p, int b, int kvh, int L_, int split) {
     mode = p.mode;
     L = L_;
@@ -63,7 +61,6 @@ struct Trav {
     bt = p.block_table + (size_t)b * p.max_blocks;
     num_pages = p.num_pages;
     ord = nullptr;
-    seg_pos = seg_stop = 0;
     const int grp = b * p.Hkv + kvh;
     int N = 0;
     if (mode == TRAV_NATURAL) {
@@ -82,75 +79,20 @@ struct Trav {
     } else if (mode == TRAV_ORDER) {
       ord = p.order + (size_t)grp * p.order_len;
       N = p.order_len;
-    } else {  // segments
-      ss = p.seg_start + (size_t)grp * p.n_seg;
-      se = p.seg_end + (size_t)grp * p.n_seg;
-      N = p.n_seg;
     }
     const int S = p.n_splits > 0 ? p.n_splits : 1;
     set_range((int)(((long long)split * N) / S), (int)(((long long)(split + 1) * N) / S));
   }
 
   __device__ void set_range(int lo, int hi) {
-    if (mode == TRAV_SEGMENTS) {
-      seg_i = lo;
-      seg_end_i = hi;
-      seg_pos = seg_stop = 0;
-    } else {
-      i = lo;
-      i_end = hi;
-    }
-  }
-
-  // Segment lists: the next piece = up to 64 consecutive tokens inside one
-  // page (page, first row, rows).  Used to pack several segments into one tile.
-  __device__ bool next_piece(int& page, int& r0, int& cnt, uint32_t* status) {
-    while (true) {
-      if (seg_pos >= seg_stop) {
-        if (seg_i >= seg_end_i) return false;
-        const int s = ss[seg_i], t = se[seg_i];
-        ++seg_i;
-        if (s > t) {
-          dev_error(status, SKV_DEV_BAD_SEGMENT);
-          continue;
-        }
-        seg_pos = max(s, 0);
-        seg_stop = min(t, L);
-        continue;
-      }
-      const int blk = seg_pos / kBlock;
-      r0 = seg_pos % kBlock;
-      cnt = min(kBlock - r0, seg_stop - seg_pos);
-      seg_pos += cnt;
-      page = bt[blk];
-      if (page < 0 || page >= num_pages) {
-        dev_error(status, SKV_DEV_BAD_PAGE);
-        continue;
-      }
-      return true;
-    }
+    i = lo;
+    i_end = hi;
   }
 
   __device__ bool next(int& t0, int& n, int& pg1, int& pg2, int& n1, uint32_t* status) {
     while (true) {
       int a, e;
-      if (mode == TRAV_SEGMENTS) {
-        if (seg_pos >= seg_stop) {
-          if (seg_i >= seg_end_i) return false;
-          int s = ss[seg_i], t = se[seg_i];
-          ++seg_i;
-          if (s > t) {
-            dev_error(status, SKV_DEV_BAD_SEGMENT);
-            continue;
-          }
-          seg_pos = max(s, 0);
-          seg_stop = min(t, L);
-          continue;
-        }
-        a = seg_pos;
-        e = min(seg_pos + kBlock, seg_stop);
-        seg_pos = e;
-      } else if (mode == TRAV_ORDER) {
+      if (mode == TRAV_ORDER) {
         if (i >= i_end) return false;
         const int j = ord[i++];
         if (j < 0 || j >= nb) {
@@ -258,8 +200,86 @@ struct Cfg {
   static_assert((kRecFloats * 4) % 16 == 0, "record strides");
 };
 
+// Persistent schedule: warp `lane`'s share of the arrival on group g's counter
+// after the warp wrote its record; the warp whose arrival completes every warp
+// of every CTA whose share meets g's tiles merges g's records into the output
+// rows (the "Pulsar Attention" Phase 2 combination, in base 2).  Kept out of
+// line: it runs once per group piece, away from the fold's registers.
+__device__ __noinline__ void merge_group_if_last(const DecodeParams& p, const int* pre, int g, int G,
+                                                 int NW, int lane) {
+  __syncwarp();
+  int last = 0, c0 = 0, c1 = -1;
+  const int b = g / p.Hkv, kvh = g % p.Hkv;
+  const long long T = pre[p.B], P = p.n_ctas;
+  if (lane == 0) {
+    const int nt = (pre[b + 1] - pre[b]) / p.Hkv;
+    const long long Tg = pre[b] + (long long)kvh * nt;
+    c0 = (int)(((Tg + 1) * P - 1) / T);
+    c1 = (int)(((Tg + nt) * P - 1) / T);
+    int ncta = 0;  // CTAs in [c0, c1] with a non-empty share
+    for (int c = c0; c <= c1; ++c) ncta += ((long long)c * T) / P != ((long long)(c + 1) * T) / P;
+    __threadfence();  // this warp's record, before its arrival
+    const int old = atomicAdd(p.ws_hdr + g, 1);
+    last = old == ncta * NW - 1;
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  c0 = __shfl_sync(0xffffffffu, c0, 0);
+  c1 = __shfl_sync(0xffffffffu, c1, 0);
+  __threadfence();  // every arrival came after its record: read them from L2
+  const int nrec = (c1 - c0 + 1) * NW;
+  for (int h = 0; h < G; ++h) {
+    // pass 1: lane r holds record r's (m, l, tiles); max of m over the records
+    float M = -INFINITY;
+    int tiles = 0;
+    for (int r0 = 0; r0 < nrec; r0 += 32) {
+      const int r = r0 + lane;
+      const int c = c0 + r / NW;
+      if (r < nrec && ((long long)c * T) / P != ((long long)(c + 1) * T) / P) {
+        const float4 ml = __ldcg(reinterpret_cast<const float4*>(
+            p.ws_rec + (((size_t)(c + g) * NW + r % NW) * G + h) * kRecFloats + 128));
+        if (ml.y > 0.f) M = fmaxf(M, ml.x);
+        if (r % NW == 0) tiles += (int)ml.z;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+    }
+    // pass 2: W = sum l 2^(m - M), O = sum O 2^(m - M); the lane owns dims 4 lane .. 4 lane + 3
+    float Wl = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      for (int r = 0; r < nrec; ++r) {
+        const int c = c0 + r / NW;
+        if (((long long)c * T) / P == ((long long)(c + 1) * T) / P) continue;
+        const float* rec = p.ws_rec + (((size_t)(c + g) * NW + r % NW) * G + h) * kRecFloats;
+        const float4 ml = __ldcg(reinterpret_cast<const float4*>(rec + 128));
+        if (!(ml.y > 0.f)) continue;
+        const float f = exp2f(ml.x - M);
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(rec + lane * 4));
+        Wl += ml.y * f;
+        acc.x += x.x * f;
+        acc.y += x.y * f;
+        acc.z += x.z * f;
+        acc.w += x.w * f;
+      }
+    }
+    const size_t row = (size_t)b * p.Hq + (size_t)kvh * G + h;
+    const float inv = (Wl > 0.f) ? 1.f / Wl : 0.f;
+    *reinterpret_cast<float4*>(p.out + row * kHeadDim + lane * 4) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (lane == 0) {
+      p.lse[row] = (Wl > 0.f) ? (M + log2f(Wl)) * 0.6931471805599453f : -INFINITY;
+      if (p.blocks_consumed) p.blocks_consumed[row] = tiles;
+    }
+  }
+}
+
 template <int G, int NW, int MINB>
-__global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB)
+    decode_kernel(const __grid_constant__ DecodeParams p) {
   using C = Cfg<G, NW, MINB>;
   constexpr int ST = C::STAGES;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -327,12 +347,23 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       }
       if (lane == 0) pre[p.B] = run;
       __syncwarp();
+      // sequences without a tile belong to no CTA's share: CTA 0 writes their
+      // (empty) results
       if (blockIdx.x == 0) {
-        if (lane == 0) p.ws_hdr[0] = run;
-        for (int b = lane; b <= p.B; b += 32) p.ws_hdr[1 + b] = pre[b];
+        for (int r = lane; r < p.B * p.Hq; r += 32) {
+          const int b = r / p.Hq;
+          if (pre[b + 1] != pre[b]) continue;
+          float4* o = reinterpret_cast<float4*>(p.out + (size_t)r * kHeadDim);
+          for (int j = 0; j < kHeadDim / 4; ++j) o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          p.lse[r] = -INFINITY;
+          if (p.blocks_consumed) p.blocks_consumed[r] = 0;
+        }
       }
     }
-    if (lane != 0) return;
+    // Segment lists are walked by the whole warp (bounds and pages fetched for
+    // 32 segments at a time); every other traversal by lane 0 alone.
+    const bool seg_mode = p.mode == TRAV_SEGMENTS;
+    if (lane != 0 && !seg_mode) return;
 
     const uint64_t pol = policy_evict_first();
     const size_t head_stride = (size_t)kBlock * kHeadDim;
@@ -424,38 +455,96 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       }
       return true;
     };
-    auto run_segments = [&](Trav& tr, int g, int slot, int kvh) -> bool {
+    // Segment lists (whole warp): lane i loads the bounds of segment base + i
+    // and the pages of its first and last block, so one round trip to memory
+    // serves 32 segments; lane 0 then packs their rows into full 64-row tiles
+    // (attention over a key set does not depend on the keys' order), one bulk
+    // copy per piece (<= 64 consecutive tokens of one page).  Pages inside a
+    // segment longer than two blocks are looked up as lane 0 reaches them.
+    auto run_segments_warp = [&](int b, int kvh, int L, int g, int slot, int split) -> bool {
+      const int grp = b * p.Hkv + kvh;
+      const int* ss = p.seg_start + (size_t)grp * p.n_seg;
+      const int* se = p.seg_end + (size_t)grp * p.n_seg;
+      const int* bt = p.block_table + (size_t)b * p.max_blocks;
+      const int S = p.n_splits > 0 ? p.n_splits : 1;
+      const int lo = (int)(((long long)split * p.n_seg) / S);
+      const int hi = (int)(((long long)(split + 1) * p.n_seg) / S);
       int pg[kMaxPieces], r0[kMaxPieces], cnt[kMaxPieces];
       int np = 0, rows = 0, tiles = 0;
-      int page = 0, first = 0, c = 0;
-      while (tr.next_piece(page, first, c, p.status)) {
-        while (c > 0) {
-          const int take = min(c, kBlock - rows);
-          pg[np] = page;
-          r0[np] = first;
-          cnt[np] = take;
-          ++np;
-          rows += take;
-          first += take;
-          c -= take;
-          if (rows == kBlock || np == kMaxPieces) {
-            if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
-            ++tiles;
-            np = rows = 0;
+      bool ok = true;
+      for (int base = lo; base < hi && ok; base += 32) {
+        const int i = base + lane;
+        int s0 = 0, s1 = 0, pa = 0, pb = 0;
+        if (i < hi) {
+          const int a = ss[i], e2 = se[i];
+          if (a > e2) dev_error(p.status, SKV_DEV_BAD_SEGMENT);
+          else {
+            s0 = max(a, 0);
+            s1 = min(e2, L);
+          }
+          if (s1 > s0) {
+            pa = bt[s0 / kBlock];
+            pb = bt[(s1 - 1) / kBlock];
+          } else {
+            s1 = s0;
+          }
+        }
+        const int n_in = min(32, hi - base);
+        for (int j = 0; j < n_in; ++j) {
+          const int a = __shfl_sync(0xffffffffu, s0, j), z = __shfl_sync(0xffffffffu, s1, j);
+          const int qa = __shfl_sync(0xffffffffu, pa, j), qb = __shfl_sync(0xffffffffu, pb, j);
+          int good = 1;
+          if (lane == 0) {
+            const int fb = a / kBlock, lb = (z - 1) / kBlock;
+            for (int pos = a; pos < z && good;) {
+              const int blk = pos / kBlock, first = pos % kBlock;
+              int c = min(kBlock - first, z - pos);
+              pos += c;
+              const int page = blk == fb ? qa : (blk == lb ? qb : bt[blk]);
+              if (page < 0 || page >= p.num_pages) {
+                dev_error(p.status, SKV_DEV_BAD_PAGE);
+                continue;
+              }
+              int f = first;
+              while (c > 0) {
+                const int take = min(c, kBlock - rows);
+                pg[np] = page;
+                r0[np] = f;
+                cnt[np] = take;
+                ++np;
+                rows += take;
+                f += take;
+                c -= take;
+                if (rows == kBlock || np == kMaxPieces) {
+                  if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) {
+                    good = 0;
+                    break;
+                  }
+                  ++tiles;
+                  np = rows = 0;
+                }
+              }
+            }
+          }
+          if (!__shfl_sync(0xffffffffu, good, 0)) {
+            ok = false;
+            break;
           }
         }
       }
-      if (rows > 0) {
-        if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
-        ++tiles;
+      int r = ok ? 1 : 0;
+      if (lane == 0 && ok) {
+        if (rows > 0) {
+          if (emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) ++tiles;
+          else r = 0;
+        }
+        if (r && tiles == 0 && !emit(0, g, slot, kvh, 0, 0, 0, 0)) r = 0;
       }
-      if (tiles == 0 && !emit(0, g, slot, kvh, 0, 0, 0, 0)) return false;
-      return true;
+      return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
     // All entries of one group segment; a segment without valid tiles still
     // issues a marker so that the consumers account for the group.
     auto run_group = [&](Trav& tr, int g, int slot, int kvh) -> bool {
-      if (tr.mode == TRAV_SEGMENTS) return run_segments(tr, g, slot, kvh);
       int t0 = 0, n = 0, pg1 = 0, pg2 = 0, n1 = 0, cnt = 0;
       while (tr.next(t0, n, pg1, pg2, n1, p.status)) {
         if (!emit(n, g, slot, kvh, t0, pg1, pg2, n1)) return false;
@@ -493,14 +582,19 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
       int L = p.seq_lens[b];
       if (L < 0 || L > p.max_seq_len) {
-        if (split == 0 && kvh == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
+        if (split == 0 && kvh == 0 && lane == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
         L = 0;
       }
-      Trav tr;
-      tr.init(p, b, kvh, L, split);
       const int g = b * p.Hkv + kvh;
-      ok = run_group(tr, g, g * p.n_splits + split, kvh);
+      if (seg_mode) {
+        ok = run_segments_warp(b, kvh, L, g, g * p.n_splits + split, split);
+      } else {
+        Trav tr;
+        tr.init(p, b, kvh, L, split);
+        ok = run_group(tr, g, g * p.n_splits + split, kvh);
+      }
     }
+    if (lane != 0) return;
     if (ok) emit(-1, -1, 0, 0, 0, 0, 0, 0);
     // Copies the consumers never waited for (abort) must land before the CTA
     // exits: learn how many entries they consumed, then drain the rest.
@@ -537,6 +631,11 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     }
   };
 
+  // Persistent schedule: after its record of group g, a warp arrives on g's
+  // counter; the last arrival merges g (merge_group_if_last).
+  const int* pre = reinterpret_cast<const int*>(smem + C::OFF_PRE);
+  auto arrive_and_merge = [&](int g) { merge_group_if_last(p, pre, g, G, NW, lane); };
+
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P) + warp * C::RPW * G;
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
 
@@ -561,7 +660,10 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       break;
     }
     if (mt.y != cur_g) {
-      if (cur_g >= 0) flush(cur_slot, k);
+      if (cur_g >= 0) {
+        flush(cur_slot, k);
+        if (p.sched == SCHED_PERSISTENT) arrive_and_merge(cur_g);
+      }
       W.reset();
       const int b = mt.y / p.Hkv, kvh = mt.y % p.Hkv;
       W.load_q(p.q, (size_t)b * p.Hq + (size_t)kvh * G, p.qscale, lane);
@@ -587,7 +689,10 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
 
   // ------------------------------------------------------------------ epilogue
   if (p.sched == SCHED_PERSISTENT) {
-    if (cur_g >= 0) flush(cur_slot, k);
+    if (cur_g >= 0) {
+      flush(cur_slot, k);
+      arrive_and_merge(cur_g);
+    }
     // Every consumer warp ends here: let the producer know once all are done.
     __syncwarp();
     mbar_arrive_if(fin_bar, lane == 0);

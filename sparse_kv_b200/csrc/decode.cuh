@@ -49,8 +49,9 @@ struct DecodeParams {
   float* lse;
   int* blocks_consumed;
   uint32_t* status;
-  // Non-ART workspace: header (total tiles, batch prefix) and per-warp partial
-  // records [slots][rec_nw][G][kRecFloats], merged by launch_merge_records.
+  // Persistent schedule's workspace: one arrival counter per KV group (zeroed
+  // before every launch) and per-warp partial records [slots][rec_nw][G][kRecFloats];
+  // the last warp to arrive for a group merges its records.
   int* ws_hdr;
   float* ws_rec;
   int rec_nw;
@@ -122,7 +123,13 @@ int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int
 int launch_merge_records(const DecodeParams& p, int G, void* stream);
 int launch_chunk(const DecodeParams& p, int Tq, int causal, int n_shards, void* stream);
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
-                  int C, int k, int* ids, int* ss, int* se, void* stream);
+                  int C, int k, int shared, int* ids, int* ss, int* se, void* stream);
+int select_cluster_size(int groups_or_B, int C, int shared);
+int launch_forecast(const uint16_t* x, const uint16_t* w, int B, int Hkv, uint16_t* f, void* stream);
+int launch_gather(const void* k_host, const void* v_host, const int* block_table, const int* seq_lens,
+                  const int* ids, int B, int Hkv, int k, int max_blocks, int num_pages, int max_seq_len,
+                  void* k_cache, void* v_cache, int* seg_start, int* seg_end, uint32_t* status,
+                  int n_ctas, void* stream);
 int num_sms();
 
 }  // namespace skv

@@ -149,7 +149,7 @@ def test_workspace_size_query():
     L = skv.lib()
     full = good_args()
     n = L.skv_decode_workspace_size(ctypes.byref(full))
-    # header (batch prefix) + per-warp partial records of 132 floats per head
+    # arrival counters + per-warp partial records of 132 floats per head
     assert n > 0 and (n % 256) == 0 and n >= 16 * 8 * 16 * 4 * 132 * 4
     # ART: per (chunk, KV group): a look-back record of 12 floats and a partial
     # record of 132 floats per head, zeroed control words, and a scratch area of
@@ -169,12 +169,13 @@ def test_workspace_size_query():
 
 
 def test_decode_launch_count():
-    # one kernel where the walk merges its own partials (small walks and
-    # segment lists take the split schedule; a query chunk writes its results
-    # directly), two where a record merge follows (large walks, ART)
+    # one kernel where the walk merges its own partials (large walks: the last
+    # arrival per group merges; small walks and segment lists: the cluster's
+    # shared memory; a query chunk writes its results directly), two where a
+    # record merge follows (ART)
     L = skv.lib()
     n = lambda a: L.skv_decode_launches(ctypes.byref(a))
-    assert n(good_args()) == 2                                    # 128 groups x 512 tiles
+    assert n(good_args()) == 1                                    # 128 groups x 512 tiles
     assert n(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == 2
     small = good_args(batch=1, q_heads=8, kv_heads=2, max_seq_len=4096, max_blocks=64)
     assert n(small) == 1                                          # 2 groups x 64 tiles
@@ -247,14 +248,15 @@ def test_strerror():
 def test_plan_small_walks_take_the_cluster_schedule():
     # up to 8 tiles per resident CTA (148 SMs x 2 CTAs here) the walk runs as
     # one cluster per KV group and merges in-kernel; one tile more, and the
-    # persistent schedule with its record merge takes over
+    # persistent schedule (arrival counters and per-warp records in the
+    # workspace, merged by each group's last arrival) takes over
     L = skv.lib()
     small = 148 * 2 * 8  # tiles
     a = good_args(batch=1, q_heads=4, kv_heads=1, max_seq_len=small * 64, max_blocks=small)
     assert L.skv_decode_launches(ctypes.byref(a)) == 1
     assert L.skv_decode_workspace_size(ctypes.byref(a)) == 0
     b = good_args(batch=1, q_heads=4, kv_heads=1, max_seq_len=(small + 1) * 64, max_blocks=small + 1)
-    assert L.skv_decode_launches(ctypes.byref(b)) == 2
+    assert L.skv_decode_launches(ctypes.byref(b)) == 1
     assert L.skv_decode_workspace_size(ctypes.byref(b)) > 0
 
 
@@ -299,7 +301,7 @@ def test_decode_plan_info():
         return p
 
     full = plan(good_args())  # 16 x 8 groups of 512 tiles
-    assert (full.schedule, full.ctas, full.splits, full.launches) == (0, 296, 0, 2)
+    assert (full.schedule, full.ctas, full.splits, full.launches) == (0, 296, 0, 1)
     assert full.workspace_bytes == L.skv_decode_workspace_size(ctypes.byref(good_args()))
     art = plan(good_args(art=_Art(1, 1e-3, 1e-4, 4)))
     assert (art.schedule, art.ctas, art.art_chunk_blocks, art.art_chunks, art.launches) == (2, 296, 16, 32, 2)
@@ -353,3 +355,31 @@ def test_withhold_hook_validates_and_clears():
     assert L.skv_test_withhold_tile(0, -1) == skv.SKV_EINVAL
     assert L.skv_test_withhold_tile(3, 2) == skv.SKV_OK
     assert L.skv_test_withhold_tile(-1, 0) == skv.SKV_OK  # clears the pending hook
+
+
+def _plan_bytes(B, Hq, Hkv, L, **kw):
+    import torch
+    import sparse_kv_b200 as skv
+    q = torch.zeros(B, 1, Hq, 128, dtype=torch.bfloat16)
+    pool = torch.zeros(2, Hkv, 64, 128, dtype=torch.bfloat16)
+    bt = torch.zeros(B, (L + 63) // 64, dtype=torch.int32)
+    sl = torch.zeros(B, dtype=torch.int32)
+    return skv.decode_workspace_size(q, pool, pool, bt, sl, torch.zeros(B, 1, Hq, 128), torch.zeros(B, 1, Hq),
+                                     max_seq_len=L, **kw)
+
+
+def test_static_workspace_holds_the_stated_shapes():
+    """The allocation-free entry point's array holds what the header promises
+    (148 SMs, as planned without a GPU): ART at the Llama shape for 64 x 32K and
+    16 x 128K (the cfg2 and cfg5 ART layers among them) and the persistent
+    schedule for 3,600 KV groups at G = 4; and refuses a larger ART call."""
+    import re
+    src = open(os.path.join(ROOT, "include", "sparsekv.h")).read()
+    m = re.search(r"#define SKV_STATIC_WORKSPACE_BYTES \((\d+)u \* 1024u \* 1024u\)", src)
+    cap = int(m.group(1)) * 1024 * 1024
+    art = dict(art=(1e-3, 1e-4, 4))
+    for B, L in [(16, 32768), (8, 131072), (64, 32768), (16, 131072)]:
+        assert 0 < _plan_bytes(B, 32, 8, L, **art) <= cap, (B, L)
+    assert _plan_bytes(450, 32, 8, 32768) <= cap        # 3,600 KV groups, no ART
+    assert _plan_bytes(225, 64, 8, 32768) <= cap        # 1,800 KV groups at G = 8
+    assert _plan_bytes(32, 32, 8, 131072, **art) > cap  # beyond: SKV_EWORKSPACE

@@ -351,6 +351,39 @@ def test_select_uses_sum_over_group_heads():
     np.testing.assert_array_equal(sc[0], [0, 1, 0])
 
 
+def test_select_shared_is_each_requests_own_selection_brute_force():
+    """Shared fixed context ("Squeezed Attention" Q1): every request ranks the
+    same centroids with its own summed query.  Checked against scores written
+    out as explicit sums and a ranking by (score desc, id asc), per request."""
+    rng = np.random.default_rng(7)
+    U, G, d, C, k = 5, 2, 8, 20, 6
+    q = bf16_bits(rng.integers(-3, 4, size=(U, G, d)).astype(np.float64))
+    cent = bf16_bits(rng.integers(-2, 3, size=(C, d)).astype(np.float64))  # many exact ties
+    ids, sc = oracle.select_shared(q, cent, k)
+    qv = skvgen.bf16_to_f64(q)
+    cv = skvgen.bf16_to_f64(cent)
+    for u in range(U):
+        score = [sum(sum(qv[u, g, j] for g in range(G)) * cv[c, j] for j in range(d)) for c in range(C)]
+        np.testing.assert_array_equal(sc[u], score)
+        best = sorted(range(C), key=lambda c: (-score[c], c))[:k]
+        assert list(ids[u]) == sorted(best)
+
+
+def test_select_shared_identical_and_permuted_requests():
+    rng = np.random.default_rng(8)
+    U, G, d, C, k = 4, 4, 16, 64, 9
+    q = bf16_bits(rng.standard_normal((U, G, d)))
+    cent = bf16_bits(rng.standard_normal((C, d)))
+    ids, _ = oracle.select_shared(q, cent, k)
+    q2 = q.copy()
+    q2[2] = q2[0]                         # two identical requests choose identically
+    ids2, _ = oracle.select_shared(q2, cent, k)
+    np.testing.assert_array_equal(ids2[2], ids2[0])
+    perm = [3, 1, 0, 2]                   # the requests' order does not matter
+    ids3, _ = oracle.select_shared(q[perm], cent, k)
+    np.testing.assert_array_equal(ids3, ids[perm])
+
+
 def test_select_all_clusters_is_full_attention():
     wl = skvgen.Workload("tiny-mix", B=1, Hq=4, Hkv=1, L=700, c_log2=4, mixture=True, seed=99)
     K, off, cent = skvgen.host_mixture_group(wl, 0, 0)
@@ -545,3 +578,63 @@ def test_oracle_threads_do_not_change_results():
     assert oracle.threads() == n0
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+# ----------------------------------------------------------------------------- lookahead (Forecast)
+
+def test_forecast_one_hot_weights_read_one_input():
+    rng = np.random.default_rng(11)
+    d = 128
+    x = bf16_bits(rng.standard_normal((3, d)))
+    perm = rng.permutation(d)
+    w = np.zeros((3, d, d))
+    w[:, perm, np.arange(d)] = 1.0             # output j reads input perm[j]
+    f = oracle.forecast(x, bf16_bits(w))
+    np.testing.assert_array_equal(f, x[:, perm])
+
+
+def test_forecast_small_integers_are_exact():
+    rng = np.random.default_rng(12)
+    d = 128
+    x = rng.integers(-2, 3, size=(4, d))
+    w = rng.integers(-1, 2, size=(4, d, d))
+    f = oracle.forecast(bf16_bits(x.astype(float)), bf16_bits(w.astype(float)))
+    exact = np.einsum("uij,ui->uj", w, x)      # |sum| <= 256: exact in bf16
+    np.testing.assert_array_equal(skvgen.bf16_to_f64(f), exact)
+
+
+def test_forecast_sums_in_fp32_in_input_order_and_rounds_to_nearest_even():
+    d = 128
+    x = np.zeros((3, d))
+    w = np.zeros((3, d, d))
+    # 2^24 + 1 rounds to 2^24 in fp32, then - 2^24 gives 0 (another order gives 1)
+    x[0, :3] = [2.0 ** 24, 1.0, -(2.0 ** 24)]
+    w[0, :3, 0] = 1.0
+    # 1 + 2^-8 is halfway between two bf16 values: to the even one, 1.0;
+    # 1 + 3 * 2^-8 is halfway too: to the even one, 1 + 2^-6
+    x[1, :2] = [1.0, 2.0 ** -8]
+    w[1, :2, 0] = 1.0
+    x[2, :2] = [1.0, 3 * 2.0 ** -8]
+    w[2, :2, 0] = 1.0
+    f = skvgen.bf16_to_f64(oracle.forecast(bf16_bits(x), bf16_bits(w)))
+    assert f[0, 0] == 0.0
+    assert f[1, 0] == 1.0
+    assert f[2, 0] == 1.0 + 2.0 ** -6
+
+
+def test_forecast_close_to_the_exact_projection():
+    rng = np.random.default_rng(13)
+    d = 128
+    x = bf16_bits(rng.standard_normal((5, d)))
+    w = bf16_bits(rng.standard_normal((5, d, d)) / 16)
+    f = skvgen.bf16_to_f64(oracle.forecast(x, w))
+    ref = np.einsum("uij,ui->uj", skvgen.bf16_to_f64(w), skvgen.bf16_to_f64(x))
+    # one bf16 rounding (relative 2^-8) plus fp32 accumulation error
+    bound = np.abs(ref) * 2.0 ** -8 + d * 2.0 ** -23 * np.einsum(
+        "uij,ui->uj", np.abs(skvgen.bf16_to_f64(w)), np.abs(skvgen.bf16_to_f64(x)))
+    assert np.all(np.abs(f - ref) <= bound)
+
+
+def test_keys_blocks_short_last_block():
+    np.testing.assert_array_equal(oracle.keys_blocks([2, 0, -1], 150),
+                                  np.r_[np.arange(0, 64), np.arange(128, 150)])
