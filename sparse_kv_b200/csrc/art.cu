@@ -34,8 +34,8 @@
 //              warp ballots) and publishes the inclusive prefix; only then does
 //              it reduce the warps' states into the chunk's record, which no
 //              decision needs.
-// Posts alternate between two buffers, so the consumers run a chunk ahead of
-// the arbiter.  The probes and states live in global memory rewritten in place
+// Posts rotate through kPosts buffers, so the consumers run up to kPosts - 1
+// chunks ahead of the arbiter, which may wait on other CTAs' look-back.  The probes and states live in global memory rewritten in place
 // (they stay in L2), which leaves the shared memory to a 3-stage ring at two
 // CTAs per SM.
 // A head that stops inside a chunk needs its state after the stop block, which
@@ -60,6 +60,11 @@
 #ifndef SKV_ART_CTAS_PER_SM
 #define SKV_ART_CTAS_PER_SM 2
 #endif
+// post buffers between the consumers and the arbiter: the consumers run up to
+// SKV_ART_POSTS - 1 chunks ahead of the arbiter's decisions
+#ifndef SKV_ART_POSTS
+#define SKV_ART_POSTS 3
+#endif
 
 namespace skv {
 namespace {
@@ -75,16 +80,18 @@ constexpr int kFixTag = 1 << 30;
 constexpr int kDrainEntry = -2;  // meta.x of the entry that ends the items (before re-folds)
 
 constexpr size_t up16(size_t x) { return (x + 15) / 16 * 16; }
+constexpr int kPosts = SKV_ART_POSTS;
+static_assert(kPosts >= 2 && kPosts <= 8, "post buffers");
 
-// Per-CTA scratch in global memory, two buffers (post parity): probes
-// [2][CB][NW][G][12] and states [2][NW][G][kRecFloats].
+// Per-CTA scratch in global memory, one buffer per post: probes
+// [kPosts][CB][NW][G][12] and states [kPosts][NW][G][kRecFloats].
 template <int G, int NW, int CB>
 __host__ __device__ constexpr size_t probe_floats() {
   return (size_t)CB * NW * G * kProbeFloats;
 }
 template <int G, int NW, int CB>
 __host__ __device__ constexpr size_t scratch_floats() {
-  return 2 * probe_floats<G, NW, CB>() + 2 * (size_t)NW * G * kRecFloats;
+  return kPosts * probe_floats<G, NW, CB>() + kPosts * (size_t)NW * G * kRecFloats;
 }
 
 template <int G, int NW, int CB, int ST>
@@ -94,12 +101,12 @@ struct ArtCfg {  // shared-memory layout
   static constexpr int THREADS = (NW + 2) * 32;  // consumers, producer, arbiter
   // a stage: K rows, V rows, and the group's q rows (loaded with a chunk's first block)
   static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes + (size_t)G * kRowBytes;
-  static constexpr int NBAR = 2 * ST + 5;  // full, empty, fin, posted[2], free[2]
+  static constexpr int NBAR = 2 * ST + 1 + 2 * kPosts;  // full, empty, fin, posted[], freed[]
   static constexpr size_t OFF_BAR = ST * STAGE_BYTES;
   static constexpr size_t OFF_META = up16(OFF_BAR + NBAR * 8);        // int4 [ST]
   static constexpr size_t OFF_FLAGS = up16(OFF_META + ST * 16);       // int [4]
-  static constexpr size_t OFF_TAG = OFF_FLAGS + 16;                   // int [2][4]
-  static constexpr size_t OFF_REQ = OFF_TAG + 32;                     // int [kReqs][4] + int [kReqs][G]
+  static constexpr size_t OFF_TAG = OFF_FLAGS + 16;                   // int [kPosts][4]
+  static constexpr size_t OFF_REQ = OFF_TAG + 16 * kPosts;            // int [kReqs][4] + int [kReqs][G]
   static constexpr size_t OFF_P = up16(OFF_REQ + kReqs * 16 + (size_t)kReqs * G * 4);  // float2 [NW][RPW][G]
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;   // float2 [NW][G]
   static constexpr size_t OFF_WCTL = up16(OFF_A + (size_t)NW * G * 8);  // int [NW][8]
@@ -163,18 +170,18 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + ST;
   uint64_t* fin_bar = empty + ST;
-  uint64_t* posted = fin_bar + 1;   // [2] a post is ready (one arrival per consumer warp)
-  uint64_t* freed = posted + 2;     // [2] the arbiter is done with a post
+  uint64_t* posted = fin_bar + 1;   // [kPosts] a post is ready (one arrival per consumer warp)
+  uint64_t* freed = posted + kPosts;  // [kPosts] the arbiter is done with a post
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows | 0 = end of chunk, group, chunk, block in chunk | blocks}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   // flags[0]: re-fold requests posted by the arbiter; flags[1]: abort (a bounded
   // wait expired); flags[2]: consumers finished (entries consumed + 1);
   // flags[3]: the arbiter has handled every chunk (no more requests)
-  volatile int* tag = reinterpret_cast<volatile int*>(smem + C::OFF_TAG);    // [2][4]: kind, group, chunk, a
+  volatile int* tag = reinterpret_cast<volatile int*>(smem + C::OFF_TAG);    // [kPosts][4]: kind, group, chunk, a
   volatile int* req = reinterpret_cast<volatile int*>(smem + C::OFF_REQ);  // [kReqs][4]: group, chunk, vmask, stopmask
   volatile int* req_t = reinterpret_cast<volatile int*>(smem + C::OFF_REQ + kReqs * 16);  // [kReqs][G]
-  float* probe = p.art_scratch + (size_t)blockIdx.x * scratch_floats<G, NW, CB>();  // [2][CB][NW][G][12]
-  float* state = probe + 2 * probe_floats<G, NW, CB>();                            // [2][NW][G][132]
+  float* probe = p.art_scratch + (size_t)blockIdx.x * scratch_floats<G, NW, CB>();  // [kPosts][CB][NW][G][12]
+  float* state = probe + kPosts * probe_floats<G, NW, CB>();                       // [kPosts][NW][G][132]
   float* local = reinterpret_cast<float*>(smem + C::OFF_LOCAL);                    // [CB][G][12]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       mbar_init(&empty[s], NW);
     }
     mbar_init(fin_bar, NW);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPosts; ++i) {
       mbar_init(&posted[i], NW);
       mbar_init(&freed[i], 1);
     }
@@ -727,8 +734,8 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     };
 
     while (true) {
-      const int par = kj & 1;
-      if (!mbar_wait_bounded(&posted[par], (kj >> 1) & 1, &flags[1])) {
+      const int par = kj % kPosts;
+      if (!mbar_wait_bounded(&posted[par], (kj / kPosts) & 1, &flags[1])) {
         if (lane == 0) fail();
         break;
       }
@@ -790,20 +797,20 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   wc[W_CURG] = -1;   // item being folded: group, chunk, re-fold slot (-1: the chunk itself)
   wc[W_CURC] = -1;
   wc[W_CURK] = -1;
-  int kpar = 0;  // parity of the next post (its buffers hold the current item)
+  int kpar = 0;  // buffer of the next post (it holds the current item)
   bool ok = true;
 
-  // Take the buffers of the next post (the arbiter is done with the post two back).
+  // Take the buffers of the next post (the arbiter is done with the post kPosts back).
   auto acquire = [&]() {
     const int kp = wc[W_KP];
-    if (kp >= 2 && !mbar_wait_bounded(&freed[kp & 1], ((kp >> 1) - 1) & 1, &flags[1])) {
+    if (kp >= kPosts && !mbar_wait_bounded(&freed[kp % kPosts], ((kp / kPosts) - 1) & 1, &flags[1])) {
       if (lane == 0) fail();
       ok = false;
     }
   };
   auto publish = [&](int kind, int g, int c, int a) {
     const int kp = wc[W_KP];
-    const int par = kp & 1;
+    const int par = kp % kPosts;
     if (warp == 0 && lane == 0) {
       tag[par * 4] = kind;
       tag[par * 4 + 1] = g;
@@ -813,11 +820,11 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     __syncwarp();
     mbar_arrive_if(&posted[par], lane == 0);
     wc[W_KP] = kp + 1;
-    kpar = (kp + 1) & 1;
+    kpar = (kp + 1) % kPosts;
   };
   // this warp's whole state -> the state area of the current post
   auto write_state = [&]() {
-    float* st_area = state + (size_t)(wc[W_KP] & 1) * NW * G * kRecFloats;
+    float* st_area = state + (size_t)(wc[W_KP] % kPosts) * NW * G * kRecFloats;
 #pragma unroll
     for (int g2 = 0; g2 < G; ++g2) {
       float x0, x1, x2, x3;

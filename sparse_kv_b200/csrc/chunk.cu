@@ -417,7 +417,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     bool ok = true;
     for (int j = 0; j < n_tiles && ok; ++j) {
       const int sb = j & 1;
-      if (!mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      // every exit from this loop is taken by the whole warp (warp-wide tcgen05 below)
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
       fence_after_sync();
       const uint32_t col_s = (uint32_t)sb * BN + (uint32_t)ch * HC;  // this half's S columns
       float s[HC];
@@ -452,12 +456,20 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], fmaxf(s[c + u], s[c + 8 + u]));
       const float tmax = p.qscale * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      if (tmax > m_used + 8.f) {  // lazy rescale: only when the max grows by more than 2^8
-        const float alpha = exp2f(m_used - tmax);  // 0 when m_used is -inf
+      // Lazy rescale: only when the max grows by more than 2^8.  The decision is
+      // taken for the whole warp (tcgen05.ld / st are warp-wide instructions and
+      // must not sit in divergent code): if any row of the warp needs it, every
+      // row moves to max(m_used, tmax), which is exact for all of them.
+      if (__any_sync(0xffffffffu, tmax > m_used + 8.f)) {
+        const float m_new = fmaxf(m_used, tmax);
+        // 0 when m_used is -inf; 1 for a row whose max did not grow (and for a
+        // row that has seen no key yet, m_used = m_new = -inf)
+        const float alpha = (m_new == m_used) ? 1.f : exp2f(m_used - m_new);
         l_sum *= alpha;
         if (o_live) {  // O_h must hold every P.V so far: wait for the one of tile j - 1
           const int jp = j - 1;
-          if (!mbar_wait_bounded(&o_done[jp & 1], (jp >> 1) & 1, abort_flag)) {
+          const bool got = mbar_wait_bounded(&o_done[jp & 1], (jp >> 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) {
             ok = false;
             break;
           }
@@ -473,7 +485,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           }
           tmem_wait_st();
         }
-        m_used = tmax;
+        m_used = m_new;
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
       // P_h = 2^(s * scale - m_h), split into two bf16 terms P_h = hi + lo
@@ -524,7 +536,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       if (kp0 < k_lo || kp0 + BN > k_hi) {
         // V(j) must have landed before its rows are cleared (v_full cannot run two
         // phases ahead: its next phase needs the P.V of this tile)
-        if (!mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, abort_flag)) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
