@@ -250,16 +250,16 @@ SKV_API skv_status attn_decode(const skv_decode_args* args, skv_stream_t stream)
  *    other host threads) race on it: serialise them.
  * Errors: as attn_decode, plus SKV_ECUDA if the address lookup fails.
  * What fits in the array (skv_decode_workspace_size on a 148-SM B200): every
- * walk without ART of up to about 3,600 KV groups at 4 query heads per KV
- * head, 1,800 at 8 (the persistent schedule needs about 17 KiB, or 34 KiB,
+ * walk without ART of up to about 5,500 KV groups at 4 query heads per KV
+ * head, 2,800 at 8 (the persistent schedule needs about 17 KiB, or 34 KiB,
  * per resident CTA and per KV group; small walks and segment lists need
  * none), and ART at the Llama-3.1-8B shape (32 query / 8 KV heads) for up to
- * 64 sequences of 32K tokens or 16 of 128K (ART needs 24 to 39 MiB of
+ * 64 sequences of 32K tokens or 16 of 128K (ART needs 36 to 57 MiB of
  * per-CTA scratch plus about 0.6 KiB per (KV group, chunk, query head)).
  * The device address is
  * looked up once per device and kept for the whole process: it assumes the
  * device's primary context is not reset (cudaDeviceReset) in between. */
-#define SKV_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+#define SKV_STATIC_WORKSPACE_BYTES (96u * 1024u * 1024u)
 SKV_API skv_status attn_decode_static_ws(const skv_decode_args* args, skv_stream_t stream);
 
 /* Centroid selection ("Squeezed Attention" Q2 step 2) for each KV group

@@ -273,9 +273,11 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
     # (group, chunk) a look-back record (12 floats) and a partial record (132
     # floats) per head, and per resident CTA (148 SMs x 2) probes of CB blocks
     # x 8 warps x G heads x 12 floats and 8 warps' states of G x 132 floats,
-    # both double-buffered; each of the first two parts rounded up to 256 B.
+    # both once per post buffer; each of the first two parts rounded up to 256 B.
     L = skv.lib()
     G, NW, ctas = 4, 8, 148 * 2
+    src = open(os.path.join(ROOT, "sparse_kv_b200", "csrc", "art.cu")).read()
+    posts = int(re.search(r"#define SKV_ART_POSTS (\d+)", src).group(1))
     a = good_args(batch=groups_b, q_heads=hkv * G, kv_heads=hkv, max_seq_len=blocks * 64, max_blocks=blocks,
                   art=_Art(1, 1e-3, 1e-4, 4))
     n = L.skv_decode_workspace_size(ctypes.byref(a))
@@ -287,7 +289,7 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
         items = groups * maxc
         ctl = up((4 + groups + groups * maxc + 2 * groups * G) * 4)
         lb = up(items * G * 12 * 4)
-        scratch = ctas * (2 * cb * NW * G * 12 + 2 * NW * G * 132) * 4
+        scratch = ctas * (posts * cb * NW * G * 12 + posts * NW * G * 132) * 4
         sizes[cb] = ctl + lb + scratch + items * G * 132 * 4
     assert n == sizes[want_cb], (n, sizes)
 
@@ -372,7 +374,8 @@ def test_static_workspace_holds_the_stated_shapes():
     """The allocation-free entry point's array holds what the header promises
     (148 SMs, as planned without a GPU): ART at the Llama shape for 64 x 32K and
     16 x 128K (the cfg2 and cfg5 ART layers among them) and the persistent
-    schedule for 3,600 KV groups at G = 4; and refuses a larger ART call."""
+    schedule for 5,500 KV groups at G = 4 (2,800 at G = 8); and refuses a
+    larger ART call."""
     import re
     src = open(os.path.join(ROOT, "include", "sparsekv.h")).read()
     m = re.search(r"#define SKV_STATIC_WORKSPACE_BYTES \((\d+)u \* 1024u \* 1024u\)", src)
@@ -380,6 +383,6 @@ def test_static_workspace_holds_the_stated_shapes():
     art = dict(art=(1e-3, 1e-4, 4))
     for B, L in [(16, 32768), (8, 131072), (64, 32768), (16, 131072)]:
         assert 0 < _plan_bytes(B, 32, 8, L, **art) <= cap, (B, L)
-    assert _plan_bytes(450, 32, 8, 32768) <= cap        # 3,600 KV groups, no ART
-    assert _plan_bytes(225, 64, 8, 32768) <= cap        # 1,800 KV groups at G = 8
-    assert _plan_bytes(32, 32, 8, 131072, **art) > cap  # beyond: SKV_EWORKSPACE
+    assert _plan_bytes(685, 32, 8, 32768) <= cap        # 5,480 KV groups, no ART
+    assert _plan_bytes(345, 64, 8, 32768) <= cap        # 2,760 KV groups at G = 8
+    assert _plan_bytes(48, 32, 8, 131072, **art) > cap  # beyond: SKV_EWORKSPACE
