@@ -90,7 +90,7 @@ def lib():
         L.attn_forecast.restype = _i
         L.skv_host_device_pointer.argtypes = [_p, ctypes.POINTER(_p)]
         L.skv_host_device_pointer.restype = _i
-        L.attn_prefetch_blocks.argtypes = [_p, _p, _p, _p, _p] + [_i] * 8 + [_p, _p, _p, _p, _p, _i, _p]
+        L.attn_prefetch_blocks.argtypes = [_p, _p, _p, _p, _p] + [_i] * 7 + [_p, _p, _p, _p, _p, _i, _p]
         L.attn_prefetch_blocks.restype = _i
         L.skv_status_of_word.argtypes = [ctypes.c_uint32]
         L.skv_status_of_word.restype = _i

@@ -386,3 +386,24 @@ def test_static_workspace_holds_the_stated_shapes():
     assert _plan_bytes(685, 32, 8, 32768) <= cap        # 5,480 KV groups, no ART
     assert _plan_bytes(345, 64, 8, 32768) <= cap        # 2,760 KV groups at G = 8
     assert _plan_bytes(48, 32, 8, 131072, **art) > cap  # beyond: SKV_EWORKSPACE
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every C function the binding declares takes as many arguments in the
+    binding as in include/sparsekv.h (a missing or extra ctypes argument would
+    shift every later one)."""
+    import re
+    src = open(os.path.join(ROOT, "include", "sparsekv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    decls = dict()
+    for m in re.finditer(r"SKV_API\s+[\w\s\*]+?\b(\w+)\s*\(([^)]*)\)\s*;", src):
+        params = m.group(2).strip()
+        decls[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    L = skv.lib()
+    checked = 0
+    for name, n in decls.items():
+        f = getattr(L, name)
+        if f.argtypes is not None:
+            assert len(f.argtypes) == n, (name, len(f.argtypes), n)
+            checked += 1
+    assert checked >= 12
