@@ -361,14 +361,14 @@ def build_select_shared(torch, skv, skvgen, wl, status):
     return step
 
 
-def build_lookahead(torch, skv, skvgen, wl, status, n_ctas=24):
+def build_lookahead(torch, skv, skvgen, wl, status, n_ctas=64):
     """Lookahead prefetch ("SparDA" 2) on a pair of cfg5-shaped layers: layer
     l is a full-attention layer whose cache is on the GPU (ART, as the routed
-    stack runs it); layer l+1 keeps its KV in page-locked host memory.  While
-    layer l attends (main stream), layer l's Forecast picks layer l+1's top-k
-    blocks from their summaries and the gather kernel pulls them into a device
-    cache (side stream, launched first so its CTAs are resident); then layer
-    l+1 attends the cache.  Returns (overlapped step, layer-l-alone step,
+    stack runs it); layer l+1 keeps its KV in page-locked host memory.  Layer
+    l's Forecast picks layer l+1's top-k blocks from their summaries (two small
+    kernels), then the gather kernel pulls them into a device cache on a side
+    stream while layer l attends on the main stream (the gather's small CTAs
+    sit beside the attention kernel's); then layer l+1 attends the cache.  Returns (overlapped step, layer-l-alone step,
     prefetch-alone step, layer-(l+1)-alone step)."""
     layers = [l for l in range(wl.n_layers - 1) if skvgen.route_bit(wl.seed, l) == 1]
     l0 = layers[0]
@@ -406,15 +406,22 @@ def build_lookahead(torch, skv, skvgen, wl, status, n_ctas=24):
     p = lambda t: ctypes.c_void_p(t.data_ptr())
     cur = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
-    def prefetch(stream_ptr):
+    def choose(stream_ptr):
         for st in (L.attn_forecast(p(x), p(w), wl.B, wl.Hkv, wl.d, p(f), stream_ptr),
                    L.attn_select_centroids(p(f), p(summ), p(off), wl.B, wl.Hkv, wl.Hkv, wl.d, mb, k, p(ids),
-                                           p(ss0), p(se0), stream_ptr),
-                   L.attn_prefetch_blocks(kp, vp, p(bt1), p(sl1), p(ids), wl.B, wl.Hkv, wl.d, k, mb,
-                                          k_host.shape[0], wl.Lmax, p(k_cache), p(v_cache), p(ss), p(se),
-                                          p(status), n_ctas, stream_ptr)):
+                                           p(ss0), p(se0), stream_ptr)):
             if st != 0:
-                raise skv.SkvError(st, "lookahead prefetch")
+                raise skv.SkvError(st, "lookahead selection")
+
+    def gather(stream_ptr):
+        st = L.attn_prefetch_blocks(kp, vp, p(bt1), p(sl1), p(ids), wl.B, wl.Hkv, wl.d, k, mb, k_host.shape[0],
+                                    wl.Lmax, p(k_cache), p(v_cache), p(ss), p(se), p(status), n_ctas, stream_ptr)
+        if st != 0:
+            raise skv.SkvError(st, "attn_prefetch_blocks")
+
+    def prefetch(stream_ptr):
+        choose(stream_ptr)
+        gather(stream_ptr)
 
     def attend_next():
         st = L.attn_decode(ctypes.byref(a1), cur())
@@ -423,10 +430,11 @@ def build_lookahead(torch, skv, skvgen, wl, status, n_ctas=24):
 
     def overlapped():
         main = torch.cuda.current_stream()
+        choose(cur())                                    # layer l's Forecast picks l+1's blocks
         side.wait_stream(main)
         with torch.cuda.stream(side):
-            prefetch(ctypes.c_void_p(side.cuda_stream))  # its CTAs take their SM slots first
-        st_fa.run()                                      # layer l on the main stream meanwhile
+            gather(ctypes.c_void_p(side.cuda_stream))    # the copy from host memory ...
+        st_fa.run()                                      # ... while layer l attends
         main.wait_stream(side)
         attend_next()                                    # layer l+1 over the fetched blocks
 

@@ -416,9 +416,10 @@ SKV_API skv_status skv_host_device_pointer(const void* host, void** dev);
  *  seg_start, seg_end int32 [batch][kv_heads][topk] (device, outputs)
  *  status_word     NULL or a device uint32: SKV_DEV_BAD_PAGE and _BAD_SEQLEN
  *                  are OR-ed in and the item copies nothing
- * Launch it on its own stream, before the kernels it should overlap, with a
- * few CTAs (16-32 saturate a PCIe link) so that it stays resident beside
- * them.  Supported: head_dim 128; 16-byte aligned pools and caches. */
+ * Its CTAs are small (64 threads, no shared memory) so that they fit on an
+ * SM beside two CTAs of the decode kernels: launch it on its own stream next
+ * to the attention it should overlap, with a few dozen CTAs (64 keep a PCIe
+ * link busy).  Supported: head_dim 128; 16-byte aligned pools and caches. */
 SKV_API skv_status attn_prefetch_blocks(const void* k_host, const void* v_host,
                                         const int32_t* block_table, const int32_t* seq_lens,
                                         const int32_t* block_ids, int batch, int kv_heads,

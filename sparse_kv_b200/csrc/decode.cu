@@ -191,7 +191,9 @@ struct Cfg {
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;        // float2 [NW][G]
   static constexpr size_t OFF_PRE = OFF_A + (size_t)NW * G * 8;            // int [B+1], int [B]
   static constexpr size_t N_PRE = (2 * (size_t)kMaxPersistentBatch + 1) * 4;
-  static constexpr size_t TOTAL = OFF_PRE + N_PRE;
+  static constexpr int MAX_PEND = 255;                                     // groups queued for the merge
+  static constexpr size_t OFF_PEND = (OFF_PRE + N_PRE + 15) / 16 * 16;     // int [1 + MAX_PEND]
+  static constexpr size_t TOTAL = OFF_PEND + (1 + MAX_PEND) * 4;
   static_assert(TOTAL <= (MINB == 2 ? 113 : 227) * 1024, "shared memory budget");
   // every region read or written with 16-byte vectors starts 16-byte aligned
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_FLAGS % 16 == 0, "alignment");
@@ -200,86 +202,113 @@ struct Cfg {
   static_assert((kRecFloats * 4) % 16 == 0, "record strides");
 };
 
-// Persistent schedule: warp `lane`'s share of the arrival on group g's counter
-// after the warp wrote its record; the warp whose arrival completes every warp
-// of every CTA whose share meets g's tiles merges g's records into the output
-// rows (the "Pulsar Attention" Phase 2 combination, in base 2).  Kept out of
-// line: it runs once per group piece, away from the fold's registers.
-__device__ __noinline__ void merge_group_if_last(const DecodeParams& p, const int* pre, int g, int G,
-                                                 int NW, int lane) {
+// Persistent schedule, group merge.  A group's tiles are shared by the CTAs
+// c0..c1 (those with a non-empty share); each of their NW consumer warps
+// leaves a partial record (O unnormalised, m in base 2, l, tiles).  After its
+// record a warp arrives on the group's counter; the warp whose arrival is the
+// last one queues the group in its CTA, and at the end of the CTA's walk its
+// warps merge the queued groups, one (group, head) pair per warp (the "Pulsar
+// Attention" Phase 2 combination, in base 2), off the walk's critical path.
+struct MergeArgs {
+  int* cnt;
+  const float* rec;
+  float* out;
+  float* lse;
+  int* consumed;
+  int B, Hq, Hkv, n_ctas;
+};
+
+__device__ __forceinline__ bool share_nonempty(long long c, long long T, long long P) {
+  return (c * T) / P != ((c + 1) * T) / P;
+}
+__device__ __forceinline__ void group_ctas(const int* pre, int B, int Hkv, int n_ctas, int g, int& c0,
+                                           int& c1) {
+  const long long T = pre[B], P = n_ctas;
+  const int b = g / Hkv, kvh = g % Hkv;
+  const int nt = (pre[b + 1] - pre[b]) / Hkv;
+  const long long Tg = pre[b] + (long long)kvh * nt;
+  c0 = (int)(((Tg + 1) * P - 1) / T);
+  c1 = (int)(((Tg + nt) * P - 1) / T);
+}
+
+// The calling warp's arrival for group g; true (on every lane) if it was the last.
+__device__ __forceinline__ bool arrive_group(const MergeArgs& p, const int* pre, int g, int NW, int lane) {
   __syncwarp();
-  int last = 0, c0 = 0, c1 = -1;
-  const int b = g / p.Hkv, kvh = g % p.Hkv;
-  const long long T = pre[p.B], P = p.n_ctas;
+  int last = 0;
   if (lane == 0) {
-    const int nt = (pre[b + 1] - pre[b]) / p.Hkv;
-    const long long Tg = pre[b] + (long long)kvh * nt;
-    c0 = (int)(((Tg + 1) * P - 1) / T);
-    c1 = (int)(((Tg + nt) * P - 1) / T);
-    int ncta = 0;  // CTAs in [c0, c1] with a non-empty share
-    for (int c = c0; c <= c1; ++c) ncta += ((long long)c * T) / P != ((long long)(c + 1) * T) / P;
+    int c0, c1;
+    group_ctas(pre, p.B, p.Hkv, p.n_ctas, g, c0, c1);
+    const long long T = pre[p.B], P = p.n_ctas;
+    int ncta = 0;
+    for (int c = c0; c <= c1; ++c) ncta += share_nonempty(c, T, P);
     __threadfence();  // this warp's record, before its arrival
-    const int old = atomicAdd(p.ws_hdr + g, 1);
-    last = old == ncta * NW - 1;
+    last = atomicAdd(p.cnt + g, 1) == ncta * NW - 1;
   }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
-  c0 = __shfl_sync(0xffffffffu, c0, 0);
-  c1 = __shfl_sync(0xffffffffu, c1, 0);
-  __threadfence();  // every arrival came after its record: read them from L2
+  return __shfl_sync(0xffffffffu, last, 0) != 0;
+}
+
+// Merge head h of group g (one warp; lane owns dims 4 lane .. 4 lane + 3).
+__device__ __noinline__ void merge_group_head(const MergeArgs p, const int* pre, int g, int h, int G,
+                                              int NW, int lane) {
+  __threadfence();  // every arrival followed its record: read them from L2
+  int c0, c1;
+  group_ctas(pre, p.B, p.Hkv, p.n_ctas, g, c0, c1);
+  const long long T = pre[p.B], P = p.n_ctas;
   const int nrec = (c1 - c0 + 1) * NW;
-  for (int h = 0; h < G; ++h) {
-    // pass 1: lane r holds record r's (m, l, tiles); max of m over the records
-    float M = -INFINITY;
-    int tiles = 0;
-    for (int r0 = 0; r0 < nrec; r0 += 32) {
-      const int r = r0 + lane;
-      const int c = c0 + r / NW;
-      if (r < nrec && ((long long)c * T) / P != ((long long)(c + 1) * T) / P) {
-        const float4 ml = __ldcg(reinterpret_cast<const float4*>(
-            p.ws_rec + (((size_t)(c + g) * NW + r % NW) * G + h) * kRecFloats + 128));
-        if (ml.y > 0.f) M = fmaxf(M, ml.x);
-        if (r % NW == 0) tiles += (int)ml.z;
-      }
+  auto rec = [&](int r) { return p.rec + (((size_t)(c0 + r / NW + g) * NW + r % NW) * G + h) * kRecFloats; };
+  // pass 1: (m, l, tiles) of 32 records per load round; max of m
+  float M = -INFINITY;
+  int tiles = 0;
+  for (int r0 = 0; r0 < nrec; r0 += 32) {
+    const int r = r0 + lane;
+    if (r < nrec && share_nonempty(c0 + r / NW, T, P)) {
+      const float4 ml = __ldcg(reinterpret_cast<const float4*>(rec(r) + 128));
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
+      if (r % NW == 0) tiles += (int)ml.z;
     }
+  }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
-    }
-    // pass 2: W = sum l 2^(m - M), O = sum O 2^(m - M); the lane owns dims 4 lane .. 4 lane + 3
-    float Wl = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-      for (int r = 0; r < nrec; ++r) {
-        const int c = c0 + r / NW;
-        if (((long long)c * T) / P == ((long long)(c + 1) * T) / P) continue;
-        const float* rec = p.ws_rec + (((size_t)(c + g) * NW + r % NW) * G + h) * kRecFloats;
-        const float4 ml = __ldcg(reinterpret_cast<const float4*>(rec + 128));
-        if (!(ml.y > 0.f)) continue;
-        const float f = exp2f(ml.x - M);
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(rec + lane * 4));
-        Wl += ml.y * f;
-        acc.x += x.x * f;
-        acc.y += x.y * f;
-        acc.z += x.z * f;
-        acc.w += x.w * f;
+  for (int o = 16; o >= 1; o >>= 1) {
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+  }
+  // pass 2: W = sum l 2^(m - M), O = sum O 2^(m - M), 8 records' loads in flight
+  float Wl = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (M != -INFINITY) {
+    for (int r0 = 0; r0 < nrec; r0 += 8) {
+      float4 ml[8], x[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int r = r0 + q;
+        const bool v = r < nrec && share_nonempty(c0 + r / NW, T, P);
+        ml[q] = v ? __ldcg(reinterpret_cast<const float4*>(rec(r) + 128)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[q] = v ? __ldcg(reinterpret_cast<const float4*>(rec(r) + lane * 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float f = (ml[q].y > 0.f) ? exp2f(ml[q].x - M) : 0.f;
+        Wl += ml[q].y * f;
+        acc.x += x[q].x * f;
+        acc.y += x[q].y * f;
+        acc.z += x[q].z * f;
+        acc.w += x[q].w * f;
       }
     }
-    const size_t row = (size_t)b * p.Hq + (size_t)kvh * G + h;
-    const float inv = (Wl > 0.f) ? 1.f / Wl : 0.f;
-    *reinterpret_cast<float4*>(p.out + row * kHeadDim + lane * 4) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    if (lane == 0) {
-      p.lse[row] = (Wl > 0.f) ? (M + log2f(Wl)) * 0.6931471805599453f : -INFINITY;
-      if (p.blocks_consumed) p.blocks_consumed[row] = tiles;
-    }
+  }
+  const int b = g / p.Hkv, kvh = g % p.Hkv;
+  const size_t row = (size_t)b * p.Hq + (size_t)kvh * G + h;
+  const float inv = (Wl > 0.f) ? 1.f / Wl : 0.f;
+  *reinterpret_cast<float4*>(p.out + row * kHeadDim + lane * 4) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (lane == 0) {
+    p.lse[row] = (Wl > 0.f) ? (M + log2f(Wl)) * 0.6931471805599453f : -INFINITY;
+    if (p.consumed) p.consumed[row] = tiles;
   }
 }
 
 template <int G, int NW, int MINB>
-__global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB)
-    decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel(const DecodeParams p) {
   using C = Cfg<G, NW, MINB>;
   constexpr int ST = C::STAGES;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -310,6 +339,7 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB)
     mbar_init(gather_bar, p.sched == SCHED_SPLIT ? p.n_splits : 1);
     mbar_init(release_bar, 1);
     flags[0] = flags[1] = flags[2] = 0;
+    *reinterpret_cast<volatile int*>(smem + C::OFF_PEND) = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -632,9 +662,22 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB)
   };
 
   // Persistent schedule: after its record of group g, a warp arrives on g's
-  // counter; the last arrival merges g (merge_group_if_last).
+  // counter; the last arrival queues g for this CTA's end-of-walk merge (a
+  // full queue merges at once).
   const int* pre = reinterpret_cast<const int*>(smem + C::OFF_PRE);
-  auto arrive_and_merge = [&](int g) { merge_group_if_last(p, pre, g, G, NW, lane); };
+  volatile int* pend = reinterpret_cast<volatile int*>(smem + C::OFF_PEND);  // [0]: count, [1..]: groups
+  auto arrive_and_merge = [&](int g) {
+    const MergeArgs ma{p.ws_hdr, p.ws_rec, p.out, p.lse, p.blocks_consumed, p.B, p.Hq, p.Hkv, p.n_ctas};
+    if (!arrive_group(ma, pre, g, NW, lane)) return;
+    int slot = 0;
+    if (lane == 0) slot = atomicAdd(const_cast<int*>(pend), 1);
+    slot = __shfl_sync(0xffffffffu, slot, 0);
+    if (slot < C::MAX_PEND) {
+      if (lane == 0) pend[1 + slot] = g;
+    } else {
+      for (int h = 0; h < G; ++h) merge_group_head(ma, pre, g, h, G, NW, lane);
+    }
+  };
 
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P) + warp * C::RPW * G;
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
@@ -693,13 +736,19 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB)
       flush(cur_slot, k);
       arrive_and_merge(cur_g);
     }
-    // Every consumer warp ends here: let the producer know once all are done.
+    // Every consumer warp ends here: let the producer know once all are done,
+    // then merge the groups this CTA completed, one (group, head) per warp.
     __syncwarp();
     mbar_arrive_if(fin_bar, lane == 0);
-    if (warp == 0) {
-      if (!mbar_wait_bounded(fin_bar, 0, nullptr) && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
-      if (lane == 0) flags[2] = (flags[1] != 0) ? 1 : e + 1;
+    const bool fin_ok = mbar_wait_bounded(fin_bar, 0, nullptr);
+    if (warp == 0 && lane == 0) {
+      if (!fin_ok) dev_error(p.status, SKV_DEV_TIMEOUT);
+      flags[2] = (flags[1] != 0) ? 1 : e + 1;
     }
+    if (!fin_ok) return;
+    const int npend = min((int)pend[0], (int)C::MAX_PEND);
+    const MergeArgs ma{p.ws_hdr, p.ws_rec, p.out, p.lse, p.blocks_consumed, p.B, p.Hq, p.Hkv, p.n_ctas};
+    for (int i = warp; i < npend * G; i += NW) merge_group_head(ma, pre, pend[1 + i / G], i % G, G, NW, lane);
     return;
   }
   // Split schedule: the CTAs of a cluster are the S pieces of one group, and

@@ -27,10 +27,13 @@
 namespace skv {
 namespace {
 
-constexpr int kGatherThreads = 256;
-constexpr int kBlockVecs = kTileBytes / 16;                   // 16-byte vectors per 16 KiB tile
-constexpr int kVecsPerThread = kBlockVecs / kGatherThreads;   // 4
-static_assert(kBlockVecs % kGatherThreads == 0, "tile split");
+// Small CTAs (two warps, few registers, no shared memory) fit beside two
+// resident CTAs of the decode kernels on the same SM, so the copy overlaps a
+// persistent attention kernel whichever starts first.
+constexpr int kGatherThreads = 64;
+constexpr int kBlockVecs = kTileBytes / 16;  // 16-byte vectors per 16 KiB tile
+constexpr int kGatherBatch = 8;              // vectors of K and of V in flight per thread
+static_assert(kBlockVecs % (kGatherThreads * kGatherBatch) == 0, "tile split");
 
 __global__ void __launch_bounds__(kHeadDim) forecast_kernel(const uint16_t* __restrict__ x,
                                                             const uint16_t* __restrict__ w, int Hkv,
@@ -71,7 +74,7 @@ __device__ __forceinline__ uint4 ld_sys_v4(const void* p) {
   return v;
 }
 
-__global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherParams p) {
+__global__ void __launch_bounds__(kGatherThreads, 1) gather_kernel(const GatherParams p) {
   const long long items = (long long)p.B * p.Hkv * p.k;
   const int tid = threadIdx.x;
   for (long long it = blockIdx.x; it < items; it += gridDim.x) {
@@ -107,21 +110,23 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
     uint4* kd = reinterpret_cast<uint4*>(p.k_cache + dst);
     uint4* vd = reinterpret_cast<uint4*>(p.v_cache + dst);
     const int nvec = n * (kRowBytes / 16);  // rows of the block that hold tokens
-    uint4 kr[kVecsPerThread], vr[kVecsPerThread];
+    for (int base = 0; base < nvec; base += kGatherThreads * kGatherBatch) {
+      uint4 kr[kGatherBatch], vr[kGatherBatch];
 #pragma unroll
-    for (int u = 0; u < kVecsPerThread; ++u) {  // every load of the block in flight at once
-      const int i = tid + u * kGatherThreads;
-      if (i < nvec) {
-        kr[u] = ld_sys_v4(ks + i);
-        vr[u] = ld_sys_v4(vs + i);
+      for (int u = 0; u < kGatherBatch; ++u) {  // all of a batch's loads in flight at once
+        const int i = base + tid + u * kGatherThreads;
+        if (i < nvec) {
+          kr[u] = ld_sys_v4(ks + i);
+          vr[u] = ld_sys_v4(vs + i);
+        }
       }
-    }
 #pragma unroll
-    for (int u = 0; u < kVecsPerThread; ++u) {
-      const int i = tid + u * kGatherThreads;
-      if (i < nvec) {
-        kd[i] = kr[u];
-        vd[i] = vr[u];
+      for (int u = 0; u < kGatherBatch; ++u) {
+        const int i = base + tid + u * kGatherThreads;
+        if (i < nvec) {
+          kd[i] = kr[u];
+          vd[i] = vr[u];
+        }
       }
     }
   }
