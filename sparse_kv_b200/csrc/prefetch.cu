@@ -32,7 +32,7 @@ namespace {
 // persistent attention kernel whichever starts first.
 constexpr int kGatherThreads = 64;
 constexpr int kBlockVecs = kTileBytes / 16;  // 16-byte vectors per 16 KiB tile
-constexpr int kGatherBatch = 8;              // vectors of K and of V in flight per thread
+constexpr int kGatherBatch = 8;              // 16-byte vectors in flight per thread
 static_assert(kBlockVecs % (kGatherThreads * kGatherBatch) == 0, "tile split");
 
 __global__ void __launch_bounds__(kHeadDim) forecast_kernel(const uint16_t* __restrict__ x,
@@ -74,7 +74,9 @@ __device__ __forceinline__ uint4 ld_sys_v4(const void* p) {
   return v;
 }
 
-__global__ void __launch_bounds__(kGatherThreads, 1) gather_kernel(const GatherParams p) {
+// at most 64 registers: 2 warps x 32 x 64 = 4096 registers, which two CTAs of
+// the decode kernels (at most 2 x 30720) leave free on an SM
+__global__ void __launch_bounds__(kGatherThreads, 16) gather_kernel(const GatherParams p) {
   const long long items = (long long)p.B * p.Hkv * p.k;
   const int tid = threadIdx.x;
   for (long long it = blockIdx.x; it < items; it += gridDim.x) {
@@ -110,23 +112,17 @@ __global__ void __launch_bounds__(kGatherThreads, 1) gather_kernel(const GatherP
     uint4* kd = reinterpret_cast<uint4*>(p.k_cache + dst);
     uint4* vd = reinterpret_cast<uint4*>(p.v_cache + dst);
     const int nvec = n * (kRowBytes / 16);  // rows of the block that hold tokens
-    for (int base = 0; base < nvec; base += kGatherThreads * kGatherBatch) {
-      uint4 kr[kGatherBatch], vr[kGatherBatch];
+    for (int t = 0; t < 2; ++t) {             // K rows, then V rows
+      const uint4* src4 = (t == 0 ? ks : vs) + tid;
+      uint4* dst4 = (t == 0 ? kd : vd) + tid;
+      for (int base = 0; base < nvec; base += kGatherThreads * kGatherBatch) {
+        uint4 r[kGatherBatch];
 #pragma unroll
-      for (int u = 0; u < kGatherBatch; ++u) {  // all of a batch's loads in flight at once
-        const int i = base + tid + u * kGatherThreads;
-        if (i < nvec) {
-          kr[u] = ld_sys_v4(ks + i);
-          vr[u] = ld_sys_v4(vs + i);
-        }
-      }
+        for (int u = 0; u < kGatherBatch; ++u)  // all of a batch's loads in flight at once
+          if (base + tid + u * kGatherThreads < nvec) r[u] = ld_sys_v4(src4 + base + u * kGatherThreads);
 #pragma unroll
-      for (int u = 0; u < kGatherBatch; ++u) {
-        const int i = base + tid + u * kGatherThreads;
-        if (i < nvec) {
-          kd[i] = kr[u];
-          vd[i] = vr[u];
-        }
+        for (int u = 0; u < kGatherBatch; ++u)
+          if (base + tid + u * kGatherThreads < nvec) dst4[base + u * kGatherThreads] = r[u];
       }
     }
   }
