@@ -181,7 +181,7 @@ size_t skv_decode_workspace_size(const skv_decode_args* args) {
 int skv_decode_launches(const skv_decode_args* args) {
   Plan pl;
   if (make_plan(args, &pl) != SKV_OK) return 0;
-  return pl.art ? 2 : 1;
+  return 1;
 }
 
 skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* plan) {
@@ -190,7 +190,7 @@ skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* pl
   Plan pl;
   const skv_status st = make_plan(args, &pl);
   if (st != SKV_OK) return st;
-  plan->launches = pl.art ? 2 : 1;
+  plan->launches = 1;
   plan->workspace_bytes = pl.ws_bytes;
   if (pl.chunk) {
     plan->schedule = SKV_SCHED_CHUNK;
@@ -268,6 +268,7 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
     p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes + pl.lb_bytes + pl.scratch_bytes);
     if (cudaMemsetAsync(ws, 0, pl.hdr_bytes, s) != cudaSuccess) return SKV_ECUDA;
     if (launch_art(p, pl.G, s) != 0) return SKV_ECUDA;
+    return SKV_OK;  // merged inside the kernel
   } else {
     p.ws_hdr = reinterpret_cast<int*>(ws);
     p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes);
@@ -282,8 +283,6 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
     if (launch_decode(p, pl.G, s) != 0) return SKV_ECUDA;
     return SKV_OK;  // merged inside the kernel
   }
-  if (launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
-  return SKV_OK;
 }
 
 skv_status attn_select_centroids(const void* q, const void* centroids, const int32_t* cluster_off,

@@ -192,8 +192,8 @@ struct Cfg {
   static constexpr size_t OFF_PRE = OFF_A + (size_t)NW * G * 8;            // int [B+1], int [B]
   static constexpr size_t N_PRE = (2 * (size_t)kMaxPersistentBatch + 1) * 4;
   static constexpr int MAX_PEND = 255;                                     // groups queued for the merge
-  static constexpr size_t OFF_PEND = (OFF_PRE + N_PRE + 15) / 16 * 16;     // int [1 + MAX_PEND]
-  static constexpr size_t TOTAL = OFF_PEND + (1 + MAX_PEND) * 4;
+  static constexpr size_t OFF_PEND = (OFF_PRE + N_PRE + 15) / 16 * 16;     // int [2 + MAX_PEND]
+  static constexpr size_t TOTAL = OFF_PEND + (2 + MAX_PEND) * 4;
   static_assert(TOTAL <= (MINB == 2 ? 113 : 227) * 1024, "shared memory budget");
   // every region read or written with 16-byte vectors starts 16-byte aligned
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_FLAGS % 16 == 0, "alignment");
@@ -204,11 +204,10 @@ struct Cfg {
 
 // Persistent schedule, group merge.  A group's tiles are shared by the CTAs
 // c0..c1 (those with a non-empty share); each of their NW consumer warps
-// leaves a partial record (O unnormalised, m in base 2, l, tiles).  After its
-// record a warp arrives on the group's counter; the warp whose arrival is the
-// last one queues the group in its CTA, and at the end of the CTA's walk its
-// warps merge the queued groups, one (group, head) pair per warp (the "Pulsar
-// Attention" Phase 2 combination, in base 2), off the walk's critical path.
+// leaves a partial record (O unnormalised, m in base 2, l, tiles).  At the end
+// of its walk a CTA arrives once on the counter of every group it touched; the
+// CTA whose arrival is the group's last merges it, one (group, head) pair per
+// warp (the "Pulsar Attention" Phase 2 combination, in base 2).
 struct MergeArgs {
   int* cnt;
   const float* rec;
@@ -229,22 +228,6 @@ __device__ __forceinline__ void group_ctas(const int* pre, int B, int Hkv, int n
   const long long Tg = pre[b] + (long long)kvh * nt;
   c0 = (int)(((Tg + 1) * P - 1) / T);
   c1 = (int)(((Tg + nt) * P - 1) / T);
-}
-
-// The calling warp's arrival for group g; true (on every lane) if it was the last.
-__device__ __forceinline__ bool arrive_group(const MergeArgs& p, const int* pre, int g, int NW, int lane) {
-  __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    int c0, c1;
-    group_ctas(pre, p.B, p.Hkv, p.n_ctas, g, c0, c1);
-    const long long T = pre[p.B], P = p.n_ctas;
-    int ncta = 0;
-    for (int c = c0; c <= c1; ++c) ncta += share_nonempty(c, T, P);
-    __threadfence();  // this warp's record, before its arrival
-    last = atomicAdd(p.cnt + g, 1) == ncta * NW - 1;
-  }
-  return __shfl_sync(0xffffffffu, last, 0) != 0;
 }
 
 // Merge head h of group g (one warp; lane owns dims 4 lane .. 4 lane + 3).
@@ -316,7 +299,8 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
   uint64_t* empty = full + ST;
   uint64_t* fin_bar = empty + ST;  // NW arrivals: the consumers are done with the ring
   // split schedule only:
-  uint64_t* fin2_bar = fin_bar + 1;     // NW arrivals: the warps' states are in the ring
+  uint64_t* fin2_bar = fin_bar + 1;     // NW arrivals: split: the warps' states are in the ring;
+                                        // persistent: the merge queue is complete
   uint64_t* fin3_bar = fin2_bar + 1;    // NW arrivals: the piece's records are written
   uint64_t* fin4_bar = fin3_bar + 1;    // G arrivals: (rank 0) the merge is done
   uint64_t* gather_bar = fin4_bar + 1;  // (rank 0) S arrivals, one per piece of the cluster
@@ -661,23 +645,11 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     }
   };
 
-  // Persistent schedule: after its record of group g, a warp arrives on g's
-  // counter; the last arrival queues g for this CTA's end-of-walk merge (a
-  // full queue merges at once).
+  // Persistent schedule: the groups this CTA touched form a contiguous range
+  // (its share of the concatenated tile lists); warp 0 notes the first.
   const int* pre = reinterpret_cast<const int*>(smem + C::OFF_PRE);
-  volatile int* pend = reinterpret_cast<volatile int*>(smem + C::OFF_PEND);  // [0]: count, [1..]: groups
-  auto arrive_and_merge = [&](int g) {
-    const MergeArgs ma{p.ws_hdr, p.ws_rec, p.out, p.lse, p.blocks_consumed, p.B, p.Hq, p.Hkv, p.n_ctas};
-    if (!arrive_group(ma, pre, g, NW, lane)) return;
-    int slot = 0;
-    if (lane == 0) slot = atomicAdd(const_cast<int*>(pend), 1);
-    slot = __shfl_sync(0xffffffffu, slot, 0);
-    if (slot < C::MAX_PEND) {
-      if (lane == 0) pend[1 + slot] = g;
-    } else {
-      for (int h = 0; h < G; ++h) merge_group_head(ma, pre, g, h, G, NW, lane);
-    }
-  };
+  // [0]: queued groups, [1]: the first group of this CTA's share, [2..]: the queue
+  volatile int* pend = reinterpret_cast<volatile int*>(smem + C::OFF_PEND);
 
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P) + warp * C::RPW * G;
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
@@ -703,10 +675,8 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       break;
     }
     if (mt.y != cur_g) {
-      if (cur_g >= 0) {
-        flush(cur_slot, k);
-        if (p.sched == SCHED_PERSISTENT) arrive_and_merge(cur_g);
-      }
+      if (cur_g >= 0) flush(cur_slot, k);
+      else if (warp == 0 && lane == 0) pend[1] = mt.y;
       W.reset();
       const int b = mt.y / p.Hkv, kvh = mt.y % p.Hkv;
       W.load_q(p.q, (size_t)b * p.Hq + (size_t)kvh * G, p.qscale, lane);
@@ -732,12 +702,13 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
 
   // ------------------------------------------------------------------ epilogue
   if (p.sched == SCHED_PERSISTENT) {
-    if (cur_g >= 0) {
-      flush(cur_slot, k);
-      arrive_and_merge(cur_g);
-    }
-    // Every consumer warp ends here: let the producer know once all are done,
-    // then merge the groups this CTA completed, one (group, head) per warp.
+    if (cur_g >= 0) flush(cur_slot, k);
+    // Every consumer warp ends here, its records written (and fenced): let the
+    // producer know once all are done.  Then the CTA arrives once on the
+    // counter of every group it touched; the arrival that completes a group
+    // (all CTAs whose share meets its tiles) queues it, and the warps merge
+    // the queued groups, one (group, head) per warp.
+    __threadfence();
     __syncwarp();
     mbar_arrive_if(fin_bar, lane == 0);
     const bool fin_ok = mbar_wait_bounded(fin_bar, 0, nullptr);
@@ -745,10 +716,37 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       if (!fin_ok) dev_error(p.status, SKV_DEV_TIMEOUT);
       flags[2] = (flags[1] != 0) ? 1 : e + 1;
     }
-    if (!fin_ok) return;
-    const int npend = min((int)pend[0], (int)C::MAX_PEND);
+    if (!fin_ok || cur_g < 0) return;
     const MergeArgs ma{p.ws_hdr, p.ws_rec, p.out, p.lse, p.blocks_consumed, p.B, p.Hq, p.Hkv, p.n_ctas};
-    for (int i = warp; i < npend * G; i += NW) merge_group_head(ma, pre, pend[1 + i / G], i % G, G, NW, lane);
+    const long long T = pre[p.B], P = p.n_ctas;
+    for (int g = pend[1] + warp; g <= cur_g; g += NW) {
+      int last = 0;
+      if (lane == 0) {
+        int c0, c1;
+        group_ctas(pre, p.B, p.Hkv, p.n_ctas, g, c0, c1);
+        int ncta = 0;
+        for (int c = c0; c <= c1; ++c) ncta += share_nonempty(c, T, P);
+        __threadfence();
+        last = atomicAdd(p.ws_hdr + g, 1) == ncta - 1;
+      }
+      if (!__shfl_sync(0xffffffffu, last, 0)) continue;
+      int slot = 0;
+      if (lane == 0) slot = atomicAdd(const_cast<int*>(pend), 1);
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      if (slot < C::MAX_PEND) {
+        if (lane == 0) pend[2 + slot] = g;
+      } else {  // a full queue: this warp merges the group now
+        for (int h = 0; h < G; ++h) merge_group_head(ma, pre, g, h, G, NW, lane);
+      }
+    }
+    __syncwarp();
+    mbar_arrive_if(fin2_bar, lane == 0);
+    if (!mbar_wait_bounded(fin2_bar, 0, nullptr)) {
+      if (lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+      return;
+    }
+    const int npend = min((int)pend[0], (int)C::MAX_PEND);
+    for (int i = warp; i < npend * G; i += NW) merge_group_head(ma, pre, pend[2 + i / G], i % G, G, NW, lane);
     return;
   }
   // Split schedule: the CTAs of a cluster are the S pieces of one group, and

@@ -82,9 +82,10 @@ __host__ __device__ inline int art_positions(const DecodeParams& p, int L) {
 }
 
 // Control words of the ART schedule: counter (4), stop chunk per group, ready
-// flag per chunk, blocks consumed and stop chunk per head.
+// flag per chunk, blocks consumed and stop chunk per head, and per group the
+// re-fold count, the arrivals expected and the arrivals so far (the merge).
 inline long long art_ctl_words(long long groups, long long maxc, int G) {
-  return 4 + groups + groups * maxc + 2 * groups * G;
+  return 4 + groups + groups * maxc + 2 * groups * G + 3 * groups;
 }
 
 // Tiles of one KV group for the index-based traversals (natural / range /
@@ -120,7 +121,6 @@ int art_ctas_per_sm(int G);
 size_t art_scratch_bytes_per_cta(int G, int CB);
 int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int d, float* out,
                  float* lse, void* stream);
-int launch_merge_records(const DecodeParams& p, int G, void* stream);
 int launch_chunk(const DecodeParams& p, int Tq, int causal, int n_shards, void* stream);
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int shared, int* ids, int* ss, int* se, void* stream);

@@ -169,14 +169,14 @@ def test_workspace_size_query():
 
 
 def test_decode_launch_count():
-    # one kernel where the walk merges its own partials (large walks: the last
-    # arrival per group merges; small walks and segment lists: the cluster's
-    # shared memory; a query chunk writes its results directly), two where a
-    # record merge follows (ART)
+    # one kernel in every schedule: the walk merges its own partials (large
+    # walks and ART: each group's last arrival queues it for a merge at the end
+    # of its CTA's walk; small walks and segment lists: the cluster's shared
+    # memory; a query chunk writes its results directly)
     L = skv.lib()
     n = lambda a: L.skv_decode_launches(ctypes.byref(a))
     assert n(good_args()) == 1                                    # 128 groups x 512 tiles
-    assert n(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == 2
+    assert n(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == 1
     small = good_args(batch=1, q_heads=8, kv_heads=2, max_seq_len=4096, max_blocks=64)
     assert n(small) == 1                                          # 2 groups x 64 tiles
     # the split schedule merges its pieces in the cluster's shared memory: no workspace
@@ -269,7 +269,8 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
     # The ART chunk is 32 blocks when the chunks in flight per group (CTAs /
     # groups) span at most 1/12 of the walk, else 16.  The workspace of a
     # chunk length CB: zeroed control words (item counter, stop chunk per
-    # group, ready flag per (group, chunk), consumed and stop per head), per
+    # group, ready flag per (group, chunk), consumed and stop per head, and the
+    # merge's re-fold count, expected and received arrivals per group), per
     # (group, chunk) a look-back record (12 floats) and a partial record (132
     # floats) per head, and per resident CTA (148 SMs x 2) probes of CB blocks
     # x 8 warps x G heads x 12 floats and 8 warps' states of G x 132 floats,
@@ -287,7 +288,7 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
     for cb in (16, 32):
         maxc = -(-blocks // cb)
         items = groups * maxc
-        ctl = up((4 + groups + groups * maxc + 2 * groups * G) * 4)
+        ctl = up((4 + groups + groups * maxc + 2 * groups * G + 3 * groups) * 4)
         lb = up(items * G * 12 * 4)
         scratch = ctas * (posts * cb * NW * G * 12 + posts * NW * G * 132) * 4
         sizes[cb] = ctl + lb + scratch + items * G * 132 * 4
@@ -306,7 +307,7 @@ def test_decode_plan_info():
     assert (full.schedule, full.ctas, full.splits, full.launches) == (0, 296, 0, 1)
     assert full.workspace_bytes == L.skv_decode_workspace_size(ctypes.byref(good_args()))
     art = plan(good_args(art=_Art(1, 1e-3, 1e-4, 4)))
-    assert (art.schedule, art.ctas, art.art_chunk_blocks, art.art_chunks, art.launches) == (2, 296, 16, 32, 2)
+    assert (art.schedule, art.ctas, art.art_chunk_blocks, art.art_chunks, art.launches) == (2, 296, 16, 32, 1)
     art5 = plan(good_args(batch=8, max_seq_len=131072, max_blocks=2048, art=_Art(1, 1e-3, 1e-4, 4)))
     assert (art5.art_chunk_blocks, art5.art_chunks) == (32, 64)
     small = plan(good_args(batch=1, q_heads=8, kv_heads=2, max_seq_len=4096, max_blocks=64))
