@@ -101,7 +101,7 @@ struct ArtCfg {  // shared-memory layout
   static constexpr int THREADS = (NW + 2) * 32;  // consumers, producer, arbiter
   // a stage: K rows, V rows, and the group's q rows (loaded with a chunk's first block)
   static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes + (size_t)G * kRowBytes;
-  static constexpr int NBAR = 2 * ST + 2 + 2 * kPosts;  // full, empty, fin, posted[], freed[], arb_done
+  static constexpr int NBAR = 2 * ST + 3 + 2 * kPosts;  // full, empty, fin, posted[], freed[], arb_done, fin2
   static constexpr size_t OFF_BAR = ST * STAGE_BYTES;
   static constexpr size_t OFF_META = up16(OFF_BAR + NBAR * 8);        // int4 [ST]
   static constexpr size_t OFF_FLAGS = up16(OFF_META + ST * 16);       // int [4]
@@ -111,8 +111,10 @@ struct ArtCfg {  // shared-memory layout
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;   // float2 [NW][G]
   static constexpr size_t OFF_WCTL = up16(OFF_A + (size_t)NW * G * 8);  // int [NW][8]
   static constexpr size_t OFF_LOCAL = OFF_WCTL + (size_t)NW * 8 * 4;    // float [CB][G][12] (arbiter)
-  static constexpr int MAX_PEND = 63;  // groups this CTA completes, merged at its end
-  static constexpr size_t OFF_PEND = OFF_LOCAL + (size_t)CB * G * kProbeFloats * 4;  // int [1 + MAX_PEND]
+  static constexpr int MAX_EV = 63;    // counted records this CTA wrote (its arrivals)
+  static constexpr int MAX_PEND = 63;   // groups this CTA completes, merged at its end
+  static constexpr size_t OFF_EV = OFF_LOCAL + (size_t)CB * G * kProbeFloats * 4;  // int [1 + MAX_EV]
+  static constexpr size_t OFF_PEND = OFF_EV + (1 + MAX_EV) * 4;                      // int [1 + MAX_PEND]
   static constexpr size_t TOTAL = OFF_PEND + (1 + MAX_PEND) * 4;
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_P % 16 == 0, "alignment");
   static_assert(OFF_A % 16 == 0 && OFF_WCTL % 16 == 0 && OFF_LOCAL % 16 == 0, "alignment");
@@ -155,7 +157,6 @@ struct Ctl {
   int* ready;
   int* consumed;
   int* head_stop;
-  int* fixes;  // re-fold requests queued for the group
   int* need;   // arrivals that complete the group's records (0: not known yet)
   int* done;   // arrivals so far
   __device__ Ctl(const DecodeParams& p, int G) {
@@ -165,8 +166,7 @@ struct Ctl {
     ready = stop_chunk + groups;
     consumed = ready + (size_t)groups * p.art_maxc;
     head_stop = consumed + (size_t)groups * G;
-    fixes = head_stop + (size_t)groups * G;
-    need = fixes + groups;
+    need = head_stop + (size_t)groups * G;
     done = need + groups;
   }
 };
@@ -247,7 +247,9 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   uint64_t* fin_bar = empty + ST;
   uint64_t* posted = fin_bar + 1;   // [kPosts] a post is ready (one arrival per consumer warp)
   uint64_t* freed = posted + kPosts;  // [kPosts] the arbiter is done with a post
-  uint64_t* arb_done = freed + kPosts;  // the arbiter has left its loop (the merge queue is final)
+  uint64_t* arb_done = freed + kPosts;  // the arbiter has left its loop (its arrivals are listed)
+  uint64_t* fin2_bar = arb_done + 1;    // NW arrivals: the merge queue is complete
+  volatile int* ev = reinterpret_cast<volatile int*>(smem + C::OFF_EV);      // [0]: count, then groups
   volatile int* pend = reinterpret_cast<volatile int*>(smem + C::OFF_PEND);  // [0]: count, then groups
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows | 0 = end of chunk, group, chunk, block in chunk | blocks}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
@@ -279,6 +281,8 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       mbar_init(&freed[i], 1);
     }
     mbar_init(arb_done, 1);
+    mbar_init(fin2_bar, NW);
+    ev[0] = 0;
     pend[0] = 0;
     flags[0] = flags[1] = flags[2] = flags[3] = 0;
     fence_barrier_init();
@@ -815,42 +819,49 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
           *reinterpret_cast<volatile int*>(ctl.stop_chunk + g) = c + 1;
           __threadfence();
         }
-        // Merge bookkeeping: this chunk's stops queue one re-fold.  If the group
-        // ends here (every head has stopped, or the walk's last chunk), the
-        // arrivals that complete its records are known: one per chunk up to
-        // this one and one per re-fold (all queued by now: earlier chunks
-        // counted theirs before releasing their ready flags).
-        if (any_live) {
-          const int nf = stopmask ? atomicAdd(ctl.fixes + g, 1) + 1 : ld_acquire(ctl.fixes + g);
-          if ((all && stopmask) || last_chunk) st_release(ctl.need + g, c + 1 + nf);
-        }
         st_release(ctl.ready + item, 1);
+      }
+      // Merge bookkeeping.  If the group ends here (every head has stopped, or
+      // this is the walk's last chunk), the arrivals that complete its records
+      // are known: one per chunk up to this one, and one per re-fold, i.e. per
+      // distinct stop chunk among the heads (earlier chunks' stops are visible:
+      // their deciders wrote them before releasing the ready flags acquired
+      // above; this chunk's were written by this warp).
+      if (any_live && ((all && stopmask) || last_chunk)) {
+        __syncwarp();
+        const int hs = lane < G ? *reinterpret_cast<volatile int*>(ctl.head_stop + (size_t)g * G + lane) : 0;
+        bool first = hs != 0;
+#pragma unroll
+        for (int j = 0; j < G - 1; ++j) {
+          const int o = __shfl_sync(0xffffffffu, hs, j);
+          if (j < lane && o == hs) first = false;
+        }
+        const int nf = __popc(__ballot_sync(0xffffffffu, first && lane < G));
+        if (lane == 0) st_release(ctl.need + g, c + 1 + nf);
       }
       *counted = any_live;
       return stopmask;
     };
 
-    // An arrival for group g once one of its counted records (a chunk's, or a
-    // re-fold's) is written; the last one queues g for this CTA's end merge.
+    // One counted record of group g (a chunk's, or a re-fold's) is written: note
+    // it; the CTA's arrivals are made at the end of its walk, in one batch.
+    // A full list arrives at once (and merges here if that completes g).
     auto arrive = [&](int g) {
       __syncwarp();
-      int now = 0;  // 1: the queue is full, merge here
+      int full_now = 0;
       if (lane == 0) {
-        __threadfence();
-        const int v = atomicAdd(ctl.done + g, 1) + 1;
-        __threadfence();
-        const int n = *reinterpret_cast<volatile int*>(ctl.need + g);
-        if (n != 0 && v == n) {
-          const int slot = pend[0];
-          if (slot < C::MAX_PEND) {
-            pend[1 + slot] = g;
-            pend[0] = slot + 1;
-          } else {
-            now = 1;
-          }
+        const int n = ev[0];
+        if (n < C::MAX_EV) {
+          ev[1 + n] = g;
+          ev[0] = n + 1;
+        } else {
+          __threadfence();
+          const int v = atomicAdd(ctl.done + g, 1) + 1;
+          __threadfence();
+          full_now = v == *reinterpret_cast<volatile int*>(ctl.need + g);
         }
       }
-      if (__shfl_sync(0xffffffffu, now, 0))
+      if (__shfl_sync(0xffffffffu, full_now, 0))
         for (int h = 0; h < G; ++h) art_merge_head(merge_args(), g, h, G, CB, lane);
     };
 
@@ -904,6 +915,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       ++kj;
       if (kind == POST_DONE) break;
     }
+    __threadfence();  // the records written above, before the CTA's arrivals
     __syncwarp();
     mbar_arrive_if(arb_done, lane == 0);
     return;
@@ -1079,9 +1091,29 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     if (!fin_ok) dev_error(p.status, SKV_DEV_TIMEOUT);
     flags[2] = (flags[1] != 0) ? 1 : e + 1;
   }
-  // Once the arbiter has left its loop, merge the groups whose last arrival
-  // happened in this CTA, one (group, head) per warp.
+  // Once the arbiter has left its loop: the CTA's arrivals (one per counted
+  // record it wrote); an arrival that completes a group queues it, and the
+  // warps merge the queued groups, one (group, head) per warp.
   if (!mbar_wait_bounded(arb_done, 0, nullptr)) {
+    if (lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+    return;
+  }
+  const int nev = min((int)ev[0], (int)C::MAX_EV);
+  for (int i = warp; i < nev; i += NW) {
+    if (lane != 0) continue;
+    const int g = ev[1 + i];
+    __threadfence();
+    const int v = atomicAdd(ctl.done + g, 1) + 1;
+    __threadfence();
+    if (v == *reinterpret_cast<volatile int*>(ctl.need + g)) {
+      const int slot = atomicAdd(const_cast<int*>(pend), 1);
+      if (slot < C::MAX_PEND) pend[1 + slot] = g;
+      else dev_error(p.status, SKV_DEV_TIMEOUT);  // MAX_PEND >= MAX_EV: cannot happen
+    }
+  }
+  __syncwarp();
+  mbar_arrive_if(fin2_bar, lane == 0);
+  if (!mbar_wait_bounded(fin2_bar, 0, nullptr)) {
     if (lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
     return;
   }

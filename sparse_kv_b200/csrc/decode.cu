@@ -233,10 +233,14 @@ __device__ __forceinline__ void group_ctas(const int* pre, int B, int Hkv, int n
 // Merge head h of group g (one warp; lane owns dims 4 lane .. 4 lane + 3).
 __device__ __noinline__ void merge_group_head(const MergeArgs p, const int* pre, int g, int h, int G,
                                               int NW, int lane) {
-  __threadfence();  // every arrival followed its record: read them from L2
+  __threadfence();  // every arrival followed its records: read them from L2
   int c0, c1;
   group_ctas(pre, p.B, p.Hkv, p.n_ctas, g, c0, c1);
   const long long T = pre[p.B], P = p.n_ctas;
+  // CTAs c0 + i with a non-empty share, as a bit mask (spans of up to 32 CTAs;
+  // a longer span, from very short shares, asks for the rest one by one)
+  const uint32_t span = __ballot_sync(0xffffffffu, c0 + lane <= c1 && share_nonempty(c0 + lane, T, P));
+  auto live = [&](int i) { return i < 32 ? ((span >> i) & 1u) != 0 : share_nonempty(c0 + i, T, P); };
   const int nrec = (c1 - c0 + 1) * NW;
   auto rec = [&](int r) { return p.rec + (((size_t)(c0 + r / NW + g) * NW + r % NW) * G + h) * kRecFloats; };
   // pass 1: (m, l, tiles) of 32 records per load round; max of m
@@ -244,7 +248,7 @@ __device__ __noinline__ void merge_group_head(const MergeArgs p, const int* pre,
   int tiles = 0;
   for (int r0 = 0; r0 < nrec; r0 += 32) {
     const int r = r0 + lane;
-    if (r < nrec && share_nonempty(c0 + r / NW, T, P)) {
+    if (r < nrec && live(r / NW)) {
       const float4 ml = __ldcg(reinterpret_cast<const float4*>(rec(r) + 128));
       if (ml.y > 0.f) M = fmaxf(M, ml.x);
       if (r % NW == 0) tiles += (int)ml.z;
@@ -264,7 +268,7 @@ __device__ __noinline__ void merge_group_head(const MergeArgs p, const int* pre,
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int r = r0 + q;
-        const bool v = r < nrec && share_nonempty(c0 + r / NW, T, P);
+        const bool v = r < nrec && live(r / NW);
         ml[q] = v ? __ldcg(reinterpret_cast<const float4*>(rec(r) + 128)) : make_float4(0.f, 0.f, 0.f, 0.f);
         x[q] = v ? __ldcg(reinterpret_cast<const float4*>(rec(r) + lane * 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -288,6 +292,45 @@ __device__ __noinline__ void merge_group_head(const MergeArgs p, const int* pre,
     p.lse[row] = (Wl > 0.f) ? (M + log2f(Wl)) * 0.6931471805599453f : -INFINITY;
     if (p.consumed) p.consumed[row] = tiles;
   }
+}
+
+// End of a CTA's persistent walk (every consumer warp): one arrival per group
+// the CTA touched (groups pend[1] .. last_g); an arrival that completes a group
+// queues it (pend[0] entries from pend[2]); then the warps merge the queued
+// groups, one (group, head) per warp.  Out of line: it runs once per CTA.
+__device__ __noinline__ void persistent_arrivals_and_merges(const MergeArgs ma, const int* pre,
+                                                            volatile int* pend, int max_pend, int last_g,
+                                                            uint64_t* fin2_bar, uint32_t* status, int G,
+                                                            int NW, int warp, int lane) {
+  const long long T = pre[ma.B], P = ma.n_ctas;
+  for (int g = pend[1] + warp; g <= last_g; g += NW) {
+    int last = 0;
+    if (lane == 0) {
+      int c0, c1;
+      group_ctas(pre, ma.B, ma.Hkv, ma.n_ctas, g, c0, c1);
+      int ncta = 0;
+      for (int c = c0; c <= c1; ++c) ncta += share_nonempty(c, T, P);
+      __threadfence();
+      last = atomicAdd(ma.cnt + g, 1) == ncta - 1;
+    }
+    if (!__shfl_sync(0xffffffffu, last, 0)) continue;
+    int slot = 0;
+    if (lane == 0) slot = atomicAdd(const_cast<int*>(pend), 1);
+    slot = __shfl_sync(0xffffffffu, slot, 0);
+    if (slot < max_pend) {
+      if (lane == 0) pend[2 + slot] = g;
+    } else {  // a full queue: this warp merges the group now
+      for (int h = 0; h < G; ++h) merge_group_head(ma, pre, g, h, G, NW, lane);
+    }
+  }
+  __syncwarp();
+  mbar_arrive_if(fin2_bar, lane == 0);
+  if (!mbar_wait_bounded(fin2_bar, 0, nullptr)) {
+    if (lane == 0) dev_error(status, SKV_DEV_TIMEOUT);
+    return;
+  }
+  const int npend = min((int)pend[0], max_pend);
+  for (int i = warp; i < npend * G; i += NW) merge_group_head(ma, pre, pend[2 + i / G], i % G, G, NW, lane);
 }
 
 template <int G, int NW, int MINB>
@@ -718,35 +761,7 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     }
     if (!fin_ok || cur_g < 0) return;
     const MergeArgs ma{p.ws_hdr, p.ws_rec, p.out, p.lse, p.blocks_consumed, p.B, p.Hq, p.Hkv, p.n_ctas};
-    const long long T = pre[p.B], P = p.n_ctas;
-    for (int g = pend[1] + warp; g <= cur_g; g += NW) {
-      int last = 0;
-      if (lane == 0) {
-        int c0, c1;
-        group_ctas(pre, p.B, p.Hkv, p.n_ctas, g, c0, c1);
-        int ncta = 0;
-        for (int c = c0; c <= c1; ++c) ncta += share_nonempty(c, T, P);
-        __threadfence();
-        last = atomicAdd(p.ws_hdr + g, 1) == ncta - 1;
-      }
-      if (!__shfl_sync(0xffffffffu, last, 0)) continue;
-      int slot = 0;
-      if (lane == 0) slot = atomicAdd(const_cast<int*>(pend), 1);
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-      if (slot < C::MAX_PEND) {
-        if (lane == 0) pend[2 + slot] = g;
-      } else {  // a full queue: this warp merges the group now
-        for (int h = 0; h < G; ++h) merge_group_head(ma, pre, g, h, G, NW, lane);
-      }
-    }
-    __syncwarp();
-    mbar_arrive_if(fin2_bar, lane == 0);
-    if (!mbar_wait_bounded(fin2_bar, 0, nullptr)) {
-      if (lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
-      return;
-    }
-    const int npend = min((int)pend[0], (int)C::MAX_PEND);
-    for (int i = warp; i < npend * G; i += NW) merge_group_head(ma, pre, pend[2 + i / G], i % G, G, NW, lane);
+    persistent_arrivals_and_merges(ma, pre, pend, C::MAX_PEND, cur_g, fin2_bar, p.status, G, NW, warp, lane);
     return;
   }
   // Split schedule: the CTAs of a cluster are the S pieces of one group, and

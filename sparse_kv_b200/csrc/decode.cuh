@@ -83,9 +83,9 @@ __host__ __device__ inline int art_positions(const DecodeParams& p, int L) {
 
 // Control words of the ART schedule: counter (4), stop chunk per group, ready
 // flag per chunk, blocks consumed and stop chunk per head, and per group the
-// re-fold count, the arrivals expected and the arrivals so far (the merge).
+// arrivals expected and the arrivals so far (the merge).
 inline long long art_ctl_words(long long groups, long long maxc, int G) {
-  return 4 + groups + groups * maxc + 2 * groups * G + 3 * groups;
+  return 4 + groups + groups * maxc + 2 * groups * G + 2 * groups;
 }
 
 // Tiles of one KV group for the index-based traversals (natural / range /

@@ -270,7 +270,7 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
     # groups) span at most 1/12 of the walk, else 16.  The workspace of a
     # chunk length CB: zeroed control words (item counter, stop chunk per
     # group, ready flag per (group, chunk), consumed and stop per head, and the
-    # merge's re-fold count, expected and received arrivals per group), per
+    # merge's expected and received arrivals per group), per
     # (group, chunk) a look-back record (12 floats) and a partial record (132
     # floats) per head, and per resident CTA (148 SMs x 2) probes of CB blocks
     # x 8 warps x G heads x 12 floats and 8 warps' states of G x 132 floats,
@@ -288,7 +288,7 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
     for cb in (16, 32):
         maxc = -(-blocks // cb)
         items = groups * maxc
-        ctl = up((4 + groups + groups * maxc + 2 * groups * G + 3 * groups) * 4)
+        ctl = up((4 + groups + groups * maxc + 2 * groups * G + 2 * groups) * 4)
         lb = up(items * G * 12 * 4)
         scratch = ctas * (posts * cb * NW * G * 12 + posts * NW * G * 132) * 4
         sizes[cb] = ctl + lb + scratch + items * G * 132 * 4
