@@ -179,20 +179,20 @@ typedef struct {
  * partials); 0 if none.  Depends only on host-side fields. */
 SKV_API size_t skv_decode_workspace_size(const skv_decode_args* args);
 
-/* Kernels one attn_decode call launches for these arguments: 1 (every
- * schedule merges its own partials inside the walk), not counting the zeroing
- * of the workspace's control words (a device memset, persistent and ART
- * schedules); 0 if the arguments are invalid.  Depends only on host-side
- * fields; for profiling and accounting. */
+/* Kernels one attn_decode call launches for these arguments (1: the walk
+ * merges its own partials -- a query chunk, or the split schedule that small
+ * walks and segment lists take; 2: the walk, then the record merge), not
+ * counting the workspace zeroing (a device memset); 0 if the arguments are
+ * invalid.  Depends only on host-side fields; for profiling and accounting. */
 SKV_API int skv_decode_launches(const skv_decode_args* args);
 
 /* The launch plan attn_decode would follow for these arguments (host-side
  * fields only; nothing is launched).  For profiling, capacity planning and
  * tests. */
 typedef enum {
-  SKV_SCHED_PERSISTENT = 0, /* persistent CTAs over all tiles; a group's last arrival merges it */
+  SKV_SCHED_PERSISTENT = 0, /* persistent CTAs over all tiles, then the record merge */
   SKV_SCHED_CLUSTER = 1,    /* one cluster of `splits` CTAs per KV group, merged in-kernel */
-  SKV_SCHED_ART = 2,        /* ART: persistent CTAs over (chunk, group) items; merged in-kernel */
+  SKV_SCHED_ART = 2,        /* ART: persistent CTAs over (chunk, group) items, then the merge */
   SKV_SCHED_CHUNK = 3       /* query chunk (q_tokens > 1) on the tensor cores */
 } skv_schedule;
 
@@ -214,17 +214,13 @@ SKV_API skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_
  * {order, window, seg_start/seg_end, kv range}; ART only with natural or
  * `order` traversal.
  * Launch shapes (they follow from host-side fields only):
- *  - long walks: persistent CTAs (2 per SM) share all tiles; each warp
- *    writes a partial record per KV group it touched to the workspace and
- *    arrives on the group's counter (zeroed by a memset before the launch),
- *    and the warp whose arrival is the group's last merges its records;
+ *  - long walks: persistent CTAs (2 per SM) share all tiles, then a merge
+ *    kernel combines the partial records in the workspace;
  *  - small walks (at most 8 tiles per resident CTA) and segment lists: one
  *    thread-block cluster of up to 16 CTAs per KV group, merged inside the
  *    kernel through distributed shared memory (no workspace); a cluster size
  *    the device cannot hold at once is halved;
- *  - ART: persistent CTAs over (chunk, group) items; every chunk's record
- *    and re-fold counts as an arrival on its group, and the CTA whose arrival
- *    completes a group merges it at the end of its walk;
+ *  - ART: persistent CTAs over (chunk, group) items, then the merge kernel;
  *  - query chunks (q_tokens > 1): one tensor-core kernel.
  * skv_decode_launches and skv_decode_workspace_size report the kernels and
  * the scratch a call needs. */

@@ -152,7 +152,7 @@ skv_status make_plan(const skv_decode_args* a, Plan* pl) {
     const long long max_ctas = (long long)num_sms() * decode_ctas_per_sm(G);
     pl->n_ctas = (int)std::max<long long>(1, std::min<long long>(max_ctas, cdiv(t_est, 4)));
     const long long slots = pl->n_ctas + groups;
-    pl->hdr_bytes = (size_t)cdiv(groups * 4ll, 256) * 256;  // one arrival counter per KV group
+    pl->hdr_bytes = (size_t)cdiv((a->batch + 2) * 4ll, 256) * 256;
     pl->ws_bytes = pl->hdr_bytes + (size_t)slots * pl->nw * G * kRecFloats * sizeof(float);
   } else {
     // one cluster of `splits` CTAs per group, merged in distributed shared
@@ -181,7 +181,7 @@ size_t skv_decode_workspace_size(const skv_decode_args* args) {
 int skv_decode_launches(const skv_decode_args* args) {
   Plan pl;
   if (make_plan(args, &pl) != SKV_OK) return 0;
-  return 1;
+  return (pl.chunk || (!pl.art && pl.sched == SCHED_SPLIT)) ? 1 : 2;
 }
 
 skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* plan) {
@@ -190,7 +190,7 @@ skv_status skv_decode_plan_info(const skv_decode_args* args, skv_decode_plan* pl
   Plan pl;
   const skv_status st = make_plan(args, &pl);
   if (st != SKV_OK) return st;
-  plan->launches = 1;
+  plan->launches = (pl.chunk || (!pl.art && pl.sched == SCHED_SPLIT)) ? 1 : 2;
   plan->workspace_bytes = pl.ws_bytes;
   if (pl.chunk) {
     plan->schedule = SKV_SCHED_CHUNK;
@@ -268,21 +268,19 @@ skv_status attn_decode(const skv_decode_args* a, skv_stream_t stream) {
     p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes + pl.lb_bytes + pl.scratch_bytes);
     if (cudaMemsetAsync(ws, 0, pl.hdr_bytes, s) != cudaSuccess) return SKV_ECUDA;
     if (launch_art(p, pl.G, s) != 0) return SKV_ECUDA;
-    return SKV_OK;  // merged inside the kernel
   } else {
     p.ws_hdr = reinterpret_cast<int*>(ws);
     p.ws_rec = reinterpret_cast<float*>(ws + pl.hdr_bytes);
-    if (pl.sched == SCHED_PERSISTENT &&
-        cudaMemsetAsync(ws, 0, (size_t)a->batch * a->kv_heads * sizeof(int), s) != cudaSuccess)
-      return SKV_ECUDA;
     const unsigned long long wh = g_withhold.exchange(0ull);
     if (wh != 0ull) {
       p.withhold_cta = (int)(wh >> 32);
       p.withhold_entry = (int)(wh & 0xFFFFFFFFull);
     }
     if (launch_decode(p, pl.G, s) != 0) return SKV_ECUDA;
-    return SKV_OK;  // merged inside the kernel
+    if (pl.sched == SCHED_SPLIT) return SKV_OK;  // merged inside the kernel
   }
+  if (launch_merge_records(p, pl.G, s) != 0) return SKV_ECUDA;
+  return SKV_OK;
 }
 
 skv_status attn_select_centroids(const void* q, const void* centroids, const int32_t* cluster_off,

@@ -101,7 +101,7 @@ struct ArtCfg {  // shared-memory layout
   static constexpr int THREADS = (NW + 2) * 32;  // consumers, producer, arbiter
   // a stage: K rows, V rows, and the group's q rows (loaded with a chunk's first block)
   static constexpr size_t STAGE_BYTES = 2 * (size_t)kTileBytes + (size_t)G * kRowBytes;
-  static constexpr int NBAR = 2 * ST + 3 + 2 * kPosts;  // full, empty, fin, posted[], freed[], arb_done, fin2
+  static constexpr int NBAR = 2 * ST + 1 + 2 * kPosts;  // full, empty, fin, posted[], freed[]
   static constexpr size_t OFF_BAR = ST * STAGE_BYTES;
   static constexpr size_t OFF_META = up16(OFF_BAR + NBAR * 8);        // int4 [ST]
   static constexpr size_t OFF_FLAGS = up16(OFF_META + ST * 16);       // int [4]
@@ -111,11 +111,7 @@ struct ArtCfg {  // shared-memory layout
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;   // float2 [NW][G]
   static constexpr size_t OFF_WCTL = up16(OFF_A + (size_t)NW * G * 8);  // int [NW][8]
   static constexpr size_t OFF_LOCAL = OFF_WCTL + (size_t)NW * 8 * 4;    // float [CB][G][12] (arbiter)
-  static constexpr int MAX_EV = 63;    // counted records this CTA wrote (its arrivals)
-  static constexpr int MAX_PEND = 63;   // groups this CTA completes, merged at its end
-  static constexpr size_t OFF_EV = OFF_LOCAL + (size_t)CB * G * kProbeFloats * 4;  // int [1 + MAX_EV]
-  static constexpr size_t OFF_PEND = OFF_EV + (1 + MAX_EV) * 4;                      // int [1 + MAX_PEND]
-  static constexpr size_t TOTAL = OFF_PEND + (1 + MAX_PEND) * 4;
+  static constexpr size_t TOTAL = OFF_LOCAL + (size_t)CB * G * kProbeFloats * 4;
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_P % 16 == 0, "alignment");
   static_assert(OFF_A % 16 == 0 && OFF_WCTL % 16 == 0 && OFF_LOCAL % 16 == 0, "alignment");
   static_assert(OFF_TAG % 16 == 0 && OFF_REQ % 16 == 0, "alignment");
@@ -157,8 +153,6 @@ struct Ctl {
   int* ready;
   int* consumed;
   int* head_stop;
-  int* need;   // arrivals that complete the group's records (0: not known yet)
-  int* done;   // arrivals so far
   __device__ Ctl(const DecodeParams& p, int G) {
     const int groups = p.B * p.Hkv;
     counter = p.art_ctl;
@@ -166,77 +160,8 @@ struct Ctl {
     ready = stop_chunk + groups;
     consumed = ready + (size_t)groups * p.art_maxc;
     head_stop = consumed + (size_t)groups * G;
-    need = head_stop + (size_t)groups * G;
-    done = need + groups;
   }
 };
-
-// What the end-of-walk merge reads (passed by value: no copy of the kernel's
-// parameters to local memory).
-struct ArtMergeArgs {
-  const float* rec;      // records [group][chunk][G][kRecFloats]
-  const int* seq_lens;
-  const int* head_stop;  // stop chunk + 1 per (group, head), 0: none
-  const int* consumed;   // blocks consumed per (group, head)
-  float* out;
-  float* lse;
-  int* blocks_consumed;
-  int Hq, Hkv, maxc, max_seq_len, mode, order_len;
-};
-
-// Merge head h of KV group g (one warp): the records of the chunks up to the
-// head's stop (or the whole walk), combined exactly ("Pulsar Attention" Phase
-// 2 in base 2); writes the output row, its lse and the blocks consumed.
-__device__ __noinline__ void art_merge_head(const ArtMergeArgs a, int g, int h, int G, int CB, int lane) {
-  __threadfence();  // every record was written before its arrival
-  const int b = g / a.Hkv, kvh = g % a.Hkv;
-  int L = a.seq_lens[b];
-  if (L < 0 || L > a.max_seq_len) L = 0;
-  const int nbk = (L + 63) / 64;
-  const int positions = nbk == 0 ? 0 : (a.mode == TRAV_ORDER ? 1 + a.order_len : nbk);
-  int nch = (positions + CB - 1) / CB;
-  const int sc = a.head_stop[(size_t)g * G + h];  // the head's stop chunk + 1 (0: none)
-  if (sc != 0 && sc < nch) nch = sc;
-  auto rec = [&](int c) { return a.rec + (((size_t)g * a.maxc + c) * G + h) * kRecFloats; };
-  float M = -INFINITY;
-  for (int c = lane; c < nch; c += 32) {
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(rec(c) + 128));
-    if (ml.y > 0.f) M = fmaxf(M, ml.x);
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float Wl = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY) {
-    for (int c0 = 0; c0 < nch; c0 += 8) {
-      float2 ml[8];
-      float4 x[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {  // 8 records' loads in flight
-        const bool v = c0 + q < nch;
-        ml[q] = v ? __ldcg(reinterpret_cast<const float2*>(rec(c0 + q) + 128)) : make_float2(0.f, 0.f);
-        x[q] = v ? __ldcg(reinterpret_cast<const float4*>(rec(c0 + q) + lane * 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float f = (ml[q].y > 0.f) ? exp2f(ml[q].x - M) : 0.f;
-        Wl += ml[q].y * f;
-        acc.x += x[q].x * f;
-        acc.y += x[q].y * f;
-        acc.z += x[q].z * f;
-        acc.w += x[q].w * f;
-      }
-    }
-  }
-  const size_t row = (size_t)b * a.Hq + (size_t)kvh * G + h;
-  const float inv = (Wl > 0.f) ? 1.f / Wl : 0.f;
-  *reinterpret_cast<float4*>(a.out + row * kHeadDim + lane * 4) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (lane == 0) {
-    a.lse[row] = (Wl > 0.f) ? (M + log2f(Wl)) * 0.6931471805599453f : -INFINITY;
-    if (a.blocks_consumed) a.blocks_consumed[row] = a.consumed[(size_t)g * G + h];
-  }
-}
 
 template <int G, int NW, int CB, int ST, int MINB>
 __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kernel(const DecodeParams p) {
@@ -247,10 +172,6 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   uint64_t* fin_bar = empty + ST;
   uint64_t* posted = fin_bar + 1;   // [kPosts] a post is ready (one arrival per consumer warp)
   uint64_t* freed = posted + kPosts;  // [kPosts] the arbiter is done with a post
-  uint64_t* arb_done = freed + kPosts;  // the arbiter has left its loop (its arrivals are listed)
-  uint64_t* fin2_bar = arb_done + 1;    // NW arrivals: the merge queue is complete
-  volatile int* ev = reinterpret_cast<volatile int*>(smem + C::OFF_EV);      // [0]: count, then groups
-  volatile int* pend = reinterpret_cast<volatile int*>(smem + C::OFF_PEND);  // [0]: count, then groups
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);  // {rows | 0 = end of chunk, group, chunk, block in chunk | blocks}
   volatile int* flags = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   // flags[0]: re-fold requests posted by the arbiter; flags[1]: abort (a bounded
@@ -266,10 +187,6 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int groups = p.B * p.Hkv;
   const Ctl ctl(p, G);
-  auto merge_args = [&]() {
-    return ArtMergeArgs{p.ws_rec, p.seq_lens, ctl.head_stop, ctl.consumed, p.out, p.lse, p.blocks_consumed,
-                        p.Hq, p.Hkv, p.art_maxc, p.max_seq_len, p.mode, p.order_len};
-  };
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
@@ -280,10 +197,6 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       mbar_init(&posted[i], NW);
       mbar_init(&freed[i], 1);
     }
-    mbar_init(arb_done, 1);
-    mbar_init(fin2_bar, NW);
-    ev[0] = 0;
-    pend[0] = 0;
     flags[0] = flags[1] = flags[2] = flags[3] = 0;
     fence_barrier_init();
   }
@@ -644,11 +557,8 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     // inclusive prefix; returns the heads that stop in the chunk, their stop
     // blocks in st_out (-1: none).  SEG lanes per head (lane t: block t), so
     // 32 / SEG heads per pass.
-    // *counted: the chunk is one of the group's chunks up to its last stop (some
-    // head was still live), so its record takes part in the merge.
     auto evaluate = [&](const float* loc, int g, int c, uint32_t vmask, bool last_chunk,
-                        int* st_out, bool* counted) -> uint32_t {
-      *counted = false;
+                        int* st_out) -> uint32_t {
       constexpr int SEG = CB <= 8 ? 8 : (CB <= 16 ? 16 : 32);
       constexpr int HPP = 32 / SEG;
       const size_t item = (size_t)g * p.art_maxc + c;
@@ -677,7 +587,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       const int sub = lane / SEG, t = lane % SEG, base = sub * SEG;
       const uint32_t segmask = (SEG == 32) ? 0xffffffffu : ((1u << SEG) - 1u);
       uint32_t stopmask = 0;
-      bool all = true, any_live = false;
+      bool all = true;
       for (int h0 = 0; h0 < G; h0 += HPP) {
         const int h = h0 + sub;
         const bool hv = h < G;
@@ -694,7 +604,6 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         const float Px[8] = {P0.z, P0.w, P1.x, P1.y, P1.z, P1.w, P2.x, P2.y};
         const int P_run = __float_as_int(P2.z), P_state = __float_as_int(P2.w);
         const bool live = hv && P_state >= 0;
-        any_live |= __any_sync(0xffffffffu, live);
         // chunk-local prefix after block t, then the global prefix
         const bool valid = live && t < CB && ((vmask >> t) & 1u);
         float M = -INFINITY, Ls = 0.f, X[8];
@@ -821,48 +730,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         }
         st_release(ctl.ready + item, 1);
       }
-      // Merge bookkeeping.  If the group ends here (every head has stopped, or
-      // this is the walk's last chunk), the arrivals that complete its records
-      // are known: one per chunk up to this one, and one per re-fold, i.e. per
-      // distinct stop chunk among the heads (earlier chunks' stops are visible:
-      // their deciders wrote them before releasing the ready flags acquired
-      // above; this chunk's were written by this warp).
-      if (any_live && ((all && stopmask) || last_chunk)) {
-        __syncwarp();
-        const int hs = lane < G ? *reinterpret_cast<volatile int*>(ctl.head_stop + (size_t)g * G + lane) : 0;
-        bool first = hs != 0;
-#pragma unroll
-        for (int j = 0; j < G - 1; ++j) {
-          const int o = __shfl_sync(0xffffffffu, hs, j);
-          if (j < lane && o == hs) first = false;
-        }
-        const int nf = __popc(__ballot_sync(0xffffffffu, first && lane < G));
-        if (lane == 0) st_release(ctl.need + g, c + 1 + nf);
-      }
-      *counted = any_live;
       return stopmask;
-    };
-
-    // One counted record of group g (a chunk's, or a re-fold's) is written: note
-    // it; the CTA's arrivals are made at the end of its walk, in one batch.
-    // A full list arrives at once (and merges here if that completes g).
-    auto arrive = [&](int g) {
-      __syncwarp();
-      int full_now = 0;
-      if (lane == 0) {
-        const int n = ev[0];
-        if (n < C::MAX_EV) {
-          ev[1 + n] = g;
-          ev[0] = n + 1;
-        } else {
-          __threadfence();
-          const int v = atomicAdd(ctl.done + g, 1) + 1;
-          __threadfence();
-          full_now = v == *reinterpret_cast<volatile int*>(ctl.need + g);
-        }
-      }
-      if (__shfl_sync(0xffffffffu, full_now, 0))
-        for (int h = 0; h < G; ++h) art_merge_head(merge_args(), g, h, G, CB, lane);
     };
 
     while (true) {
@@ -879,8 +747,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         merge_probes(probe + (size_t)par * probe_floats<G, NW, CB>(), (uint32_t)tg_a);
         __syncwarp();  // the chunk-local prefixes are visible to every lane
         int st[G];
-        bool counted = false;
-        const uint32_t stopmask = evaluate(local, tg_g, tg_c, (uint32_t)tg_a, last_chunk, st, &counted);
+        const uint32_t stopmask = evaluate(local, tg_g, tg_c, (uint32_t)tg_a, last_chunk, st);
         if (stopmask) {
           if (n_req - n_fix >= kReqs) {
             if (lane == 0) fail();  // cannot happen: the consumers serve requests every chunk
@@ -901,10 +768,8 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         }
         // the chunk's records (after the decision: they are not on its path)
         reduce_states(st_area, tg_g, tg_c, (1u << G) - 1u);
-        if (counted) arrive(tg_g);
       } else if (kind == POST_FIX) {
         reduce_states(st_area, tg_g, tg_c, (uint32_t)tg_a);
-        arrive(tg_g);
         ++n_fix;
       } else if (kind == POST_QUIT) {
         __syncwarp();
@@ -915,24 +780,10 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
       ++kj;
       if (kind == POST_DONE) break;
     }
-    __threadfence();  // the records written above, before the CTA's arrivals
-    __syncwarp();
-    mbar_arrive_if(arb_done, lane == 0);
     return;
   }
 
   // ------------------------------------------------------------------ consumers
-  // sequences without a block are in no item: CTA 0 writes their (empty) rows
-  if (blockIdx.x == 0) {
-    for (int r = threadIdx.x; r < p.B * p.Hq; r += NW * 32) {
-      const int L = p.seq_lens[r / p.Hq];
-      if (L > 0 && L <= p.max_seq_len) continue;
-      float4* o = reinterpret_cast<float4*>(p.out + (size_t)r * kHeadDim);
-      for (int j = 0; j < kHeadDim / 4; ++j) o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      p.lse[r] = -INFINITY;
-      if (p.blocks_consumed) p.blocks_consumed[r] = 0;
-    }
-  }
   Warp<G, NW> W;
   W.setup(warp, lane);
   const int rb = warp * C::RPW;
@@ -1086,39 +937,10 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   }
   __syncwarp();
   mbar_arrive_if(fin_bar, lane == 0);
-  const bool fin_ok = mbar_wait_bounded(fin_bar, 0, nullptr);
-  if (warp == 0 && lane == 0) {
-    if (!fin_ok) dev_error(p.status, SKV_DEV_TIMEOUT);
-    flags[2] = (flags[1] != 0) ? 1 : e + 1;
+  if (warp == 0) {
+    if (!mbar_wait_bounded(fin_bar, 0, nullptr) && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+    if (lane == 0) flags[2] = (flags[1] != 0) ? 1 : e + 1;
   }
-  // Once the arbiter has left its loop: the CTA's arrivals (one per counted
-  // record it wrote); an arrival that completes a group queues it, and the
-  // warps merge the queued groups, one (group, head) per warp.
-  if (!mbar_wait_bounded(arb_done, 0, nullptr)) {
-    if (lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
-    return;
-  }
-  const int nev = min((int)ev[0], (int)C::MAX_EV);
-  for (int i = warp; i < nev; i += NW) {
-    if (lane != 0) continue;
-    const int g = ev[1 + i];
-    __threadfence();
-    const int v = atomicAdd(ctl.done + g, 1) + 1;
-    __threadfence();
-    if (v == *reinterpret_cast<volatile int*>(ctl.need + g)) {
-      const int slot = atomicAdd(const_cast<int*>(pend), 1);
-      if (slot < C::MAX_PEND) pend[1 + slot] = g;
-      else dev_error(p.status, SKV_DEV_TIMEOUT);  // MAX_PEND >= MAX_EV: cannot happen
-    }
-  }
-  __syncwarp();
-  mbar_arrive_if(fin2_bar, lane == 0);
-  if (!mbar_wait_bounded(fin2_bar, 0, nullptr)) {
-    if (lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
-    return;
-  }
-  const int npend = min((int)pend[0], (int)C::MAX_PEND);
-  for (int i = warp; i < npend * G; i += NW) art_merge_head(merge_args(), pend[1 + i / G], i % G, G, CB, lane);
 }
 
 // Resident CTAs per SM, and the deepest ring (up to 6 stages) that fits in

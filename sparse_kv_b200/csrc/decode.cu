@@ -12,14 +12,12 @@
 // online-softmax state (m, l, O) for the G query heads of the group (the warp
 // arithmetic is in tile.cuh).
 //
-// Schedules.  Long index-based walks run persistently: two CTAs per SM take
-// even shares of the concatenated tile lists of all KV groups (a share may
+// Schedules.  Index-based traversals run persistently: one CTA per SM takes
+// an even share of the concatenated tile lists of all KV groups (a share may
 // span group boundaries; consumers then write a partial record per warp and
-// start the next group without any CTA-wide synchronisation).  Each warp
-// arrives on its group's counter after writing its record, and the last
-// arrival merges the group's records into the output, so one launch does the
-// whole walk.  Small walks and segment lists split each group across a
-// thread-block cluster and merge in distributed shared memory.
+// start the next group without any CTA-wide synchronisation).  Segment lists
+// split each group across a fixed number of CTAs.  Both end with an exact
+// merge of the per-warp records (launch_merge_records).
 #include "common.cuh"
 #include "decode.cuh"
 #include "tile.cuh"
@@ -51,9 +49,13 @@ struct Trav {
   int ra, re;      // natural / range token interval
   int A, Rs, nt1;  // window: [0, A) then [Rs, L)
   const int* ord;
+  // segments
+  const int* ss;
+  const int* se;
+  int seg_i, seg_end_i, seg_pos, seg_stop;
 
-  // Whole traversal of group (b, kvh), then narrowed with set_range (tile
-  // indices).  Segment lists are walked by the producer warp directly.
+  // Whole traversal of group (b, kvh), then narrowed with set_range
+  // (index-based modes: tile indices; segments: segment indices).
   __device__ void init(const DecodeParams& p, int b, int kvh, int L_, int split) {
     mode = p.mode;
     L = L_;
@@ -61,6 +63,7 @@ struct Trav {
     bt = p.block_table + (size_t)b * p.max_blocks;
     num_pages = p.num_pages;
     ord = nullptr;
+    seg_pos = seg_stop = 0;
     const int grp = b * p.Hkv + kvh;
     int N = 0;
     if (mode == TRAV_NATURAL) {
@@ -79,20 +82,75 @@ struct Trav {
     } else if (mode == TRAV_ORDER) {
       ord = p.order + (size_t)grp * p.order_len;
       N = p.order_len;
+    } else {  // segments
+      ss = p.seg_start + (size_t)grp * p.n_seg;
+      se = p.seg_end + (size_t)grp * p.n_seg;
+      N = p.n_seg;
     }
     const int S = p.n_splits > 0 ? p.n_splits : 1;
     set_range((int)(((long long)split * N) / S), (int)(((long long)(split + 1) * N) / S));
   }
 
   __device__ void set_range(int lo, int hi) {
-    i = lo;
-    i_end = hi;
+    if (mode == TRAV_SEGMENTS) {
+      seg_i = lo;
+      seg_end_i = hi;
+      seg_pos = seg_stop = 0;
+    } else {
+      i = lo;
+      i_end = hi;
+    }
+  }
+
+  // Segment lists: the next piece = up to 64 consecutive tokens inside one
+  // page (page, first row, rows).  Used to pack several segments into one tile.
+  __device__ bool next_piece(int& page, int& r0, int& cnt, uint32_t* status) {
+    while (true) {
+      if (seg_pos >= seg_stop) {
+        if (seg_i >= seg_end_i) return false;
+        const int s = ss[seg_i], t = se[seg_i];
+        ++seg_i;
+        if (s > t) {
+          dev_error(status, SKV_DEV_BAD_SEGMENT);
+          continue;
+        }
+        seg_pos = max(s, 0);
+        seg_stop = min(t, L);
+        continue;
+      }
+      const int blk = seg_pos / kBlock;
+      r0 = seg_pos % kBlock;
+      cnt = min(kBlock - r0, seg_stop - seg_pos);
+      seg_pos += cnt;
+      page = bt[blk];
+      if (page < 0 || page >= num_pages) {
+        dev_error(status, SKV_DEV_BAD_PAGE);
+        continue;
+      }
+      return true;
+    }
   }
 
   __device__ bool next(int& t0, int& n, int& pg1, int& pg2, int& n1, uint32_t* status) {
     while (true) {
       int a, e;
-      if (mode == TRAV_ORDER) {
+      if (mode == TRAV_SEGMENTS) {
+        if (seg_pos >= seg_stop) {
+          if (seg_i >= seg_end_i) return false;
+          int s = ss[seg_i], t = se[seg_i];
+          ++seg_i;
+          if (s > t) {
+            dev_error(status, SKV_DEV_BAD_SEGMENT);
+            continue;
+          }
+          seg_pos = max(s, 0);
+          seg_stop = min(t, L);
+          continue;
+        }
+        a = seg_pos;
+        e = min(seg_pos + kBlock, seg_stop);
+        seg_pos = e;
+      } else if (mode == TRAV_ORDER) {
         if (i >= i_end) return false;
         const int j = ord[i++];
         if (j < 0 || j >= nb) {
@@ -191,9 +249,7 @@ struct Cfg {
   static constexpr size_t OFF_A = OFF_P + (size_t)NW * RPW * G * 8;        // float2 [NW][G]
   static constexpr size_t OFF_PRE = OFF_A + (size_t)NW * G * 8;            // int [B+1], int [B]
   static constexpr size_t N_PRE = (2 * (size_t)kMaxPersistentBatch + 1) * 4;
-  static constexpr int MAX_PEND = 255;                                     // groups queued for the merge
-  static constexpr size_t OFF_PEND = (OFF_PRE + N_PRE + 15) / 16 * 16;     // int [2 + MAX_PEND]
-  static constexpr size_t TOTAL = OFF_PEND + (2 + MAX_PEND) * 4;
+  static constexpr size_t TOTAL = OFF_PRE + N_PRE;
   static_assert(TOTAL <= (MINB == 2 ? 113 : 227) * 1024, "shared memory budget");
   // every region read or written with 16-byte vectors starts 16-byte aligned
   static_assert(OFF_BAR % 16 == 0 && OFF_META % 16 == 0 && OFF_FLAGS % 16 == 0, "alignment");
@@ -201,137 +257,6 @@ struct Cfg {
   static_assert((RPW * G * 8) % 16 == 0 || G == 1, "pbuf rows");
   static_assert((kRecFloats * 4) % 16 == 0, "record strides");
 };
-
-// Persistent schedule, group merge.  A group's tiles are shared by the CTAs
-// c0..c1 (those with a non-empty share); each of their NW consumer warps
-// leaves a partial record (O unnormalised, m in base 2, l, tiles).  At the end
-// of its walk a CTA arrives once on the counter of every group it touched; the
-// CTA whose arrival is the group's last merges it, one (group, head) pair per
-// warp (the "Pulsar Attention" Phase 2 combination, in base 2).
-struct MergeArgs {
-  int* cnt;
-  const float* rec;
-  float* out;
-  float* lse;
-  int* consumed;
-  int B, Hq, Hkv, n_ctas;
-};
-
-__device__ __forceinline__ bool share_nonempty(long long c, long long T, long long P) {
-  return (c * T) / P != ((c + 1) * T) / P;
-}
-__device__ __forceinline__ void group_ctas(const int* pre, int B, int Hkv, int n_ctas, int g, int& c0,
-                                           int& c1) {
-  const long long T = pre[B], P = n_ctas;
-  const int b = g / Hkv, kvh = g % Hkv;
-  const int nt = (pre[b + 1] - pre[b]) / Hkv;
-  const long long Tg = pre[b] + (long long)kvh * nt;
-  c0 = (int)(((Tg + 1) * P - 1) / T);
-  c1 = (int)(((Tg + nt) * P - 1) / T);
-}
-
-// Merge head h of group g (one warp; lane owns dims 4 lane .. 4 lane + 3).
-__device__ __noinline__ void merge_group_head(const MergeArgs p, const int* pre, int g, int h, int G,
-                                              int NW, int lane) {
-  __threadfence();  // every arrival followed its records: read them from L2
-  int c0, c1;
-  group_ctas(pre, p.B, p.Hkv, p.n_ctas, g, c0, c1);
-  const long long T = pre[p.B], P = p.n_ctas;
-  // CTAs c0 + i with a non-empty share, as a bit mask (spans of up to 32 CTAs;
-  // a longer span, from very short shares, asks for the rest one by one)
-  const uint32_t span = __ballot_sync(0xffffffffu, c0 + lane <= c1 && share_nonempty(c0 + lane, T, P));
-  auto live = [&](int i) { return i < 32 ? ((span >> i) & 1u) != 0 : share_nonempty(c0 + i, T, P); };
-  const int nrec = (c1 - c0 + 1) * NW;
-  auto rec = [&](int r) { return p.rec + (((size_t)(c0 + r / NW + g) * NW + r % NW) * G + h) * kRecFloats; };
-  // pass 1: (m, l, tiles) of 32 records per load round; max of m
-  float M = -INFINITY;
-  int tiles = 0;
-  for (int r0 = 0; r0 < nrec; r0 += 32) {
-    const int r = r0 + lane;
-    if (r < nrec && live(r / NW)) {
-      const float4 ml = __ldcg(reinterpret_cast<const float4*>(rec(r) + 128));
-      if (ml.y > 0.f) M = fmaxf(M, ml.x);
-      if (r % NW == 0) tiles += (int)ml.z;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
-  }
-  // pass 2: W = sum l 2^(m - M), O = sum O 2^(m - M), 8 records' loads in flight
-  float Wl = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY) {
-    for (int r0 = 0; r0 < nrec; r0 += 8) {
-      float4 ml[8], x[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int r = r0 + q;
-        const bool v = r < nrec && live(r / NW);
-        ml[q] = v ? __ldcg(reinterpret_cast<const float4*>(rec(r) + 128)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        x[q] = v ? __ldcg(reinterpret_cast<const float4*>(rec(r) + lane * 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float f = (ml[q].y > 0.f) ? exp2f(ml[q].x - M) : 0.f;
-        Wl += ml[q].y * f;
-        acc.x += x[q].x * f;
-        acc.y += x[q].y * f;
-        acc.z += x[q].z * f;
-        acc.w += x[q].w * f;
-      }
-    }
-  }
-  const int b = g / p.Hkv, kvh = g % p.Hkv;
-  const size_t row = (size_t)b * p.Hq + (size_t)kvh * G + h;
-  const float inv = (Wl > 0.f) ? 1.f / Wl : 0.f;
-  *reinterpret_cast<float4*>(p.out + row * kHeadDim + lane * 4) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (lane == 0) {
-    p.lse[row] = (Wl > 0.f) ? (M + log2f(Wl)) * 0.6931471805599453f : -INFINITY;
-    if (p.consumed) p.consumed[row] = tiles;
-  }
-}
-
-// End of a CTA's persistent walk (every consumer warp): one arrival per group
-// the CTA touched (groups pend[1] .. last_g); an arrival that completes a group
-// queues it (pend[0] entries from pend[2]); then the warps merge the queued
-// groups, one (group, head) per warp.  Out of line: it runs once per CTA.
-__device__ __noinline__ void persistent_arrivals_and_merges(const MergeArgs ma, const int* pre,
-                                                            volatile int* pend, int max_pend, int last_g,
-                                                            uint64_t* fin2_bar, uint32_t* status, int G,
-                                                            int NW, int warp, int lane) {
-  const long long T = pre[ma.B], P = ma.n_ctas;
-  for (int g = pend[1] + warp; g <= last_g; g += NW) {
-    int last = 0;
-    if (lane == 0) {
-      int c0, c1;
-      group_ctas(pre, ma.B, ma.Hkv, ma.n_ctas, g, c0, c1);
-      int ncta = 0;
-      for (int c = c0; c <= c1; ++c) ncta += share_nonempty(c, T, P);
-      __threadfence();
-      last = atomicAdd(ma.cnt + g, 1) == ncta - 1;
-    }
-    if (!__shfl_sync(0xffffffffu, last, 0)) continue;
-    int slot = 0;
-    if (lane == 0) slot = atomicAdd(const_cast<int*>(pend), 1);
-    slot = __shfl_sync(0xffffffffu, slot, 0);
-    if (slot < max_pend) {
-      if (lane == 0) pend[2 + slot] = g;
-    } else {  // a full queue: this warp merges the group now
-      for (int h = 0; h < G; ++h) merge_group_head(ma, pre, g, h, G, NW, lane);
-    }
-  }
-  __syncwarp();
-  mbar_arrive_if(fin2_bar, lane == 0);
-  if (!mbar_wait_bounded(fin2_bar, 0, nullptr)) {
-    if (lane == 0) dev_error(status, SKV_DEV_TIMEOUT);
-    return;
-  }
-  const int npend = min((int)pend[0], max_pend);
-  for (int i = warp; i < npend * G; i += NW) merge_group_head(ma, pre, pend[2 + i / G], i % G, G, NW, lane);
-}
 
 template <int G, int NW, int MINB>
 __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel(const DecodeParams p) {
@@ -342,8 +267,7 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
   uint64_t* empty = full + ST;
   uint64_t* fin_bar = empty + ST;  // NW arrivals: the consumers are done with the ring
   // split schedule only:
-  uint64_t* fin2_bar = fin_bar + 1;     // NW arrivals: split: the warps' states are in the ring;
-                                        // persistent: the merge queue is complete
+  uint64_t* fin2_bar = fin_bar + 1;     // NW arrivals: the warps' states are in the ring
   uint64_t* fin3_bar = fin2_bar + 1;    // NW arrivals: the piece's records are written
   uint64_t* fin4_bar = fin3_bar + 1;    // G arrivals: (rank 0) the merge is done
   uint64_t* gather_bar = fin4_bar + 1;  // (rank 0) S arrivals, one per piece of the cluster
@@ -366,7 +290,6 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     mbar_init(gather_bar, p.sched == SCHED_SPLIT ? p.n_splits : 1);
     mbar_init(release_bar, 1);
     flags[0] = flags[1] = flags[2] = 0;
-    *reinterpret_cast<volatile int*>(smem + C::OFF_PEND) = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -404,23 +327,12 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       }
       if (lane == 0) pre[p.B] = run;
       __syncwarp();
-      // sequences without a tile belong to no CTA's share: CTA 0 writes their
-      // (empty) results
       if (blockIdx.x == 0) {
-        for (int r = lane; r < p.B * p.Hq; r += 32) {
-          const int b = r / p.Hq;
-          if (pre[b + 1] != pre[b]) continue;
-          float4* o = reinterpret_cast<float4*>(p.out + (size_t)r * kHeadDim);
-          for (int j = 0; j < kHeadDim / 4; ++j) o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-          p.lse[r] = -INFINITY;
-          if (p.blocks_consumed) p.blocks_consumed[r] = 0;
-        }
+        if (lane == 0) p.ws_hdr[0] = run;
+        for (int b = lane; b <= p.B; b += 32) p.ws_hdr[1 + b] = pre[b];
       }
     }
-    // Segment lists are walked by the whole warp (bounds and pages fetched for
-    // 32 segments at a time); every other traversal by lane 0 alone.
-    const bool seg_mode = p.mode == TRAV_SEGMENTS;
-    if (lane != 0 && !seg_mode) return;
+    if (lane != 0) return;
 
     const uint64_t pol = policy_evict_first();
     const size_t head_stride = (size_t)kBlock * kHeadDim;
@@ -512,96 +424,38 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       }
       return true;
     };
-    // Segment lists (whole warp): lane i loads the bounds of segment base + i
-    // and the pages of its first and last block, so one round trip to memory
-    // serves 32 segments; lane 0 then packs their rows into full 64-row tiles
-    // (attention over a key set does not depend on the keys' order), one bulk
-    // copy per piece (<= 64 consecutive tokens of one page).  Pages inside a
-    // segment longer than two blocks are looked up as lane 0 reaches them.
-    auto run_segments_warp = [&](int b, int kvh, int L, int g, int slot, int split) -> bool {
-      const int grp = b * p.Hkv + kvh;
-      const int* ss = p.seg_start + (size_t)grp * p.n_seg;
-      const int* se = p.seg_end + (size_t)grp * p.n_seg;
-      const int* bt = p.block_table + (size_t)b * p.max_blocks;
-      const int S = p.n_splits > 0 ? p.n_splits : 1;
-      const int lo = (int)(((long long)split * p.n_seg) / S);
-      const int hi = (int)(((long long)(split + 1) * p.n_seg) / S);
+    auto run_segments = [&](Trav& tr, int g, int slot, int kvh) -> bool {
       int pg[kMaxPieces], r0[kMaxPieces], cnt[kMaxPieces];
       int np = 0, rows = 0, tiles = 0;
-      bool ok = true;
-      for (int base = lo; base < hi && ok; base += 32) {
-        const int i = base + lane;
-        int s0 = 0, s1 = 0, pa = 0, pb = 0;
-        if (i < hi) {
-          const int a = ss[i], e2 = se[i];
-          if (a > e2) dev_error(p.status, SKV_DEV_BAD_SEGMENT);
-          else {
-            s0 = max(a, 0);
-            s1 = min(e2, L);
-          }
-          if (s1 > s0) {
-            pa = bt[s0 / kBlock];
-            pb = bt[(s1 - 1) / kBlock];
-          } else {
-            s1 = s0;
-          }
-        }
-        const int n_in = min(32, hi - base);
-        for (int j = 0; j < n_in; ++j) {
-          const int a = __shfl_sync(0xffffffffu, s0, j), z = __shfl_sync(0xffffffffu, s1, j);
-          const int qa = __shfl_sync(0xffffffffu, pa, j), qb = __shfl_sync(0xffffffffu, pb, j);
-          int good = 1;
-          if (lane == 0) {
-            const int fb = a / kBlock, lb = (z - 1) / kBlock;
-            for (int pos = a; pos < z && good;) {
-              const int blk = pos / kBlock, first = pos % kBlock;
-              int c = min(kBlock - first, z - pos);
-              pos += c;
-              const int page = blk == fb ? qa : (blk == lb ? qb : bt[blk]);
-              if (page < 0 || page >= p.num_pages) {
-                dev_error(p.status, SKV_DEV_BAD_PAGE);
-                continue;
-              }
-              int f = first;
-              while (c > 0) {
-                const int take = min(c, kBlock - rows);
-                pg[np] = page;
-                r0[np] = f;
-                cnt[np] = take;
-                ++np;
-                rows += take;
-                f += take;
-                c -= take;
-                if (rows == kBlock || np == kMaxPieces) {
-                  if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) {
-                    good = 0;
-                    break;
-                  }
-                  ++tiles;
-                  np = rows = 0;
-                }
-              }
-            }
-          }
-          if (!__shfl_sync(0xffffffffu, good, 0)) {
-            ok = false;
-            break;
+      int page = 0, first = 0, c = 0;
+      while (tr.next_piece(page, first, c, p.status)) {
+        while (c > 0) {
+          const int take = min(c, kBlock - rows);
+          pg[np] = page;
+          r0[np] = first;
+          cnt[np] = take;
+          ++np;
+          rows += take;
+          first += take;
+          c -= take;
+          if (rows == kBlock || np == kMaxPieces) {
+            if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
+            ++tiles;
+            np = rows = 0;
           }
         }
       }
-      int r = ok ? 1 : 0;
-      if (lane == 0 && ok) {
-        if (rows > 0) {
-          if (emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) ++tiles;
-          else r = 0;
-        }
-        if (r && tiles == 0 && !emit(0, g, slot, kvh, 0, 0, 0, 0)) r = 0;
+      if (rows > 0) {
+        if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
+        ++tiles;
       }
-      return __shfl_sync(0xffffffffu, r, 0) != 0;
+      if (tiles == 0 && !emit(0, g, slot, kvh, 0, 0, 0, 0)) return false;
+      return true;
     };
     // All entries of one group segment; a segment without valid tiles still
     // issues a marker so that the consumers account for the group.
     auto run_group = [&](Trav& tr, int g, int slot, int kvh) -> bool {
+      if (tr.mode == TRAV_SEGMENTS) return run_segments(tr, g, slot, kvh);
       int t0 = 0, n = 0, pg1 = 0, pg2 = 0, n1 = 0, cnt = 0;
       while (tr.next(t0, n, pg1, pg2, n1, p.status)) {
         if (!emit(n, g, slot, kvh, t0, pg1, pg2, n1)) return false;
@@ -639,19 +493,14 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
       int L = p.seq_lens[b];
       if (L < 0 || L > p.max_seq_len) {
-        if (split == 0 && kvh == 0 && lane == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
+        if (split == 0 && kvh == 0) dev_error(p.status, SKV_DEV_BAD_SEQLEN);
         L = 0;
       }
+      Trav tr;
+      tr.init(p, b, kvh, L, split);
       const int g = b * p.Hkv + kvh;
-      if (seg_mode) {
-        ok = run_segments_warp(b, kvh, L, g, g * p.n_splits + split, split);
-      } else {
-        Trav tr;
-        tr.init(p, b, kvh, L, split);
-        ok = run_group(tr, g, g * p.n_splits + split, kvh);
-      }
+      ok = run_group(tr, g, g * p.n_splits + split, kvh);
     }
-    if (lane != 0) return;
     if (ok) emit(-1, -1, 0, 0, 0, 0, 0, 0);
     // Copies the consumers never waited for (abort) must land before the CTA
     // exits: learn how many entries they consumed, then drain the rest.
@@ -688,12 +537,6 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     }
   };
 
-  // Persistent schedule: the groups this CTA touched form a contiguous range
-  // (its share of the concatenated tile lists); warp 0 notes the first.
-  const int* pre = reinterpret_cast<const int*>(smem + C::OFF_PRE);
-  // [0]: queued groups, [1]: the first group of this CTA's share, [2..]: the queue
-  volatile int* pend = reinterpret_cast<volatile int*>(smem + C::OFF_PEND);
-
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P) + warp * C::RPW * G;
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
 
@@ -719,7 +562,6 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
     }
     if (mt.y != cur_g) {
       if (cur_g >= 0) flush(cur_slot, k);
-      else if (warp == 0 && lane == 0) pend[1] = mt.y;
       W.reset();
       const int b = mt.y / p.Hkv, kvh = mt.y % p.Hkv;
       W.load_q(p.q, (size_t)b * p.Hq + (size_t)kvh * G, p.qscale, lane);
@@ -746,22 +588,13 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
   // ------------------------------------------------------------------ epilogue
   if (p.sched == SCHED_PERSISTENT) {
     if (cur_g >= 0) flush(cur_slot, k);
-    // Every consumer warp ends here, its records written (and fenced): let the
-    // producer know once all are done.  Then the CTA arrives once on the
-    // counter of every group it touched; the arrival that completes a group
-    // (all CTAs whose share meets its tiles) queues it, and the warps merge
-    // the queued groups, one (group, head) per warp.
-    __threadfence();
+    // Every consumer warp ends here: let the producer know once all are done.
     __syncwarp();
     mbar_arrive_if(fin_bar, lane == 0);
-    const bool fin_ok = mbar_wait_bounded(fin_bar, 0, nullptr);
-    if (warp == 0 && lane == 0) {
-      if (!fin_ok) dev_error(p.status, SKV_DEV_TIMEOUT);
-      flags[2] = (flags[1] != 0) ? 1 : e + 1;
+    if (warp == 0) {
+      if (!mbar_wait_bounded(fin_bar, 0, nullptr) && lane == 0) dev_error(p.status, SKV_DEV_TIMEOUT);
+      if (lane == 0) flags[2] = (flags[1] != 0) ? 1 : e + 1;
     }
-    if (!fin_ok || cur_g < 0) return;
-    const MergeArgs ma{p.ws_hdr, p.ws_rec, p.out, p.lse, p.blocks_consumed, p.B, p.Hq, p.Hkv, p.n_ctas};
-    persistent_arrivals_and_merges(ma, pre, pend, C::MAX_PEND, cur_g, fin2_bar, p.status, G, NW, warp, lane);
     return;
   }
   // Split schedule: the CTAs of a cluster are the S pieces of one group, and

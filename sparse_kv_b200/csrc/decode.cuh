@@ -49,9 +49,8 @@ struct DecodeParams {
   float* lse;
   int* blocks_consumed;
   uint32_t* status;
-  // Persistent schedule's workspace: one arrival counter per KV group (zeroed
-  // before every launch) and per-warp partial records [slots][rec_nw][G][kRecFloats];
-  // the last warp to arrive for a group merges its records.
+  // Non-ART workspace: header (total tiles, batch prefix) and per-warp partial
+  // records [slots][rec_nw][G][kRecFloats], merged by launch_merge_records.
   int* ws_hdr;
   float* ws_rec;
   int rec_nw;
@@ -82,10 +81,9 @@ __host__ __device__ inline int art_positions(const DecodeParams& p, int L) {
 }
 
 // Control words of the ART schedule: counter (4), stop chunk per group, ready
-// flag per chunk, blocks consumed and stop chunk per head, and per group the
-// arrivals expected and the arrivals so far (the merge).
+// flag per chunk, blocks consumed and stop chunk per head.
 inline long long art_ctl_words(long long groups, long long maxc, int G) {
-  return 4 + groups + groups * maxc + 2 * groups * G + 2 * groups;
+  return 4 + groups + groups * maxc + 2 * groups * G;
 }
 
 // Tiles of one KV group for the index-based traversals (natural / range /
@@ -121,6 +119,7 @@ int art_ctas_per_sm(int G);
 size_t art_scratch_bytes_per_cta(int G, int CB);
 int launch_merge(const float* o_parts, const float* lse_parts, int S, int N, int d, float* out,
                  float* lse, void* stream);
+int launch_merge_records(const DecodeParams& p, int G, void* stream);
 int launch_chunk(const DecodeParams& p, int Tq, int causal, int n_shards, void* stream);
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int shared, int* ids, int* ss, int* se, void* stream);

@@ -46,9 +46,11 @@ def device_workload(wl, layer=0, nan_fill=True, keys=True, values=True):
 
 
 def outputs(wl, device="cuda"):
+    """Output buffers filled with NaN: a row the kernels never write cannot pass
+    as a stale copy of an earlier call's result."""
     import torch
-    out = torch.empty((wl.B, wl.Tq, wl.Hq, wl.d), dtype=torch.float32, device=device)
-    lse = torch.empty((wl.B, wl.Tq, wl.Hq), dtype=torch.float32, device=device)
+    out = torch.full((wl.B, wl.Tq, wl.Hq, wl.d), float("nan"), dtype=torch.float32, device=device)
+    lse = torch.full((wl.B, wl.Tq, wl.Hq), float("nan"), dtype=torch.float32, device=device)
     return out, lse
 
 

@@ -149,7 +149,7 @@ def test_workspace_size_query():
     L = skv.lib()
     full = good_args()
     n = L.skv_decode_workspace_size(ctypes.byref(full))
-    # arrival counters + per-warp partial records of 132 floats per head
+    # header (batch prefix) + per-warp partial records of 132 floats per head
     assert n > 0 and (n % 256) == 0 and n >= 16 * 8 * 16 * 4 * 132 * 4
     # ART: per (chunk, KV group): a look-back record of 12 floats and a partial
     # record of 132 floats per head, zeroed control words, and a scratch area of
@@ -169,14 +169,13 @@ def test_workspace_size_query():
 
 
 def test_decode_launch_count():
-    # one kernel in every schedule: the walk merges its own partials (large
-    # walks and ART: each group's last arrival queues it for a merge at the end
-    # of its CTA's walk; small walks and segment lists: the cluster's shared
-    # memory; a query chunk writes its results directly)
+    # one kernel where the walk merges its own partials (small walks and
+    # segment lists take the split schedule; a query chunk writes its results
+    # directly), two where a record merge follows (large walks, ART)
     L = skv.lib()
     n = lambda a: L.skv_decode_launches(ctypes.byref(a))
-    assert n(good_args()) == 1                                    # 128 groups x 512 tiles
-    assert n(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == 1
+    assert n(good_args()) == 2                                    # 128 groups x 512 tiles
+    assert n(good_args(art=_Art(1, 1e-3, 1e-4, 4))) == 2
     small = good_args(batch=1, q_heads=8, kv_heads=2, max_seq_len=4096, max_blocks=64)
     assert n(small) == 1                                          # 2 groups x 64 tiles
     # the split schedule merges its pieces in the cluster's shared memory: no workspace
@@ -248,15 +247,14 @@ def test_strerror():
 def test_plan_small_walks_take_the_cluster_schedule():
     # up to 8 tiles per resident CTA (148 SMs x 2 CTAs here) the walk runs as
     # one cluster per KV group and merges in-kernel; one tile more, and the
-    # persistent schedule (arrival counters and per-warp records in the
-    # workspace, merged by each group's last arrival) takes over
+    # persistent schedule with its record merge takes over
     L = skv.lib()
     small = 148 * 2 * 8  # tiles
     a = good_args(batch=1, q_heads=4, kv_heads=1, max_seq_len=small * 64, max_blocks=small)
     assert L.skv_decode_launches(ctypes.byref(a)) == 1
     assert L.skv_decode_workspace_size(ctypes.byref(a)) == 0
     b = good_args(batch=1, q_heads=4, kv_heads=1, max_seq_len=(small + 1) * 64, max_blocks=small + 1)
-    assert L.skv_decode_launches(ctypes.byref(b)) == 1
+    assert L.skv_decode_launches(ctypes.byref(b)) == 2
     assert L.skv_decode_workspace_size(ctypes.byref(b)) > 0
 
 
@@ -269,8 +267,7 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
     # The ART chunk is 32 blocks when the chunks in flight per group (CTAs /
     # groups) span at most 1/12 of the walk, else 16.  The workspace of a
     # chunk length CB: zeroed control words (item counter, stop chunk per
-    # group, ready flag per (group, chunk), consumed and stop per head, and the
-    # merge's expected and received arrivals per group), per
+    # group, ready flag per (group, chunk), consumed and stop per head), per
     # (group, chunk) a look-back record (12 floats) and a partial record (132
     # floats) per head, and per resident CTA (148 SMs x 2) probes of CB blocks
     # x 8 warps x G heads x 12 floats and 8 warps' states of G x 132 floats,
@@ -288,7 +285,7 @@ def test_plan_art_chunk_length(groups_b, hkv, blocks, want_cb):
     for cb in (16, 32):
         maxc = -(-blocks // cb)
         items = groups * maxc
-        ctl = up((4 + groups + groups * maxc + 2 * groups * G + 2 * groups) * 4)
+        ctl = up((4 + groups + groups * maxc + 2 * groups * G) * 4)
         lb = up(items * G * 12 * 4)
         scratch = ctas * (posts * cb * NW * G * 12 + posts * NW * G * 132) * 4
         sizes[cb] = ctl + lb + scratch + items * G * 132 * 4
@@ -304,10 +301,10 @@ def test_decode_plan_info():
         return p
 
     full = plan(good_args())  # 16 x 8 groups of 512 tiles
-    assert (full.schedule, full.ctas, full.splits, full.launches) == (0, 296, 0, 1)
+    assert (full.schedule, full.ctas, full.splits, full.launches) == (0, 296, 0, 2)
     assert full.workspace_bytes == L.skv_decode_workspace_size(ctypes.byref(good_args()))
     art = plan(good_args(art=_Art(1, 1e-3, 1e-4, 4)))
-    assert (art.schedule, art.ctas, art.art_chunk_blocks, art.art_chunks, art.launches) == (2, 296, 16, 32, 1)
+    assert (art.schedule, art.ctas, art.art_chunk_blocks, art.art_chunks, art.launches) == (2, 296, 16, 32, 2)
     art5 = plan(good_args(batch=8, max_seq_len=131072, max_blocks=2048, art=_Art(1, 1e-3, 1e-4, 4)))
     assert (art5.art_chunk_blocks, art5.art_chunks) == (32, 64)
     small = plan(good_args(batch=1, q_heads=8, kv_heads=2, max_seq_len=4096, max_blocks=64))
