@@ -123,7 +123,7 @@ int launch_merge_records(const DecodeParams& p, int G, void* stream);
 int launch_chunk(const DecodeParams& p, int Tq, int causal, int n_shards, void* stream);
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int shared, int* ids, int* ss, int* se, void* stream);
-int select_cluster_size(int groups_or_B, int C, int shared);
+int select_cluster_size(int B);
 int launch_forecast(const uint16_t* x, const uint16_t* w, int B, int Hkv, uint16_t* f, void* stream);
 int launch_gather(const void* k_host, const void* v_host, const int* block_table, const int* seq_lens,
                   const int* ids, int B, int Hkv, int k, int max_blocks, int num_pages, int max_seq_len,

@@ -7,21 +7,20 @@
 // scores, ties to the lower index, written in ascending id order with their
 // key ranges.
 //
-// Structure: a thread-block cluster of S CTAs shares the centroid rows of one
-// KV head: CTA r bulk-copies rows [r C / S, (r + 1) C / S) into a shared-memory
-// ring (no multicast) and scores them against every query it serves.  Each
+// Shared centroids (attn_select_centroids_shared): a thread-block cluster of S
+// CTAs shares the centroid rows of one KV head: CTA r bulk-copies rows
+// [r C / S, (r + 1) C / S) into a shared-memory ring (no multicast) and scores
+// them against every query it serves.  Each
 // score goes, as an order-preserving 32-bit key, straight into the shared
 // memory of the CTA that owns that query's selection (st.shared::cluster);
 // after its last row the CTA arrives remotely on every owner's gather barrier.
 // An owner then finds the k-th largest key by a radix select (8 bits per pass,
 // warp-aggregated histogram updates, early exit once the boundary digit holds
 // exactly the keys still needed) and writes the kept ids in ascending order.
-//   per-sequence centroids (attn_select_centroids): one cluster per KV group
-//     (b, kvh); its S CTAs split the group's centroids, rank 0 owns the query.
-//   shared centroids (attn_select_centroids_shared, "Squeezed Attention" Q1:
-//     one fixed context clustered once, reused by every request): one cluster
-//     per KV head and up to 8 requests; CTA j owns request j's selection, and
-//     every centroid row is read once for all of the cluster's requests.
+// One cluster per KV head and up to 8 requests ("Squeezed Attention" Q1: one
+// fixed context clustered once, reused by every request): CTA j owns request
+// j's selection, and every centroid row is read once for all of the cluster's
+// requests.
 #include "common.cuh"
 #include "decode.cuh"
 
@@ -46,13 +45,223 @@ constexpr size_t kOffBar = kOffScal + 16;
 constexpr size_t kSelSmem = kOffBar + (kSelStages + 1) * 8;
 static_assert(kOffKeys % 16 == 0 && kOffQ % 16 == 0 && kOffBar % 8 == 0, "alignment");
 
+// Per-sequence centroids (attn_select_centroids): one CTA per KV group (b, kvh),
+// the group's query heads summed once.  Centroid rows stream into shared
+// memory in 64 KiB chunks by bulk-async copies (two stages); each row is scored
+// by 16 lanes with 16-byte shared loads and a shuffle reduction.  A radix
+// select over order-preserving 32-bit score keys finds the k-th largest score;
+// the kept clusters are those above it plus the lowest-index ones equal to it,
+// written in ascending id order with their key ranges.  (Splitting a group's
+// centroids over a cluster of CTAs, as the shared-centroid kernel below does for
+// its requests, measured slower here: the radix select on one CTA per group is
+// the critical path, and the cluster's set-up and gather only add to it.)
+constexpr int kSeqThreads = 512;
+constexpr int kSeqMaxClusters = 4096;
+constexpr int kSeqChunk = 256;                             // centroids per stage
+constexpr int kSeqChunkBytes = kSeqChunk * kHeadDim * 2;      // 64 KiB
+constexpr int kSeqStages = 2;
+// shared memory: stages | keys u32[kSeqMaxClusters] | q sum f32[128] | flags u8[kSeqMaxClusters] |
+//                histogram int[256] | warp sums int[16] | scalars int[4] | mbarriers
+constexpr size_t kSeqOffKeys = (size_t)kSeqStages * kSeqChunkBytes;
+constexpr size_t kSeqOffQ = kSeqOffKeys + sizeof(uint32_t) * kSeqMaxClusters;
+constexpr size_t kSeqOffFlag = kSeqOffQ + 128 * 4;
+constexpr size_t kSeqOffHist = kSeqOffFlag + kSeqMaxClusters;
+constexpr size_t kSeqOffWsum = kSeqOffHist + 256 * 4;
+constexpr size_t kSeqOffScal = kSeqOffWsum + 16 * 4;
+constexpr size_t kSeqOffBar = kSeqOffScal + 16;
+constexpr size_t kSeqSmem = kSeqOffBar + kSeqStages * 8;
+
+// Order-preserving map of an fp32 score to an unsigned key.
+__device__ __forceinline__ uint32_t seq_score_key(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive prefix of per-thread counts (threads own contiguous
+// runs in index order); returns the thread's offset, total in *total.
+__device__ __forceinline__ int seq_block_scan(int cnt, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, m);
+    if (lane >= m) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int base = 0, tot = 0;
+  for (int w = 0; w < kSeqThreads / 32; ++w) {
+    if (w < warp) base += wsum[w];
+    tot += wsum[w];
+  }
+  __syncthreads();
+  *total = tot;
+  return base + incl - cnt;
+}
+
+__global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t* __restrict__ q,
+                                                            const uint16_t* __restrict__ cent,
+                                                            const int* __restrict__ off, int Hq,
+                                                            int Hkv, int C, int k, int* ids, int* ss,
+                                                            int* se) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t* key = reinterpret_cast<uint32_t*>(smem + kSeqOffKeys);
+  float* qs = reinterpret_cast<float*>(smem + kSeqOffQ);
+  unsigned char* flag = smem + kSeqOffFlag;
+  int* hist = reinterpret_cast<int*>(smem + kSeqOffHist);
+  int* wsum = reinterpret_cast<int*>(smem + kSeqOffWsum);
+  int* scal = reinterpret_cast<int*>(smem + kSeqOffScal);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kSeqOffBar);
+
+  const int g = blockIdx.x, b = g / Hkv, kvh = g % Hkv, G = Hq / Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nchunks = (C + kSeqChunk - 1) / kSeqChunk;
+  const unsigned char* cg = reinterpret_cast<const unsigned char*>(cent + (size_t)g * C * kHeadDim);
+
+  // Centroid rows stream through kSeqStages shared-memory stages by bulk copy.
+  auto issue = [&](int chunk) {
+    const int st = chunk % kSeqStages;
+    const int rows = min(kSeqChunk, C - chunk * kSeqChunk);
+    const uint32_t bytes = (uint32_t)rows * kHeadDim * 2;
+    mbar_arrive_expect_tx(&bar[st], bytes);
+    const unsigned char* src = cg + (size_t)chunk * kSeqChunkBytes;
+    unsigned char* dst = smem + (size_t)st * kSeqChunkBytes;
+    for (uint32_t o = 0; o < bytes; o += 16384)
+      bulk_load(dst + o, src + o, min(16384u, bytes - o), &bar[st], policy_evict_first());
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kSeqStages; ++i) mbar_init(&bar[i], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int i = 0; i < kSeqStages && i < nchunks; ++i) issue(i);
+
+  if (tid < kHeadDim) {
+    float sum = 0.f;
+    for (int h = 0; h < G; ++h)
+      sum += __uint_as_float((uint32_t)q[((size_t)b * Hq + kvh * G + h) * kHeadDim + tid] << 16);
+    qs[tid] = sum;
+  }
+  for (int c = tid; c < C; c += kSeqThreads) flag[c] = 0;
+  __syncthreads();
+
+  // ---- scores: 16 lanes per centroid row (8 dims each), 2 rows per warp step
+  const int ch = lane & 15;
+  float qv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) qv[e] = qs[ch * 8 + e];
+  for (int chunk = 0; chunk < nchunks; ++chunk) {
+    const int st = chunk % kSeqStages;
+    if (!mbar_wait_bounded(&bar[st], (chunk / kSeqStages) & 1, nullptr)) break;
+    const unsigned char* sc = smem + (size_t)st * kSeqChunkBytes;
+    const int rows = min(kSeqChunk, C - chunk * kSeqChunk);
+#pragma unroll 4
+    for (int rb = warp * 2; rb < rows; rb += (kSeqThreads / 32) * 2) {  // warp-uniform bound
+      const int r = rb + (lane >> 4);
+      const bool valid = r < rows;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) w = *reinterpret_cast<const uint4*>(sc + (size_t)r * kHeadDim * 2 + ch * 16);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      float acc = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc = fmaf(qv[2 * u], __uint_as_float(ws[u] << 16), acc);
+        acc = fmaf(qv[2 * u + 1], __uint_as_float(ws[u] & 0xFFFF0000u), acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      if (valid && ch == 0) key[chunk * kSeqChunk + r] = seq_score_key(acc);
+    }
+    __syncthreads();  // stage st fully read
+    if (tid == 0 && chunk + kSeqStages < nchunks) issue(chunk + kSeqStages);
+  }
+  __syncthreads();
+
+  // ---- radix select: the k-th largest key T, 8 bits at a time from the top
+  uint32_t prefix = 0, pmask = 0;
+  int kk = k;  // rank still to find below the fixed prefix
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kSeqThreads) hist[i] = 0;
+    __syncthreads();
+    for (int c = tid; c < C; c += kSeqThreads) {
+      const uint32_t kc = key[c];
+      if ((kc & pmask) == prefix) atomicAdd(&hist[(kc >> shift) & 0xFFu], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {  // bins from the top: find the digit holding rank kk
+      int cnt[8], run = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[255 - (lane * 8 + j)];
+        run += cnt[j];
+      }
+      int incl = run;  // inclusive prefix over lanes (bins in descending order)
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, m);
+        if (lane >= m) incl += y;
+      }
+      int before = incl - run;
+      const bool mine = before < kk && kk <= incl;
+      if (mine) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (before < kk && kk <= before + cnt[j]) {
+            scal[0] = 255 - (lane * 8 + j);  // digit
+            scal[1] = kk - before;           // rank within that digit
+          }
+          before += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= (uint32_t)scal[0] << shift;
+    pmask |= 0xFFu << shift;
+    kk = scal[1];
+    __syncthreads();
+  }
+  const uint32_t T = prefix;  // the k-th largest key; kk of the keys equal to T are taken
+
+  // ---- flags: keys above T, plus the first kk keys equal to T in index order
+  const int per = (C + kSeqThreads - 1) / kSeqThreads;
+  const int c0 = tid * per;
+  int nties = 0;
+  for (int c = c0; c < c0 + per && c < C; ++c) nties += (key[c] == T);
+  int tot = 0;
+  int tie_rank = seq_block_scan(nties, wsum, &tot);
+  int cnt = 0;
+  for (int c = c0; c < c0 + per && c < C; ++c) {
+    const uint32_t kc = key[c];
+    int f = kc > T;
+    if (kc == T) f = (tie_rank++ < kk);
+    flag[c] = (unsigned char)f;
+    cnt += f;
+  }
+
+  // ---- compact in ascending id order
+  int pos = seq_block_scan(cnt, wsum, &tot);
+  const size_t ob = (size_t)g * k;
+  const int* og = off + (size_t)g * (C + 1);
+  for (int c = c0; c < c0 + per && c < C; ++c) {
+    if (flag[c]) {
+      ids[ob + pos] = c;
+      ss[ob + pos] = og[c];
+      se[ob + pos] = og[c + 1];
+      ++pos;
+    }
+  }
+}
+
+
 struct SelParams {
   const uint16_t* q;     // bf16 [B][Hq][128]
-  const uint16_t* cent;  // bf16 [B or 1][Hkv][C][128]
-  const int* off;        // [B or 1][Hkv][C + 1]
+  const uint16_t* cent;  // bf16 [Hkv][C][128], shared by every request
+  const int* off;        // [Hkv][C + 1]
   int B, Hq, Hkv, C, k;
-  int shared;            // 1: one centroid set per KV head for every request
-  int S;                 // CTAs per cluster
+  int S;                 // CTAs (and requests) per cluster
   int* ids;
   int* ss;
   int* se;
@@ -215,9 +424,8 @@ __device__ void topk_write(const uint32_t* key, int C, int k, int* hist, int* ws
   }
 }
 
-// QM: most queries a CTA scores (1: per-sequence centroids, kSelMaxQ: shared).
-template <int QM>
-__global__ void __launch_bounds__(kSelThreads, QM == 1 ? 2 : 1) select_kernel(const SelParams p) {
+__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams p) {
+  constexpr int QM = kSelMaxQ;  // most queries a CTA scores
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t* key = reinterpret_cast<uint32_t*>(smem + kOffKeys);
   float* qs = reinterpret_cast<float*>(smem + kOffQ);
@@ -230,24 +438,14 @@ __global__ void __launch_bounds__(kSelThreads, QM == 1 ? 2 : 1) select_kernel(co
   const int S = p.S;
   const uint32_t rank = cluster_rank();
   const int kvh = blockIdx.y, G = p.Hq / p.Hkv;
-  // the requests this cluster serves and the centroid set they share
-  int b0, nq, cset;
-  if (p.shared) {
-    b0 = blockIdx.z * S;
-    nq = min(S, p.B - b0);
-    cset = kvh;
-  } else {
-    b0 = blockIdx.z;
-    nq = 1;
-    cset = blockIdx.z * p.Hkv + kvh;
-  }
+  // the requests this cluster serves; they share KV head kvh's centroids
+  const int b0 = blockIdx.z * S, nq = min(S, p.B - b0), cset = kvh;
   const int r0 = (int)(((long long)rank * p.C) / S), r1 = (int)(((long long)(rank + 1) * p.C) / S);
   const int rows = r1 - r0;
   const int nst = (rows + kStageRows - 1) / kStageRows;
   const unsigned char* src0 =
       reinterpret_cast<const unsigned char*>(p.cent + ((size_t)cset * p.C + r0) * kHeadDim);
-  // does this CTA own a selection (and how many arrivals complete its gather)?
-  const bool owner = p.shared ? (int)rank < nq : rank == 0;
+  const bool owner = (int)rank < nq;  // this CTA owns request rank's selection
 
   auto issue = [&](int chunk) {
     const int st = chunk % kSelStages;
@@ -288,10 +486,10 @@ __global__ void __launch_bounds__(kSelThreads, QM == 1 ? 2 : 1) select_kernel(co
   for (int j = 0; j < QM; ++j)
 #pragma unroll
     for (int e = 0; e < 8; ++e) qv[j][e] = j < nq ? qs[j * kHeadDim + ch * 8 + e] : 0.f;
-  // remote key slots: the owner of query j is rank 0 (per-sequence) or rank j (shared)
+  // remote key slots: query j's owner is rank j
   uint32_t kaddr[QM];
 #pragma unroll
-  for (int j = 0; j < QM; ++j) kaddr[j] = map_to(key, p.shared ? (uint32_t)min(j, S - 1) : 0u);
+  for (int j = 0; j < QM; ++j) kaddr[j] = map_to(key, (uint32_t)min(j, S - 1));
   bool ok = true;
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   for (int chunk = 0; chunk < nst; ++chunk) {
@@ -330,7 +528,7 @@ __global__ void __launch_bounds__(kSelThreads, QM == 1 ? 2 : 1) select_kernel(co
   }
   // this CTA's keys are stored: arrive on every owner's gather barrier
   __syncthreads();
-  if (tid < (p.shared ? nq : 1)) arrive_remote(map_to(&bar[kSelStages], (uint32_t)tid));
+  if (tid < nq) arrive_remote(map_to(&bar[kSelStages], (uint32_t)tid));
   if (!owner) return;  // (nothing reads this CTA's shared memory)
 
   bool got = false;
@@ -339,7 +537,7 @@ __global__ void __launch_bounds__(kSelThreads, QM == 1 ? 2 : 1) select_kernel(co
     while (!(got = try_wait_acq_cluster(&bar[kSelStages], 0)))
       if (globaltimer() - t0 > 4 * kWaitLimitNs) break;
   }
-  const int b = p.shared ? b0 + (int)rank : b0;
+  const int b = b0 + (int)rank;
   const size_t ob = ((size_t)b * p.Hkv + kvh) * p.k;
   const int* og = p.off + (size_t)cset * (p.C + 1);
   if (!ok || !got) {  // a bounded wait expired: no selection (empty ranges)
@@ -355,19 +553,25 @@ __global__ void __launch_bounds__(kSelThreads, QM == 1 ? 2 : 1) select_kernel(co
 
 }  // namespace
 
-// CTAs per cluster: per-sequence centroids split over enough CTAs to fill the
-// GPU about twice (at most 8, at least ~32 rows each); shared centroids take
-// up to 8 requests per cluster.
-int select_cluster_size(int groups_or_B, int C, int shared) {
-  if (shared) return groups_or_B < kSelMaxQ ? (groups_or_B < 1 ? 1 : groups_or_B) : kSelMaxQ;
-  int S = (2 * num_sms()) / (groups_or_B > 0 ? groups_or_B : 1);
-  S = S < 1 ? 1 : (S > 8 ? 8 : S);
-  while (S > 1 && C / S < 32) --S;
-  return S;
-}
+// Requests (and CTAs) per cluster of the shared-centroid kernel: up to 8.
+int select_cluster_size(int B) { return B < 1 ? 1 : (B < kSelMaxQ ? B : kSelMaxQ); }
 
 int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B, int Hq, int Hkv,
                   int C, int k, int shared, int* ids, int* ss, int* se, void* stream) {
+  static std::atomic<bool> attr_set[64][2];  // per device; racing first calls only repeat the set-up
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
+  if (!shared) {  // one CTA per KV group
+    if (!attr_set[dev][0]) {
+      cudaError_t e = cudaFuncSetAttribute(select_seq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kSeqSmem);
+      if (e != cudaSuccess) return (int)e;
+      attr_set[dev][0] = true;
+    }
+    select_seq_kernel<<<B * Hkv, kSeqThreads, kSeqSmem, static_cast<cudaStream_t>(stream)>>>(
+        q, cent, off, Hq, Hkv, C, k, ids, ss, se);
+    return (int)cudaGetLastError();
+  }
   SelParams p{};
   p.q = q;
   p.cent = cent;
@@ -377,22 +581,18 @@ int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B
   p.Hkv = Hkv;
   p.C = C;
   p.k = k;
-  p.shared = shared;
-  p.S = select_cluster_size(shared ? B : B * Hkv, C, shared);
+  p.S = select_cluster_size(B);
   p.ids = ids;
   p.ss = ss;
   p.se = se;
-  static std::atomic<bool> attr_set[64][2];  // per device; racing first calls only repeat the set-up
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
-  auto kern = shared ? select_kernel<kSelMaxQ> : select_kernel<1>;
-  if (!attr_set[dev][shared ? 1 : 0]) {
+  auto kern = select_kernel;
+  if (!attr_set[dev][1]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelSmem);
     if (e != cudaSuccess) return (int)e;
-    attr_set[dev][shared ? 1 : 0] = true;
+    attr_set[dev][1] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.S, Hkv, shared ? (B + p.S - 1) / p.S : B);
+  cfg.gridDim = dim3(p.S, Hkv, (B + p.S - 1) / p.S);
   cfg.blockDim = dim3(kSelThreads, 1, 1);
   cfg.dynamicSmemBytes = kSelSmem;
   cfg.stream = static_cast<cudaStream_t>(stream);

@@ -75,8 +75,8 @@ def test_shared_selection_and_attention(B, L, c_log2, topk):
 
 
 def test_per_sequence_selection_cluster_split_matches_oracle():
-    """The per-sequence call splits each group's centroids over a cluster of
-    CTAs; batches of different size get different splits (1 to 8 CTAs)."""
+    """The per-sequence call (one CTA per KV group) over 1 to 320 groups and
+    256 to 4096 clusters, with top-k from 7 to 300."""
     import torch
     import sparse_kv_b200 as skv
     for B, Hkv, c_log2, topk in [(1, 1, 12, 300), (2, 8, 10, 102), (40, 8, 8, 7)]:
