@@ -102,35 +102,6 @@ struct Trav {
     }
   }
 
-  // Segment lists: the next piece = up to 64 consecutive tokens inside one
-  // page (page, first row, rows).  Used to pack several segments into one tile.
-  __device__ bool next_piece(int& page, int& r0, int& cnt, uint32_t* status) {
-    while (true) {
-      if (seg_pos >= seg_stop) {
-        if (seg_i >= seg_end_i) return false;
-        const int s = ss[seg_i], t = se[seg_i];
-        ++seg_i;
-        if (s > t) {
-          dev_error(status, SKV_DEV_BAD_SEGMENT);
-          continue;
-        }
-        seg_pos = max(s, 0);
-        seg_stop = min(t, L);
-        continue;
-      }
-      const int blk = seg_pos / kBlock;
-      r0 = seg_pos % kBlock;
-      cnt = min(kBlock - r0, seg_stop - seg_pos);
-      seg_pos += cnt;
-      page = bt[blk];
-      if (page < 0 || page >= num_pages) {
-        dev_error(status, SKV_DEV_BAD_PAGE);
-        continue;
-      }
-      return true;
-    }
-  }
-
   __device__ bool next(int& t0, int& n, int& pg1, int& pg2, int& n1, uint32_t* status) {
     while (true) {
       int a, e;
@@ -332,7 +303,10 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
         for (int b = lane; b <= p.B; b += 32) p.ws_hdr[1 + b] = pre[b];
       }
     }
-    if (lane != 0) return;
+    // Segment lists on the split schedule keep the whole warp: it resolves
+    // segments 32 at a time (below); elsewhere lane 0 alone produces.
+    const bool warp_segments = p.sched == SCHED_SPLIT && p.mode == TRAV_SEGMENTS;
+    if (!warp_segments && lane != 0) return;
 
     const uint64_t pol = policy_evict_first();
     const size_t head_stride = (size_t)kBlock * kHeadDim;
@@ -384,10 +358,7 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       }
       return true;
     };
-    // Segment lists: rows of several segments are packed into full 64-row
-    // tiles (attention over a key set does not depend on the keys' order);
-    // one bulk copy per piece (<= 64 consecutive tokens of one page).
-    constexpr int kMaxPieces = 8;
+    constexpr int kMaxPieces = 8;  // bulk copies (pieces) packed into one ring entry
     auto emit_packed = [&](int n, const int* pg, const int* r0, const int* cnt, int np, int g,
                            int slot, int kvh) -> bool {
       if (e == withhold) return false;
@@ -424,38 +395,98 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       }
       return true;
     };
-    auto run_segments = [&](Trav& tr, int g, int slot, int kvh) -> bool {
+    // Segment lists: rows of several segments are packed into full 64-row
+    // tiles (attention over a key set does not depend on the keys' order),
+    // one bulk copy per piece (<= 64 consecutive tokens of one page).  The
+    // segments are resolved by the whole warp, 32 at a time: lane i loads segment i's bounds and the pages of its first two
+    // blocks (independent loads, one round trip for the batch) into shared
+    // memory, and lane 0 then issues the copies without waiting on global
+    // memory (a segment reaching past two blocks loads its further pages as it
+    // goes).  Called by every lane; returns lane 0's verdict on all lanes.
+    auto run_segments_warp = [&](Trav& tr, int g, int slot, int kvh) -> bool {
+      int4* stage = reinterpret_cast<int4*>(smem + C::OFF_PRE);  // [32] {start, stop, page0, page1}
       int pg[kMaxPieces], r0[kMaxPieces], cnt[kMaxPieces];
       int np = 0, rows = 0, tiles = 0;
-      int page = 0, first = 0, c = 0;
-      while (tr.next_piece(page, first, c, p.status)) {
-        while (c > 0) {
-          const int take = min(c, kBlock - rows);
-          pg[np] = page;
-          r0[np] = first;
-          cnt[np] = take;
-          ++np;
-          rows += take;
-          first += take;
-          c -= take;
-          if (rows == kBlock || np == kMaxPieces) {
-            if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
-            ++tiles;
-            np = rows = 0;
+      bool good = true;
+      for (int base = tr.seg_i; base < tr.seg_end_i; base += 32) {
+        const int i = base + lane;
+        int4 v = make_int4(0, 0, -1, -1);
+        if (i < tr.seg_end_i) {
+          int a = tr.ss[i], t = tr.se[i];
+          if (a > t) {
+            dev_error(p.status, SKV_DEV_BAD_SEGMENT);
+            a = t = 0;
+          }
+          a = max(a, 0);
+          t = min(t, tr.L);
+          if (t > a) {
+            const int b0 = a / kBlock;
+            int p0 = tr.bt[b0], p1 = -1;
+            if ((t - 1) / kBlock > b0) p1 = tr.bt[b0 + 1];
+            if (p0 < 0 || p0 >= tr.num_pages) {
+              dev_error(p.status, SKV_DEV_BAD_PAGE);
+              p0 = -1;
+            }
+            if ((t - 1) / kBlock > b0 && (p1 < 0 || p1 >= tr.num_pages)) {
+              dev_error(p.status, SKV_DEV_BAD_PAGE);
+              p1 = -1;
+            }
+            v = make_int4(a, t, p0, p1);
           }
         }
+        __syncwarp();  // lane 0 is done with the previous batch
+        stage[lane] = v;
+        __syncwarp();
+        if (lane == 0) {
+          const int nseg = min(32, tr.seg_end_i - base);
+          for (int k2 = 0; k2 < nseg && good; ++k2) {
+            const int4 sv = stage[k2];
+            const int b0 = sv.x / kBlock;
+            for (int pos = sv.x; pos < sv.y && good;) {
+              const int blk = pos / kBlock, first = pos % kBlock;
+              const int c = min(kBlock - first, sv.y - pos);
+              pos += c;
+              int page = blk == b0 ? sv.z : blk == b0 + 1 ? sv.w : tr.bt[blk];
+              if (blk > b0 + 1 && (page < 0 || page >= tr.num_pages)) {
+                dev_error(p.status, SKV_DEV_BAD_PAGE);
+                page = -1;
+              }
+              if (page < 0) continue;  // (flagged)
+              for (int f = first, left = c; left > 0;) {
+                const int take = min(left, kBlock - rows);
+                pg[np] = page;
+                r0[np] = f;
+                cnt[np] = take;
+                ++np;
+                rows += take;
+                f += take;
+                left -= take;
+                if (rows == kBlock || np == kMaxPieces) {
+                  if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) {
+                    good = false;
+                    break;
+                  }
+                  ++tiles;
+                  np = rows = 0;
+                }
+              }
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, good, 0)) return false;
       }
-      if (rows > 0) {
-        if (!emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) return false;
-        ++tiles;
+      if (lane == 0) {
+        if (rows > 0) {
+          if (emit_packed(rows, pg, r0, cnt, np, g, slot, kvh)) ++tiles;
+          else good = false;
+        }
+        if (good && tiles == 0 && !emit(0, g, slot, kvh, 0, 0, 0, 0)) good = false;
       }
-      if (tiles == 0 && !emit(0, g, slot, kvh, 0, 0, 0, 0)) return false;
-      return true;
+      return __shfl_sync(0xffffffffu, good, 0);
     };
     // All entries of one group segment; a segment without valid tiles still
     // issues a marker so that the consumers account for the group.
     auto run_group = [&](Trav& tr, int g, int slot, int kvh) -> bool {
-      if (tr.mode == TRAV_SEGMENTS) return run_segments(tr, g, slot, kvh);
       int t0 = 0, n = 0, pg1 = 0, pg2 = 0, n1 = 0, cnt = 0;
       while (tr.next(t0, n, pg1, pg2, n1, p.status)) {
         if (!emit(n, g, slot, kvh, t0, pg1, pg2, n1)) return false;
@@ -499,7 +530,12 @@ __global__ void __launch_bounds__(Cfg<G, NW, MINB>::THREADS, MINB) decode_kernel
       Trav tr;
       tr.init(p, b, kvh, L, split);
       const int g = b * p.Hkv + kvh;
-      ok = run_group(tr, g, g * p.n_splits + split, kvh);
+      if (warp_segments) {
+        ok = run_segments_warp(tr, g, g * p.n_splits + split, kvh);
+        if (lane != 0) return;
+      } else {
+        ok = run_group(tr, g, g * p.n_splits + split, kvh);
+      }
     }
     if (ok) emit(-1, -1, 0, 0, 0, 0, 0, 0);
     // Copies the consumers never waited for (abort) must land before the CTA
