@@ -344,6 +344,12 @@ def test_status_of_word_maps_device_bits():
     assert skv.status_of_word(B["timeout"]) == skv.SKV_ETIMEOUT
     for k in ("bad_page", "bad_seqlen", "bad_order", "bad_segment"):
         assert skv.status_of_word(B[k]) == skv.SKV_EINVAL
+    # the binding's bits are the header's SKV_DEV_* values
+    import re
+    hdr = open(os.path.join(ROOT, "include", "sparsekv.h")).read()
+    found = {m.group(1).lower(): int(m.group(2), 16)
+             for m in re.finditer(r"#define SKV_DEV_(\w+) (0x[0-9a-fA-F]+)u", hdr)}
+    assert found == B
     # a timeout outranks bad-input bits: the outputs are not valid at all
     assert skv.status_of_word(B["timeout"] | B["bad_page"]) == skv.SKV_ETIMEOUT
     assert skv.strerror(skv.SKV_ETIMEOUT) == "device wait timed out"

@@ -221,6 +221,39 @@ def test_token_segments_unaligned():
             check_close(res[0][b, hs], res[1][b, hs], O[0], lse[0])
 
 
+def test_token_segments_many():
+    # long segment lists (420 per group: the producer warp resolves them in
+    # batches of 32), segments of 1 to 300 tokens (some over more than two
+    # pages), empty ones, and ones past seq_len
+    torch = _torch()
+    lens = [20000, 13001, 700]
+    wl = skvgen.Workload("sp", B=3, Hq=8, Hkv=2, L=max(lens), lens=lens, paging="perm", seed=41)
+    dev = device_workload(wl)
+    n_seg = 420
+    rng = np.random.default_rng(5)
+    ss = np.zeros((3, 2, n_seg), dtype=np.int32)
+    se = np.zeros((3, 2, n_seg), dtype=np.int32)
+    for b in range(3):
+        for h in range(2):
+            pos = 0
+            for i in range(n_seg):
+                gap = int(rng.integers(0, 40))
+                ln = int(rng.choice([0, 1, 5, 63, 64, 65, 130, 300]))
+                ss[b, h, i] = pos + gap
+                se[b, h, i] = pos + gap + ln
+                pos = se[b, h, i]
+    res = run_decode(wl, dev, segments=(torch.tensor(ss, device="cuda"), torch.tensor(se, device="cuda")))
+    assert res[3] == 0
+    q = skvgen.host_q(wl)
+    for b in range(3):
+        for kvh in range(2):
+            keys = oracle.keys_segments(np.minimum(ss[b, kvh], lens[b]), np.minimum(se[b, kvh], lens[b]))
+            assert len(keys) > 0
+            O, lse_o = oracle_keys_attend(wl, b, kvh, keys, q=q)
+            hs = slice(kvh * 4, kvh * 4 + 4)
+            check_close(res[0][b, hs], res[1][b, hs], O[0], lse_o[0], f"group ({b},{kvh})")
+
+
 # ----------------------------------------------------------------------------- ART
 
 def test_art_zero_thresholds_is_full_attention():
