@@ -180,6 +180,15 @@ __global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t*
   }
   __syncthreads();
 
+  // the token ranges of this thread's clusters, loaded while the selection runs
+  const int per = (C + kSeqThreads - 1) / kSeqThreads;  // clusters per thread (<= 8)
+  const int c0 = tid * per;
+  const int* og = off + (size_t)g * (C + 1);
+  int tok[kSeqMaxClusters / kSeqThreads + 1];
+#pragma unroll
+  for (int i = 0; i <= kSeqMaxClusters / kSeqThreads; ++i)
+    tok[i] = (i <= per && c0 + i <= C) ? og[c0 + i] : 0;
+
   // ---- radix select: the k-th largest key T, 8 bits at a time from the top
   uint32_t prefix = 0, pmask = 0;
   int kk = k;  // rank still to find below the fixed prefix
@@ -226,8 +235,6 @@ __global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t*
   const uint32_t T = prefix;  // the k-th largest key; kk of the keys equal to T are taken
 
   // ---- flags: keys above T, plus the first kk keys equal to T in index order
-  const int per = (C + kSeqThreads - 1) / kSeqThreads;
-  const int c0 = tid * per;
   int nties = 0;
   for (int c = c0; c < c0 + per && c < C; ++c) nties += (key[c] == T);
   int tot = 0;
@@ -244,12 +251,13 @@ __global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t*
   // ---- compact in ascending id order
   int pos = seq_block_scan(cnt, wsum, &tot);
   const size_t ob = (size_t)g * k;
-  const int* og = off + (size_t)g * (C + 1);
-  for (int c = c0; c < c0 + per && c < C; ++c) {
-    if (flag[c]) {
+#pragma unroll
+  for (int i = 0; i < kSeqMaxClusters / kSeqThreads; ++i) {
+    const int c = c0 + i;
+    if (i < per && c < C && flag[c]) {
       ids[ob + pos] = c;
-      ss[ob + pos] = og[c];
-      se[ob + pos] = og[c + 1];
+      ss[ob + pos] = tok[i];
+      se[ob + pos] = tok[i + 1];
       ++pos;
     }
   }
