@@ -72,8 +72,9 @@ namespace {
 constexpr int kProbeFloats = 12;  // per (block, warp, head): m, l, pad, pad, O[0:8]
 constexpr int kReqs = 32;         // re-run requests in flight (a few chunks' worth)
 enum PostKind : int { POST_END = 1, POST_FIX = 2, POST_QUIT = 3, POST_DONE = 4 };
-// ring entry tags (meta.w): block in chunk (bits 0..7), request slot (8..15), last
-// chunk of the group, last tile of the chunk, re-fold flag
+// ring entry tags (meta.w): block in chunk (bits 0..7), request slot (8..15), first
+// entry of an item, last chunk of the group, last tile of the chunk, re-fold flag
+constexpr int kFirstTag = 1 << 27;
 constexpr int kLastChunkTag = 1 << 28;
 constexpr int kLastTag = 1 << 29;
 constexpr int kFixTag = 1 << 30;
@@ -271,13 +272,14 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         if (!((vm >> t) & 1u)) continue;
         const int nt = __shfl_sync(0xffffffffu, n, t), pgt = __shfl_sync(0xffffffffu, page, t);
         int r1 = 1;
-        if (lane == 0) r1 = emit(nt, g, c, kFixTag | (slot << 8) | t, pgt, kvh, first ? qsrc : nullptr);
+        if (lane == 0)
+          r1 = emit(nt, g, c, kFixTag | (slot << 8) | t | (first ? kFirstTag : 0), pgt, kvh, first ? qsrc : nullptr);
         ok = __shfl_sync(0xffffffffu, r1, 0) != 0;
         first = false;
       }
       if (ok) {
         int r1 = 1;
-        if (lane == 0) r1 = emit(0, g, c, kFixTag | (slot << 8), 0, 0, nullptr);
+        if (lane == 0) r1 = emit(0, g, c, kFixTag | (slot << 8) | (first ? kFirstTag : 0), 0, 0, nullptr);
         ok = __shfl_sync(0xffffffffu, r1, 0) != 0;
       }
     };
@@ -398,7 +400,7 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
         const int b = cur.g / p.Hkv;
         const uint16_t* qsrc = p.q + ((size_t)b * p.Hq + (size_t)cur.kvh * G) * kHeadDim;
         const int last = cur.vm ? 31 - __clz(cur.vm) : -1;
-        bool cut = false;
+        bool cut = false, any = false;  // (any: an entry of the item was issued)
         int sc_ahead = 0;  // lane 0: the group's stop chunk, loaded a tile before it is checked
         for (int i = 0; i < cur.npos && ok; ++i) {
           if (!((cur.vm >> i) & 1u)) continue;
@@ -411,14 +413,16 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
           const int ni = __shfl_sync(0xffffffffu, cur.n, i), pgi = __shfl_sync(0xffffffffu, cur.page, i);
           int r = 1;
           if (lane == 0)
-            r = emit(ni, cur.g, cur.c, i | (i == last ? kLastTag | cur.lastc : 0), pgi, cur.kvh,
-                     (cur.vm & ((1u << i) - 1u)) ? nullptr : qsrc);
+            r = emit(ni, cur.g, cur.c, i | (i == last ? kLastTag | cur.lastc : 0) | (any ? 0 : kFirstTag),
+                     pgi, cur.kvh, any ? nullptr : qsrc);
+          any = true;
           ok = __shfl_sync(0xffffffffu, r, 0) != 0;
           prefetch();
         }
         if (ok && (cut || last < 0)) {  // no tile carried the end of the chunk
           int r = 1;
-          if (lane == 0) r = emit(0, cur.g, cur.c, cur.npos | cur.lastc, 0, 0, nullptr);
+          // (the item's first entry when no tile was issued)
+          if (lane == 0) r = emit(0, cur.g, cur.c, cur.npos | cur.lastc | (any ? 0 : kFirstTag), 0, 0, nullptr);
           ok = __shfl_sync(0xffffffffu, r, 0) != 0;
         }
       }
@@ -791,12 +795,9 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
   float2* abuf = reinterpret_cast<float2*>(smem + C::OFF_A) + warp * G;
   // Warp-uniform counters used at chunk boundaries live in shared memory (one
   // block per warp): the fold loop is register-bound.
-  enum { W_KP = 0, W_CURG, W_CURC, W_CURK };
+  enum { W_KP = 0 };
   volatile int* wc = reinterpret_cast<volatile int*>(smem + C::OFF_WCTL) + warp * 8;
   wc[W_KP] = 0;      // posts made
-  wc[W_CURG] = -1;   // item being folded: group, chunk, re-fold slot (-1: the chunk itself)
-  wc[W_CURC] = -1;
-  wc[W_CURK] = -1;
   int kpar = 0;  // buffer of the next post (it holds the current item)
   bool ok = true;
 
@@ -869,12 +870,9 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     }
     const bool fix = (mt.w & kFixTag) != 0;
     const int slot = fix ? ((mt.w >> 8) & 0xFF) : -1;
-    if (mt.y != wc[W_CURG] || mt.z != wc[W_CURC] || slot != wc[W_CURK]) {
+    if (mt.w & kFirstTag) {
       // a new item (a chunk, or the re-fold of one): take the next post's buffers
       acquire();
-      wc[W_CURG] = mt.y;
-      wc[W_CURC] = mt.z;
-      wc[W_CURK] = slot;
       W.reset();
       if (n > 0)  // an item's first block carries the group's q rows
         W.load_q(reinterpret_cast<const uint16_t*>(smem + s * C::STAGE_BYTES + 2 * kTileBytes), 0,
@@ -902,22 +900,25 @@ __global__ void __launch_bounds__(ArtCfg<G, NW, CB, ST>::THREADS, MINB) art_kern
     release();
     const int pos = mt.w & 0xFF;
     if (!fix) {
-      // this warp's running state after block `pos` of the chunk
+      // this warp's running state after block `pos` of the chunk (32-bit offsets:
+      // the probes of every post together are far below 2^31 floats; the
+      // per-head offsets are constants)
       vmask |= 1u << pos;
-      float* pw = probe + (size_t)kpar * probe_floats<G, NW, CB>() +
-                  ((size_t)pos * NW + warp) * G * kProbeFloats;
+      float* pw = probe + (uint32_t)(kpar * (int)probe_floats<G, NW, CB>() +
+                                     (pos * NW + warp) * (G * kProbeFloats));
       if (W.owner) {
 #pragma unroll
         for (int j = 0; j < Lanes<G, NW>::VPL; ++j)
           *reinterpret_cast<float2*>(pw + W.hd[j] * kProbeFloats) = make_float2(W.m_st[j], W.l_st[j]);
       }
       if (lane < 2) {
+        float* px = pw + 4 + lane * 4;
 #pragma unroll
         for (int g2 = 0; g2 < G; ++g2) {
           float x0, x1, x2, x3;
           unpack2(W.acc[g2][0], x0, x1);
           unpack2(W.acc[g2][1], x2, x3);
-          *reinterpret_cast<float4*>(pw + g2 * kProbeFloats + 4 + lane * 4) = make_float4(x0, x1, x2, x3);
+          *reinterpret_cast<float4*>(px + g2 * kProbeFloats) = make_float4(x0, x1, x2, x3);
         }
       }
       if (mt.w & kLastTag) {  // the chunk's last tile: post the chunk
