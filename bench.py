@@ -71,12 +71,13 @@ def peaks():
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML every few ms in a
-    background thread while the timed region runs (read-only queries)."""
+    """Samples SM clock and clock-event reasons through NVML every millisecond
+    in a background thread while the timed region runs (read-only queries; a
+    short timed region still yields several samples)."""
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, uuid, period_s=0.005):
+    def __init__(self, uuid, period_s=0.001):
         self.uuid, self.period = uuid, period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.ok = False
