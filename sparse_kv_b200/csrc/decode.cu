@@ -52,7 +52,7 @@ struct Trav {
   // segments
   const int* ss;
   const int* se;
-  int seg_i, seg_end_i, seg_pos, seg_stop;
+  int seg_i, seg_end_i;  // (walked by the producer warp, run_segments_warp)
 
   // Whole traversal of group (b, kvh), then narrowed with set_range
   // (index-based modes: tile indices; segments: segment indices).
@@ -63,7 +63,6 @@ struct Trav {
     bt = p.block_table + (size_t)b * p.max_blocks;
     num_pages = p.num_pages;
     ord = nullptr;
-    seg_pos = seg_stop = 0;
     const int grp = b * p.Hkv + kvh;
     int N = 0;
     if (mode == TRAV_NATURAL) {
@@ -95,33 +94,18 @@ struct Trav {
     if (mode == TRAV_SEGMENTS) {
       seg_i = lo;
       seg_end_i = hi;
-      seg_pos = seg_stop = 0;
     } else {
       i = lo;
       i_end = hi;
     }
   }
 
+  // Index-based modes (segment lists take the split schedule, whose producer
+  // warp packs them: run_segments_warp).
   __device__ bool next(int& t0, int& n, int& pg1, int& pg2, int& n1, uint32_t* status) {
     while (true) {
       int a, e;
-      if (mode == TRAV_SEGMENTS) {
-        if (seg_pos >= seg_stop) {
-          if (seg_i >= seg_end_i) return false;
-          int s = ss[seg_i], t = se[seg_i];
-          ++seg_i;
-          if (s > t) {
-            dev_error(status, SKV_DEV_BAD_SEGMENT);
-            continue;
-          }
-          seg_pos = max(s, 0);
-          seg_stop = min(t, L);
-          continue;
-        }
-        a = seg_pos;
-        e = min(seg_pos + kBlock, seg_stop);
-        seg_pos = e;
-      } else if (mode == TRAV_ORDER) {
+      if (mode == TRAV_ORDER) {
         if (i >= i_end) return false;
         const int j = ord[i++];
         if (j < 0 || j >= nb) {
