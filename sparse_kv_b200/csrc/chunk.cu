@@ -58,9 +58,9 @@ constexpr size_t OFF_Q = 0;
 constexpr size_t OFF_K = OFF_Q + (size_t)kTile;      // K stage s at +s*kTile
 constexpr size_t OFF_V = OFF_K + (size_t)kStages * kTile;  // V stage s at +s*kTile
 constexpr size_t OFF_BAR = OFF_V + (size_t)kStages * kTile;
-// k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full, o_done[2],
+// k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done[2],
 // xbar[4] (one per softmax warp pair)
-constexpr int NBAR = 17;
+constexpr int NBAR = 18;
 constexpr size_t OFF_XCH = OFF_BAR + NBAR * 8;       // float [2 parity][2 halves][128 rows]
 constexpr size_t OFF_TMEM = OFF_XCH + 2 * 2 * BM * 4;
 constexpr size_t OFF_FLAG = OFF_TMEM + 16;
@@ -231,9 +231,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* v_full = bar + 4;
   uint64_t* v_empty = bar + 6;
   uint64_t* s_full = bar + 8;
+  // [2]: every softmax thread has written its P row of the tiles with j & 1 == b
+  // (one barrier per parity: Q K^T(j + 1) is issued before P V(j), so a warp can
+  // reach tile j + 1 and arrive for it while another still works on tile j)
   uint64_t* p_full = bar + 10;
-  uint64_t* o_done = bar + 11;  // [2]: P.V of tiles with j & 1 == b
-  uint64_t* xbar = bar + 13;    // [4]: the two softmax warps of a TMEM lane quarter
+  uint64_t* o_done = bar + 12;  // [2]: P.V of tiles with j & 1 == b
+  uint64_t* xbar = bar + 14;    // [4]: the two softmax warps of a TMEM lane quarter
   volatile float* xch = reinterpret_cast<volatile float*>(smem + OFF_XCH);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
@@ -271,7 +274,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     }
     mbar_init(&s_full[0], 1);    // tcgen05.commit after Q K^T
     mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 256);      // every softmax thread has written its half P row
+    mbar_init(&p_full[0], 256);  // every softmax thread has written its half P row
+    mbar_init(&p_full[1], 256);
     mbar_init(&o_done[0], 1);    // tcgen05.commit after P V of even tiles
     mbar_init(&o_done[1], 1);    // ... and of odd tiles
     for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);  // one arrival per warp of the pair
@@ -382,7 +386,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       bool ok = issue_qk(0);
       for (int j = 0; ok && j < n_tiles; ++j) {
         if (j + 1 < n_tiles && !issue_qk(j + 1)) { ok = false; break; }
-        if (!mbar_wait_bounded(p_full, j & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
         if (!mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
         fence_after_sync();
         const uint32_t v_addr = smem_u32(smem + OFF_V + (size_t)(j & 1) * kTile);
@@ -549,7 +553,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       }
       fence_async_smem();
       fence_before_sync();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
       o_live = true;
     }
     // ---- epilogue: combine the two halves' (m, l, O) of this row
