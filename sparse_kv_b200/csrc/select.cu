@@ -5,7 +5,11 @@
 // The query heads of a GQA group are summed once (one selection per KV
 // group), and score_c = qsum . centroid_c.  The kept clusters are the k best
 // scores, ties to the lower index, written in ascending id order with their
-// key ranges.
+// key ranges.  Per-sequence centroids (attn_select_centroids): a CTA pair
+// (cluster of 2) per KV group, each CTA bulk-copying and scoring half of the
+// group's centroid rows (an SM's copy throughput, not DRAM, bounds the
+// scoring at one CTA per group) and storing the keys into the first CTA's
+// shared memory, which then selects.
 //
 // Shared centroids (attn_select_centroids_shared): a thread-block cluster of S
 // CTAs shares the centroid rows of one KV head: CTA r bulk-copies rows
@@ -71,6 +75,21 @@ constexpr size_t kSeqOffScal = kSeqOffWsum + 16 * 4;
 constexpr size_t kSeqOffBar = kSeqOffScal + 16;
 constexpr size_t kSeqSmem = kSeqOffBar + kSeqStages * 8;
 
+// ---- thread-block cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // Order-preserving map of an fp32 score to an unsigned key.
 __device__ __forceinline__ uint32_t seq_score_key(float s) {
   const uint32_t u = __float_as_uint(s);
@@ -99,7 +118,7 @@ __device__ __forceinline__ int seq_block_scan(int cnt, int* wsum, int* total) {
   return base + incl - cnt;
 }
 
-__global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t* __restrict__ q,
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t* __restrict__ q,
                                                             const uint16_t* __restrict__ cent,
                                                             const int* __restrict__ off, int Hq,
                                                             int Hkv, int C, int k, int* ids, int* ss,
@@ -113,14 +132,22 @@ __global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t*
   int* scal = reinterpret_cast<int*>(smem + kSeqOffScal);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kSeqOffBar);
 
-  const int g = blockIdx.x, b = g / Hkv, kvh = g % Hkv, G = Hq / Hkv;
+  // A CTA pair per KV group: rank r scores chunks [c_begin, c_end) of the
+  // group's centroid rows (its half) and stores every key into rank 0's key
+  // array; rank 0 then selects.
+  const uint32_t rank = cluster_rank();
+  const int g = blockIdx.x >> 1, b = g / Hkv, kvh = g % Hkv, G = Hq / Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nchunks = (C + kSeqChunk - 1) / kSeqChunk;
+  const int half = (nchunks + 1) / 2;
+  const int c_begin = min(nchunks, (int)rank * half), c_end = min(nchunks, c_begin + half);
+  const int nmine = c_end - c_begin;
   const unsigned char* cg = reinterpret_cast<const unsigned char*>(cent + (size_t)g * C * kHeadDim);
 
-  // Centroid rows stream through kSeqStages shared-memory stages by bulk copy.
-  auto issue = [&](int chunk) {
-    const int st = chunk % kSeqStages;
+  // This CTA's centroid rows stream through kSeqStages shared-memory stages by
+  // bulk copy (i: this CTA's chunk count, chunk = c_begin + i).
+  auto issue = [&](int i) {
+    const int st = i % kSeqStages, chunk = c_begin + i;
     const int rows = min(kSeqChunk, C - chunk * kSeqChunk);
     const uint32_t bytes = (uint32_t)rows * kHeadDim * 2;
     mbar_arrive_expect_tx(&bar[st], bytes);
@@ -134,8 +161,10 @@ __global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t*
     fence_barrier_init();
   }
   __syncthreads();
+  // the partner runs (its shared memory exists) before the first remote store
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   if (tid == 0)
-    for (int i = 0; i < kSeqStages && i < nchunks; ++i) issue(i);
+    for (int i = 0; i < kSeqStages && i < nmine; ++i) issue(i);
 
   if (tid < kHeadDim) {
     float sum = 0.f;
@@ -145,15 +174,17 @@ __global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t*
   }
   for (int c = tid; c < C; c += kSeqThreads) flag[c] = 0;
   __syncthreads();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  const uint32_t key0 = map_to(key, 0);  // rank 0's key array
 
   // ---- scores: 16 lanes per centroid row (8 dims each), 2 rows per warp step
   const int ch = lane & 15;
   float qv[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) qv[e] = qs[ch * 8 + e];
-  for (int chunk = 0; chunk < nchunks; ++chunk) {
-    const int st = chunk % kSeqStages;
-    if (!mbar_wait_bounded(&bar[st], (chunk / kSeqStages) & 1, nullptr)) break;
+  for (int i = 0; i < nmine; ++i) {
+    const int st = i % kSeqStages, chunk = c_begin + i;
+    if (!mbar_wait_bounded(&bar[st], (i / kSeqStages) & 1, nullptr)) break;
     const unsigned char* sc = smem + (size_t)st * kSeqChunkBytes;
     const int rows = min(kSeqChunk, C - chunk * kSeqChunk);
 #pragma unroll 4
@@ -173,12 +204,17 @@ __global__ void __launch_bounds__(kSeqThreads) select_seq_kernel(const uint16_t*
       acc += __shfl_xor_sync(0xffffffffu, acc, 4);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      if (valid && ch == 0) key[chunk * kSeqChunk + r] = seq_score_key(acc);
+      if (valid && ch == 0)
+        st_cluster_u32(key0 + 4u * (uint32_t)(chunk * kSeqChunk + r), seq_score_key(acc));
     }
     __syncthreads();  // stage st fully read
-    if (tid == 0 && chunk + kSeqStages < nchunks) issue(chunk + kSeqStages);
+    if (tid == 0 && i + kSeqStages < nmine) issue(i + kSeqStages);
   }
-  __syncthreads();
+  // every key of both halves is in rank 0's array (release / acquire at
+  // cluster scope); rank 1 is done
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+  if (rank != 0) return;
 
   // the token ranges of this thread's clusters, loaded while the selection runs
   const int per = (C + kSeqThreads - 1) / kSeqThreads;  // clusters per thread (<= 8)
@@ -281,19 +317,6 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t map_to(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
 // Arrive on an mbarrier of another CTA of the cluster; release at cluster scope
 // orders this thread's earlier (remote) shared-memory stores before it.
 __device__ __forceinline__ void arrive_remote(uint32_t bar_addr) {
@@ -569,14 +592,14 @@ int launch_select(const uint16_t* q, const uint16_t* cent, const int* off, int B
   static std::atomic<bool> attr_set[64][2];  // per device; racing first calls only repeat the set-up
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
-  if (!shared) {  // one CTA per KV group
+  if (!shared) {  // a CTA pair per KV group
     if (!attr_set[dev][0]) {
       cudaError_t e = cudaFuncSetAttribute(select_seq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)kSeqSmem);
       if (e != cudaSuccess) return (int)e;
       attr_set[dev][0] = true;
     }
-    select_seq_kernel<<<B * Hkv, kSeqThreads, kSeqSmem, static_cast<cudaStream_t>(stream)>>>(
+    select_seq_kernel<<<2 * B * Hkv, kSeqThreads, kSeqSmem, static_cast<cudaStream_t>(stream)>>>(
         q, cent, off, Hq, Hkv, C, k, ids, ss, se);
     return (int)cudaGetLastError();
   }

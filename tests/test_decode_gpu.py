@@ -5,8 +5,8 @@ import pytest
 
 import oracle
 import skvgen
-from helpers import (check_art, check_close, check_selection, device_workload, group_inputs,
-                     oracle_keys_attend, outputs, run_decode)
+from helpers import (TOPK_FLAG_GAP, check_art, check_close, check_selection, check_topk_valid,
+                     device_workload, group_inputs, oracle_keys_attend, outputs, run_decode)
 
 pytestmark = pytest.mark.gpu
 
@@ -478,6 +478,38 @@ def test_select_and_attend_small_mixture():
         O, lse = oracle_keys_attend(wl, b, kvh, keys, q=q)
         hs = slice(kvh * 4, kvh * 4 + 4)
         check_close(res[0][b, hs], res[1][b, hs], O[0], lse[0])
+
+
+@pytest.mark.parametrize("C", [1, 255, 256, 257, 768, 1000, 4096])
+def test_select_pair_halves_every_chunk_count(C):
+    """The per-sequence selection splits a group's centroid rows, in chunks of
+    256, between the two CTAs of a pair: one chunk (the second CTA scores
+    nothing), a ragged last chunk, odd and even chunk counts, and the largest C.
+    Random bf16 queries and centroids; ids against the oracle's top-k."""
+    torch = _torch()
+    import sparse_kv_b200 as skv
+    B, Hq, Hkv, d = 2, 8, 2, 128
+    G, k = Hq // Hkv, min(C, 37)
+    qb = skvgen.host_normal_bf16(900 + C, skvgen.S_Q, B * Hq * d).reshape(B, Hq, d)
+    cb = skvgen.host_normal_bf16(900 + C, skvgen.S_CENTER, B * Hkv * C * d).reshape(B, Hkv, C, d)
+    off = np.ascontiguousarray(np.broadcast_to(np.arange(C + 1, dtype=np.int32) * 5, (B, Hkv, C + 1)))
+
+    def as_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+    ids = torch.empty((B, Hkv, k), dtype=torch.int32, device="cuda")
+    ss, se = torch.empty_like(ids), torch.empty_like(ids)
+    skv.attn_select_centroids(as_bf16(qb), as_bf16(cb), torch.from_numpy(off).cuda(), k, ids, ss, se)
+    torch.cuda.synchronize()
+    ids_h = ids.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            want, sc = oracle.select(qb[b, h * G:(h + 1) * G][None], cb[b, h][None], k)
+            if not np.array_equal(want[0], ids_h[b, h]):
+                assert oracle.topk_boundary_gap(sc, k)[0] <= TOPK_FLAG_GAP, f"C={C} ({b},{h})"
+                check_topk_valid(ids_h[b, h], sc[0], k, f"C={C} ({b},{h})")
+    np.testing.assert_array_equal(ss.cpu().numpy(), np.take_along_axis(off, ids_h, axis=2))
+    np.testing.assert_array_equal(se.cpu().numpy(), np.take_along_axis(off, ids_h + 1, axis=2))
 
 
 def test_select_ties_go_to_lower_index():
