@@ -184,7 +184,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSeqThreads) select_
   for (int e = 0; e < 8; ++e) qv[e] = qs[ch * 8 + e];
   for (int i = 0; i < nmine; ++i) {
     const int st = i % kSeqStages, chunk = c_begin + i;
-    if (!mbar_wait_bounded(&bar[st], (i / kSeqStages) & 1, nullptr)) break;
+    // an expired wait ends the loop for the whole CTA at once (block barriers follow)
+    if (__syncthreads_or(!mbar_wait_bounded(&bar[st], (i / kSeqStages) & 1, nullptr))) break;
     const unsigned char* sc = smem + (size_t)st * kSeqChunkBytes;
     const int rows = min(kSeqChunk, C - chunk * kSeqChunk);
 #pragma unroll 4
@@ -525,7 +526,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams 
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   for (int chunk = 0; chunk < nst; ++chunk) {
     const int st = chunk % kSelStages;
-    if (!mbar_wait_bounded(&bar[st], (chunk / kSelStages) & 1, nullptr)) {
+    // an expired wait ends the loop for the whole CTA at once (block barriers follow)
+    if (__syncthreads_or(!mbar_wait_bounded(&bar[st], (chunk / kSelStages) & 1, nullptr))) {
       ok = false;
       break;
     }
