@@ -362,14 +362,17 @@ def build_select_shared(torch, skv, skvgen, wl, status):
     return step
 
 
-def build_lookahead(torch, skv, skvgen, wl, status, n_ctas=64):
+def build_lookahead(torch, skv, skvgen, wl, status, n_ctas=20):
     """Lookahead prefetch ("SparDA" 2) on a pair of cfg5-shaped layers: layer
     l is a full-attention layer whose cache is on the GPU (ART, as the routed
     stack runs it); layer l+1 keeps its KV in page-locked host memory.  Layer
     l's Forecast picks layer l+1's top-k blocks from their summaries (two small
     kernels), then the gather kernel pulls them into a device cache on a side
     stream while layer l attends on the main stream (the gather's small CTAs
-    sit beside the attention kernel's); then layer l+1 attends the cache.  Returns (overlapped step, layer-l-alone step,
+    sit beside the attention kernel's); then layer l+1 attends the cache.
+    n_ctas = 20 gather CTAs: alone they take about as long as layer l's
+    attention, and each further resident CTA slows that attention more than it
+    speeds the copy (the pair measured 0.98 ms at 20 CTAs, 1.16 ms at 64).  Returns (overlapped step, layer-l-alone step,
     prefetch-alone step, layer-(l+1)-alone step)."""
     layers = [l for l in range(wl.n_layers - 1) if skvgen.route_bit(wl.seed, l) == 1]
     l0 = layers[0]

@@ -416,8 +416,10 @@ SKV_API skv_status skv_host_device_pointer(const void* host, void** dev);
  *                  are OR-ed in and the item copies nothing
  * Its CTAs are small (64 threads, no shared memory) so that they fit on an
  * SM beside two CTAs of the decode kernels: launch it on its own stream next
- * to the attention it should overlap, with a few dozen CTAs (64 keep a PCIe
- * link busy).  Supported: head_dim 128; 16-byte aligned pools and caches. */
+ * to the attention it should overlap.  Alone, about 32 CTAs keep a PCIe link
+ * busy; beside an attention kernel each resident CTA also slows that kernel,
+ * so the fastest pair uses fewer (about 20 beside a 0.8 ms layer on B200).
+ * Supported: head_dim 128; 16-byte aligned pools and caches. */
 SKV_API skv_status attn_prefetch_blocks(const void* k_host, const void* v_host,
                                         const int32_t* block_table, const int32_t* seq_lens,
                                         const int32_t* block_ids, int batch, int kv_heads,
